@@ -1,0 +1,127 @@
+"""fp64 CPU oracle for the fused attention forward -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline / reference leg may import this package.  The CUDA library and its
+Python binding never import it, and it imports nothing from them.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, double precision, OpenMP
+over (batch, head)); this module only marshals numpy arrays through ctypes.
+Every input must already be the exact values the GPU path sees (fp16/bf16
+rounded, then widened to float64).
+
+Functions
+---------
+attn_fwd(q, k, v, causal, scale)            -> (o, lse)   definition order
+attn_fwd_blocked(q, k, v, causal, scale, block_m=128, block_n=64) -> (o, lse)
+attn_probs(q, k, causal, scale)             -> p [B, H, Nq, Nk]
+num_threads() / set_num_threads(n)
+
+Layouts: q, o [B, Nq, H, d]; k, v [B, Nk, H, d]; lse [B, H, Nq].
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_lib_path = None
+
+
+def load(path=None):
+    """Load (building first if stale) the oracle library; returns the CDLL."""
+    global _lib, _lib_path
+    path = path or _build.LIB
+    if _lib is not None and _lib_path == path:
+        return _lib
+    if path == _build.LIB and _build.needs_build():
+        _build.build()
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    i, d = ctypes.c_int, ctypes.c_double
+    lib.oracle_attn_fwd_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, d]
+    lib.oracle_attn_fwd_f64.restype = i
+    lib.oracle_attn_fwd_blocked_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i, i]
+    lib.oracle_attn_fwd_blocked_f64.restype = i
+    lib.oracle_attn_probs_f64.argtypes = [dp, dp, dp, i, i, i, i, i, i, d]
+    lib.oracle_attn_probs_f64.restype = i
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = i
+    lib.oracle_set_num_threads.argtypes = [i]
+    lib.oracle_set_num_threads.restype = None
+    if path == _build.LIB:
+        _lib, _lib_path = lib, path
+    return lib
+
+
+def _f64(x):
+    """Contiguous float64 numpy view/copy of a numpy array or CPU torch tensor."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shapes(q, k, v=None):
+    if q.ndim != 4 or k.ndim != 4:
+        raise ValueError("q and k must be [B, N, H, d]")
+    B, Nq, H, d = q.shape
+    if k.shape[0] != B or k.shape[2] != H or k.shape[3] != d:
+        raise ValueError("k must be [B, Nk, H, d] with q's B, H, d")
+    if v is not None and v.shape != k.shape:
+        raise ValueError("v must have k's shape")
+    return B, H, Nq, k.shape[1], d
+
+
+def attn_fwd(q, k, v, causal=False, scale=None, lib=None):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, Nk, d = _shapes(q, k, v)
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    o = np.zeros((B, Nq, H, d), dtype=np.float64)
+    lse = np.zeros((B, H, Nq), dtype=np.float64)
+    rc = (lib or load()).oracle_attn_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                             B, H, Nq, Nk, d, int(bool(causal)), scale)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_f64 failed ({rc})")
+    return o, lse
+
+
+def attn_fwd_blocked(q, k, v, causal=False, scale=None, block_m=128, block_n=64, lib=None):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, Nk, d = _shapes(q, k, v)
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    o = np.zeros((B, Nq, H, d), dtype=np.float64)
+    lse = np.zeros((B, H, Nq), dtype=np.float64)
+    rc = (lib or load()).oracle_attn_fwd_blocked_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                                     B, H, Nq, Nk, d, int(bool(causal)), scale,
+                                                     int(block_m), int(block_n))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_blocked_f64 failed ({rc})")
+    return o, lse
+
+
+def attn_probs(q, k, causal=False, scale=None, lib=None):
+    q, k = _f64(q), _f64(k)
+    B, H, Nq, Nk, d = _shapes(q, k)
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    p = np.zeros((B, H, Nq, Nk), dtype=np.float64)
+    rc = (lib or load()).oracle_attn_probs_f64(_ptr(q), _ptr(k), _ptr(p),
+                                               B, H, Nq, Nk, d, int(bool(causal)), scale)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_probs_f64 failed ({rc})")
+    return p
+
+
+def num_threads():
+    return load().oracle_num_threads()
+
+
+def set_num_threads(n):
+    load().oracle_set_num_threads(int(n))
+
+
+__all__ = ["attn_fwd", "attn_fwd_blocked", "attn_probs", "num_threads", "set_num_threads", "load"]

@@ -1,0 +1,249 @@
+/*
+ * Attention forward oracle -- plain, slow, fp64 CPU reference.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file: only the test suite, the smoke check and the benchmark's
+ * cpu_baseline / reference leg do.  It shares no code, header, table or helper
+ * with the CUDA library.
+ *
+ * What it computes (FlashAttention/ops-transformer article on ai6s.net,
+ * section "传统注意力的显存陷阱" -- the conventional attention definition:
+ * scores = Q K^T / sqrt(d_k), probabilities = softmax over the key axis,
+ * output = probabilities . V), generalised to an explicit scale, an optional
+ * causal mask and an fp32-style natural-log row LSE:
+ *
+ *   for every batch b, head h, query i:
+ *     allowed(i, j)  <=>  j < Nk  and (not causal or j <= i + (Nk - Nq))
+ *     s_ij  = scale * sum_t q[b,i,h,t] * k[b,j,h,t]          (allowed j only)
+ *     m_i   = max_j s_ij
+ *     p_ij  = exp(s_ij - m_i)
+ *     l_i   = sum_j p_ij
+ *     O[b,i,h,:] = sum_j p_ij v[b,j,h,:] / l_i
+ *     lse[b,h,i] = m_i + ln l_i
+ *   A row with no allowed key gives O = 0 and lse = -inf.
+ *
+ * Readings where the article is silent (each one is listed in the design
+ * notes): the scale is an explicit argument (the article divides by sqrt(d_k)
+ * and its API example passes none); a causal mask with Nq != Nk is aligned to
+ * the bottom-right corner; lse is the natural-log row LSE of the scaled,
+ * masked scores.
+ *
+ * Layouts: q, o are [B, Nq, H, d]; k, v are [B, Nk, H, d]; lse is [B, H, Nq];
+ * p (probabilities, tiny cases only) is [B, H, Nq, Nk].  Everything is double.
+ *
+ * Two orderings are provided.  oracle_attn_fwd_f64 follows the definition
+ * literally and materialises each (b, h) score matrix.  The blocked variant
+ * follows the article's "FlashAttention的核心逻辑" section: an outer loop over
+ * query blocks, an inner loop over key/value blocks, a running row maximum and
+ * row sum updated block by block (the online softmax update, written out in
+ * its standard form because the article only names it), and one
+ * normalisation after the inner loop.  Both must agree to rounding.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define IDX4(b, n, h, t, N, H, D) ((((long)(b) * (N) + (n)) * (H) + (h)) * (D) + (t))
+
+static int is_allowed(long i, long j, long Nq, long Nk, int causal)
+{
+    if (j >= Nk) return 0;
+    if (causal && j > i + (Nk - Nq)) return 0;
+    return 1;
+}
+
+static double dot_qk(const double* q, const double* k, int b, int h, long i, long j,
+                     int H, int Nq, int Nk, int d)
+{
+    double acc = 0.0;
+    const double* qi = q + IDX4(b, i, h, 0, Nq, H, d);
+    const double* kj = k + IDX4(b, j, h, 0, Nk, H, d);
+    for (int t = 0; t < d; ++t) acc += qi[t] * kj[t];
+    return acc;
+}
+
+static int check_args(int B, int H, int Nq, int Nk, int d)
+{
+    return (B > 0 && H > 0 && Nq > 0 && Nk > 0 && d > 0) ? 0 : -1;
+}
+
+/* Definition order: materialise S for one (b, h), then softmax, then P.V. */
+int oracle_attn_fwd_f64(const double* q, const double* k, const double* v,
+                        double* o, double* lse,
+                        int B, int H, int Nq, int Nk, int d, int causal, double scale)
+{
+    if (check_args(B, H, Nq, Nk, d)) return -1;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        double* S = (double*)malloc(sizeof(double) * (size_t)Nq * (size_t)Nk);
+        if (!S) {
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        /* scores, -inf where not allowed */
+        for (long i = 0; i < Nq; ++i)
+            for (long j = 0; j < Nk; ++j)
+                S[i * Nk + j] = is_allowed(i, j, Nq, Nk, causal)
+                                    ? scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d)
+                                    : -INFINITY;
+        for (long i = 0; i < Nq; ++i) {
+            double* Si = S + i * Nk;
+            double m = -INFINITY;
+            for (long j = 0; j < Nk; ++j) if (Si[j] > m) m = Si[j];
+            double* oi = o + IDX4(b, i, h, 0, Nq, H, d);
+            if (m == -INFINITY) {          /* no allowed key in this row */
+                for (int t = 0; t < d; ++t) oi[t] = 0.0;
+                lse[((long)b * H + h) * Nq + i] = -INFINITY;
+                continue;
+            }
+            double l = 0.0;
+            for (long j = 0; j < Nk; ++j) {
+                Si[j] = (Si[j] == -INFINITY) ? 0.0 : exp(Si[j] - m);   /* Si now holds p_ij */
+                l += Si[j];
+            }
+            for (int t = 0; t < d; ++t) {
+                double acc = 0.0;
+                for (long j = 0; j < Nk; ++j)
+                    if (Si[j] != 0.0) acc += Si[j] * v[IDX4(b, j, h, t, Nk, H, d)];
+                oi[t] = acc / l;
+            }
+            lse[((long)b * H + h) * Nq + i] = m + log(l);
+        }
+        free(S);
+    }
+    return err;
+}
+
+/* Row-normalised probabilities P[b,h,i,j] (masked entries are exactly 0). */
+int oracle_attn_probs_f64(const double* q, const double* k, double* p,
+                          int B, int H, int Nq, int Nk, int d, int causal, double scale)
+{
+    if (check_args(B, H, Nq, Nk, d)) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        for (long i = 0; i < Nq; ++i) {
+            double* Pi = p + (bh * Nq + i) * (long)Nk;
+            double m = -INFINITY;
+            for (long j = 0; j < Nk; ++j) {
+                Pi[j] = is_allowed(i, j, Nq, Nk, causal)
+                            ? scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d)
+                            : -INFINITY;
+                if (Pi[j] > m) m = Pi[j];
+            }
+            if (m == -INFINITY) { for (long j = 0; j < Nk; ++j) Pi[j] = 0.0; continue; }
+            double l = 0.0;
+            for (long j = 0; j < Nk; ++j) {
+                Pi[j] = (Pi[j] == -INFINITY) ? 0.0 : exp(Pi[j] - m);
+                l += Pi[j];
+            }
+            for (long j = 0; j < Nk; ++j) Pi[j] /= l;
+        }
+    }
+    return 0;
+}
+
+/*
+ * Blocked online order (the article's core-logic section): query blocks of
+ * block_m rows, key/value blocks of block_n rows.  Per query row the running
+ * state is (m, l, acc[d]); for each key block:
+ *   m' = max(m, max_j s_ij);  alpha = exp(m - m');
+ *   l  = alpha * l + sum_j exp(s_ij - m');
+ *   acc = alpha * acc + sum_j exp(s_ij - m') v_j;   m = m'
+ * and after the last block O = acc / l, lse = m + ln l.
+ */
+int oracle_attn_fwd_blocked_f64(const double* q, const double* k, const double* v,
+                                double* o, double* lse,
+                                int B, int H, int Nq, int Nk, int d, int causal, double scale,
+                                int block_m, int block_n)
+{
+    if (check_args(B, H, Nq, Nk, d) || block_m <= 0 || block_n <= 0) return -1;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        double* m = (double*)malloc(sizeof(double) * (size_t)block_m);
+        double* l = (double*)malloc(sizeof(double) * (size_t)block_m);
+        double* acc = (double*)malloc(sizeof(double) * (size_t)block_m * (size_t)d);
+        double* s = (double*)malloc(sizeof(double) * (size_t)block_n);
+        if (!m || !l || !acc || !s) {
+#pragma omp atomic write
+            err = -2;
+            free(m); free(l); free(acc); free(s);
+            continue;
+        }
+        for (long i0 = 0; i0 < Nq; i0 += block_m) {
+            const long rows = (Nq - i0 < block_m) ? (Nq - i0) : block_m;
+            for (long r = 0; r < rows; ++r) {
+                m[r] = -INFINITY;
+                l[r] = 0.0;
+                for (int t = 0; t < d; ++t) acc[r * d + t] = 0.0;
+            }
+            for (long j0 = 0; j0 < Nk; j0 += block_n) {
+                const long cols = (Nk - j0 < block_n) ? (Nk - j0) : block_n;
+                for (long r = 0; r < rows; ++r) {
+                    const long i = i0 + r;
+                    double bmax = -INFINITY;
+                    for (long c = 0; c < cols; ++c) {
+                        const long j = j0 + c;
+                        s[c] = is_allowed(i, j, Nq, Nk, causal)
+                                   ? scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d)
+                                   : -INFINITY;
+                        if (s[c] > bmax) bmax = s[c];
+                    }
+                    if (bmax == -INFINITY) continue;       /* nothing allowed in this block */
+                    const double mnew = (bmax > m[r]) ? bmax : m[r];
+                    const double alpha = (m[r] == -INFINITY) ? 0.0 : exp(m[r] - mnew);
+                    double bsum = 0.0;
+                    for (int t = 0; t < d; ++t) acc[r * d + t] *= alpha;
+                    for (long c = 0; c < cols; ++c) {
+                        if (s[c] == -INFINITY) continue;
+                        const double pc = exp(s[c] - mnew);
+                        bsum += pc;
+                        const double* vj = v + IDX4(b, j0 + c, h, 0, Nk, H, d);
+                        for (int t = 0; t < d; ++t) acc[r * d + t] += pc * vj[t];
+                    }
+                    l[r] = alpha * l[r] + bsum;
+                    m[r] = mnew;
+                }
+            }
+            for (long r = 0; r < rows; ++r) {
+                const long i = i0 + r;
+                double* oi = o + IDX4(b, i, h, 0, Nq, H, d);
+                if (l[r] == 0.0) {
+                    for (int t = 0; t < d; ++t) oi[t] = 0.0;
+                    lse[((long)b * H + h) * Nq + i] = -INFINITY;
+                } else {
+                    for (int t = 0; t < d; ++t) oi[t] = acc[r * d + t] / l[r];
+                    lse[((long)b * H + h) * Nq + i] = m[r] + log(l[r]);
+                }
+            }
+        }
+        free(m); free(l); free(acc); free(s);
+    }
+    return err;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -1,0 +1,72 @@
+"""Plant plausible mistakes in a copy of the oracle and check the pins catch them.
+
+Each mutant is the oracle's C source with one textual slip (a dropped term, a
+wrong sign, corner or index, a missing normalisation), compiled into a
+throw-away library.  The pin suite (test_oracle.py) is then run against it in a
+subprocess and must fail.  The committed oracle itself is never modified.
+"""
+import os
+import subprocess
+import sys
+import textwrap
+
+import pytest
+
+from oracle import build as obuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTANTS = {
+    "dropped_scale": [("? scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d)\n                                    : -INFINITY;\n        for (long i = 0; i < Nq; ++i) {",
+                       "? dot_qk(q, k, b, h, i, j, H, Nq, Nk, d)\n                                    : -INFINITY;\n        for (long i = 0; i < Nq; ++i) {")],
+    "top_left_mask": [("if (causal && j > i + (Nk - Nq)) return 0;", "if (causal && j > i) return 0;")],
+    "flipped_mask": [("if (causal && j > i + (Nk - Nq)) return 0;", "if (causal && j < i + (Nk - Nq)) return 0;")],
+    "no_max_in_exp": [("Si[j] = (Si[j] == -INFINITY) ? 0.0 : exp(Si[j] - m);   /* Si now holds p_ij */",
+                       "Si[j] = (Si[j] == -INFINITY) ? 0.0 : exp(Si[j]);   /* Si now holds p_ij */")],
+    "lse_without_max": [("lse[((long)b * H + h) * Nq + i] = m + log(l);\n        }\n        free(S);",
+                         "lse[((long)b * H + h) * Nq + i] = log(l);\n        }\n        free(S);")],
+    "v_column_index": [("acc += Si[j] * v[IDX4(b, j, h, t, Nk, H, d)];",
+                        "acc += Si[j] * v[IDX4(b, j, h, 0, Nk, H, d)];")],
+    "key_head_index": [("const double* kj = k + IDX4(b, j, h, 0, Nk, H, d);",
+                        "const double* kj = k + IDX4(b, j, 0, 0, Nk, H, d);")],
+    "missing_normalisation": [("oi[t] = acc / l;", "oi[t] = acc;")],
+    "blocked_l_not_rescaled": [("l[r] = alpha * l[r] + bsum;", "l[r] = l[r] + bsum;")],
+    "blocked_acc_not_rescaled": [("for (int t = 0; t < d; ++t) acc[r * d + t] *= alpha;",
+                                  "for (int t = 0; t < d; ++t) acc[r * d + t] *= 1.0;")],
+}
+
+RUNNER = textwrap.dedent("""
+    import sys
+    sys.path.insert(0, {root!r})
+    import oracle
+    from oracle import build
+    lib = oracle.load({lib!r})
+    oracle._lib, oracle._lib_path = lib, build.LIB
+    import pytest
+    sys.exit(pytest.main(["-x", "-q", "-p", "no:cacheprovider",
+                          {tests!r}]))
+""")
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    src = open(obuild.SRC).read()
+    for old, new in MUTANTS[name]:
+        assert src.count(old) == 1, f"mutation anchor for {name} not unique/present"
+        src = src.replace(old, new)
+    mpath = tmp_path / f"{name}.c"
+    mpath.write_text(src)
+    lib = obuild.build(src=str(mpath), out=str(tmp_path / f"lib{name}.so"))
+    code = RUNNER.format(root=ROOT, lib=lib, tests=os.path.join(ROOT, "tests", "test_oracle.py"))
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         cwd=str(tmp_path), timeout=600)
+    assert res.returncode != 0, f"mutant {name} survived the pin suite:\n{res.stdout[-2000:]}"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    """Control: the same harness on an unmodified copy passes."""
+    lib = obuild.build(src=obuild.SRC, out=str(tmp_path / "libcopy.so"))
+    code = RUNNER.format(root=ROOT, lib=lib, tests=os.path.join(ROOT, "tests", "test_oracle.py"))
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         cwd=str(tmp_path), timeout=600)
+    assert res.returncode == 0, res.stdout[-3000:] + res.stderr[-2000:]
