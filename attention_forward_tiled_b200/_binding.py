@@ -1,0 +1,199 @@
+"""ctypes binding of libattn.so: argument marshalling only.
+
+Every step of the attention forward runs in the CUDA kernels behind the C ABI
+(include/attn.h).  PyTorch is used for device memory and streams; there is no
+CPU or PyTorch fallback: if the library is missing or the call fails, an
+exception is raised.
+"""
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn.so")
+
+ATTN_F16, ATTN_BF16 = 0, 1
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_CUDA = -3
+ATTN_ERR_TIMEOUT = -4
+
+# every entry point declared in include/attn.h: name -> (restype, argtypes)
+_vp, _i, _f, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong
+SIGNATURES = {
+    "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "attn_fwd_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "attn_fwd_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_get_status": (_i, [_vp]),
+    "attn_error_string": (ctypes.c_char_p, [_i]),
+    "attn_version": (_i, []),
+    "attn_debug_set": (_i, [_i, _u64]),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code, where=""):
+        self.code = code
+        msg = error_string(code) if _lib is not None else f"attn status {code}"
+        super().__init__(f"{where}: {msg}" if where else msg)
+
+
+def load_library(path=LIB_PATH):
+    """Load libattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built: run `python -m attention_forward_tiled_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def error_string(code):
+    return load_library().attn_error_string(int(code)).decode()
+
+
+def version():
+    return load_library().attn_version()
+
+
+def debug_set(inject=0, wait_timeout_ns=0):
+    return load_library().attn_debug_set(int(inject), int(wait_timeout_ns))
+
+
+def _dtype_code(t):
+    import torch
+    if t == torch.float16:
+        return ATTN_F16
+    if t == torch.bfloat16:
+        return ATTN_BF16
+    raise TypeError(f"unsupported dtype {t}; expected float16 or bfloat16")
+
+
+def _check(q, k, v):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [batch, seq, heads, head_dim]")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
+    B, Nq, H, d = q.shape
+    if k.shape[0] != B or k.shape[2] != H or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Nk, H, d] with q's B, H, d")
+    return B, H, Nq, k.shape[1], d
+
+
+def _stream_ptr(stream, device):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_lse=True,
+             stream=None, path="auto", splits=0):
+    """Fused attention forward on CUDA tensors laid out [B, N, H, d].
+
+    Returns (out, lse): out [B, Nq, H, d] in q's dtype, lse [B, H, Nq] float32
+    (None when return_lse is False and no lse buffer is given).
+    path: "auto" (decode kernels when Nq == 1), "prefill" or "decode".
+    """
+    import torch
+    lib = load_library()
+    B, H, Nq, Nk, d = _check(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor like q")
+    if lse is not None and (lse.shape != (B, H, Nq) or lse.dtype != torch.float32
+                            or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [B, H, Nq] tensor")
+    dt = _dtype_code(q.dtype)
+    lse_ptr = ctypes.c_void_p(lse.data_ptr() if lse is not None else 0)
+    with torch.cuda.device(q.device):
+        s = _stream_ptr(stream, q.device)
+        ptrs = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()), lse_ptr)
+        if path == "auto":
+            rc = lib.attn_fwd(*ptrs, B, H, Nq, Nk, d, int(bool(causal)), scale, dt, s)
+        elif path == "prefill":
+            rc = lib.attn_fwd_prefill(*ptrs, B, H, Nq, Nk, d, int(bool(causal)), scale, dt, s)
+        elif path == "decode":
+            rc = lib.attn_fwd_decode(*ptrs, B, H, Nk, d, scale, dt, int(splits), s)
+        else:
+            raise ValueError(f"unknown path {path!r}")
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+    return out, lse
+
+
+def get_status(stream=None, device=None):
+    """Synchronise the stream and return (then clear) the device status word."""
+    import torch
+    lib = load_library()
+    device = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(device):
+        return lib.attn_get_status(_stream_ptr(stream, device))
+
+
+class HostRunner:
+    """End-to-end call from host buffers: H2D copies, the kernel, D2H copy of O (and lse).
+
+    Device buffers are allocated once at construction; each call copies the host
+    tensors (pinned for asynchronous copies) to them on the runner's stream,
+    runs attn_fwd and copies the results back into pinned host tensors.
+    """
+
+    def __init__(self, B, H, Nq, Nk, d, dtype, device="cuda", causal=False, scale=None,
+                 with_lse=True):
+        import torch
+        self.device = torch.device(device)
+        self.causal, self.scale = causal, scale
+        self.q = torch.empty((B, Nq, H, d), dtype=dtype, device=self.device)
+        self.k = torch.empty((B, Nk, H, d), dtype=dtype, device=self.device)
+        self.v = torch.empty_like(self.k)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, Nq), dtype=torch.float32, device=self.device) if with_lse else None
+        self.out_host = torch.empty(self.out.shape, dtype=dtype, pin_memory=True)
+        self.lse_host = (torch.empty(self.lse.shape, dtype=torch.float32, pin_memory=True)
+                         if with_lse else None)
+
+    @property
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v))
+
+    @property
+    def d2h_bytes(self):
+        n = self.out.numel() * self.out.element_size()
+        return n + (self.lse.numel() * 4 if self.lse is not None else 0)
+
+    def __call__(self, q_host, k_host, v_host, stream=None):
+        import torch
+        stream = stream or torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(stream):
+            self.q.copy_(q_host, non_blocking=True)
+            self.k.copy_(k_host, non_blocking=True)
+            self.v.copy_(v_host, non_blocking=True)
+            attn_fwd(self.q, self.k, self.v, causal=self.causal, scale=self.scale, out=self.out,
+                     lse=self.lse, stream=stream)
+            self.out_host.copy_(self.out, non_blocking=True)
+            if self.lse is not None:
+                self.lse_host.copy_(self.lse, non_blocking=True)
+        return self.out_host, self.lse_host

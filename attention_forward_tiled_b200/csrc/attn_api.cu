@@ -1,0 +1,356 @@
+// attn_api.cu -- the C ABI of libattn.so (declared in include/attn.h).
+//
+// Host side only: argument validation, tensor-map encoding for the
+// tensor-memory accelerator, launch configuration, the split-KV workspace and
+// the device status word.  Every arithmetic step of the attention forward runs
+// in the kernels of prefill_sm100.cuh and decode_sm100.cuh; there is no CPU
+// fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "attn.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+using namespace attn_b200;
+
+// Device status word: kernels record ATTN_ERR_TIMEOUT here instead of trapping.
+__device__ int g_attn_status = 0;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+constexpr int kMaxDevices = 64;
+constexpr int kHeadsPerGroup = 8;  // prefill scheduling group (K/V of 8 heads stay in L2)
+
+std::atomic<int> g_inject{0};
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  int* status_ptr = nullptr;
+  bool attr_set[8] = {};  // per kernel instantiation: max dynamic shared memory raised
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Probe the current device once: sm_100 check, SM count, status-word address.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceState& s = g_dev[dev];
+  if (!s.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    s.supported = (major == 10 && minor == 0);
+    s.sm_count = sms;
+    if (s.supported) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_attn_status) != cudaSuccess) return ATTN_ERR_CUDA;
+      s.status_ptr = static_cast<int*>(ptr);
+    }
+    s.probed = true;
+  }
+  if (!s.supported) return ATTN_ERR_UNSUPPORTED;
+  *out = &s;
+  return ATTN_OK;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename Kernel>
+int ensure_smem_attr(DeviceState* ds, int slot, Kernel kernel, int bytes) {
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (ds->attr_set[slot]) return ATTN_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  ds->attr_set[slot] = true;
+  return ATTN_OK;
+}
+
+// 4-D view (d, H, N, B) of a contiguous [B, N, H, d] tensor; box (64, 1, 128, 1), 128B swizzle.
+int encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, int dtype) {
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return ATTN_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
+                                 (cuuint64_t)N * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType ty =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = encode(map, ty, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Shared argument checks of every entry point (nothing is enqueued on failure).
+int validate(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype) {
+  if (!q || !k || !v || !out) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(out, 16))
+    return ATTN_ERR_INVALID_ARG;
+  if (lse && misaligned(lse, 4)) return ATTN_ERR_INVALID_ARG;
+  // tensor-map limits: the batch stride (N*H*d*2 bytes) must stay below 2^40
+  const unsigned long long row_bytes = (unsigned long long)H * d * 2;
+  if ((unsigned long long)Nq * row_bytes >= (1ull << 40) ||
+      (unsigned long long)Nk * row_bytes >= (1ull << 40))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = (size_t)B * Nq * row_bytes;
+  const size_t kv_bytes = (size_t)B * Nk * row_bytes;
+  const size_t lse_bytes = (size_t)B * H * Nq * sizeof(float);
+  if (overlaps(out, q_bytes, q, q_bytes) || overlaps(out, q_bytes, k, kv_bytes) ||
+      overlaps(out, q_bytes, v, kv_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  if (lse && (overlaps(lse, lse_bytes, out, q_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
+              overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes)))
+    return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+template <int D, bool BF16>
+int launch_prefill(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
+                   float* lse, int B, int H, int Nq, int Nk, int causal, float scale,
+                   cudaStream_t stream) {
+  using C = PrefillCfg<D>;
+  auto kernel = attn_prefill_kernel<D, BF16>;
+  const int slot = (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  PrefillParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  if (int rc = encode_bnhd(&p.tm_q, q, B, Nq, H, D, dtype)) return rc;
+  if (int rc = encode_bnhd(&p.tm_k, k, B, Nk, H, D, dtype)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v, B, Nk, H, D, dtype)) return rc;
+  if (int rc = encode_bnhd(&p.tm_o, out, B, Nq, H, D, dtype)) return rc;
+  p.out = out;
+  p.lse = lse;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.causal = causal;
+  p.n_qpairs = (Nq + 255) / 256;
+  p.group_heads = kHeadsPerGroup;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.inject = g_inject.load();
+  p.timeout_ns = g_timeout_ns.load();
+  const long long units = (long long)B * H * p.n_qpairs;
+  if (units >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+  kernel<<<dim3((unsigned)units), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Split count for the decode kernel: minimise the largest per-CTA tile count
+// (items are dealt round-robin to one persistent CTA per SM), preferring fewer splits.
+int choose_splits(long long BH, int ntiles, int grid) {
+  int best = 1;
+  long long best_load = -1;
+  for (int s = 1; s <= ntiles; ++s) {
+    const int tps = (ntiles + s - 1) / s;
+    const int s_eff = (ntiles + tps - 1) / tps;
+    if (s_eff != s) continue;
+    const long long items = BH * s;
+    const long long g = std::min<long long>(items, grid);
+    const long long load = ((items + g - 1) / g) * tps;
+    if (best_load < 0 || load * 100 < best_load * 98) {  // need a 2% gain to add splits
+      best = s;
+      best_load = load;
+    }
+  }
+  return best;
+}
+
+template <int D, bool BF16>
+int launch_decode(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
+                  float* lse, int B, int H, int Nk, float scale, int splits_req,
+                  cudaStream_t stream) {
+  using C = DecodeCfg<D>;
+  auto kernel = attn_decode_partial_kernel<D, BF16>;
+  const int slot = 4 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  const int ntiles = (Nk + 127) / 128;
+  const long long BH = (long long)B * H;
+  int splits = splits_req > 0 ? splits_req : choose_splits(BH, ntiles, ds->sm_count);
+  if (splits < 1 || splits > ntiles) return ATTN_ERR_INVALID_ARG;
+  const int tps = (ntiles + splits - 1) / splits;
+  splits = (ntiles + tps - 1) / tps;  // no empty split
+  const long long items = BH * splits;
+  if (items >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+
+  DecodeParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  if (int rc = encode_bnhd(&p.tm_k, k, B, Nk, H, D, dtype)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v, B, Nk, H, D, dtype)) return rc;
+  float* part = nullptr;
+  const size_t ws_bytes = (size_t)items * (D + 2) * sizeof(float);
+  if (cudaMallocAsync(reinterpret_cast<void**>(&part), ws_bytes, stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  p.q = q;
+  p.part = part;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Nk = Nk;
+  p.splits = splits;
+  p.tiles_per_split = tps;
+  p.n_items = (int)items;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  const int grid = (int)std::min<long long>(items, ds->sm_count);
+  kernel<<<dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  int rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  if (rc == ATTN_OK) {
+    attn_decode_combine_kernel<D, BF16>
+        <<<dim3((unsigned)((BH + 3) / 4)), dim3(128), 0, stream>>>(part, out, lse, (int)BH, splits);
+    rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (cudaFreeAsync(part, stream) != cudaSuccess) rc = ATTN_ERR_CUDA;
+  return rc;
+}
+
+int dispatch_prefill(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
+                     float* lse, int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                     int dtype, cudaStream_t stream) {
+  const bool bf16 = dtype == ATTN_BF16;
+  if (d == 128)
+    return bf16 ? launch_prefill<128, true>(ds, q, k, v, out, lse, B, H, Nq, Nk, causal, scale, stream)
+                : launch_prefill<128, false>(ds, q, k, v, out, lse, B, H, Nq, Nk, causal, scale, stream);
+  return bf16 ? launch_prefill<64, true>(ds, q, k, v, out, lse, B, H, Nq, Nk, causal, scale, stream)
+              : launch_prefill<64, false>(ds, q, k, v, out, lse, B, H, Nq, Nk, causal, scale, stream);
+}
+
+int dispatch_decode(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
+                    float* lse, int B, int H, int Nk, int d, float scale, int dtype, int splits,
+                    cudaStream_t stream) {
+  const bool bf16 = dtype == ATTN_BF16;
+  if (d == 128)
+    return bf16 ? launch_decode<128, true>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, stream)
+                : launch_decode<128, false>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, stream);
+  return bf16 ? launch_decode<64, true>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, stream)
+              : launch_decode<64, false>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
+                     attn_stream_t stream) {
+  if (int rc = validate(q, k, v, out, lse, B, H, Nq, Nk, d, causal, scale, dtype)) return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  return dispatch_prefill(ds, q, k, v, out, lse, B, H, Nq, Nk, d, causal, scale, dtype,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                    int H, int Nk, int d, float scale, int dtype, int splits,
+                    attn_stream_t stream) {
+  if (int rc = validate(q, k, v, out, lse, B, H, 1, Nk, d, 0, scale, dtype)) return rc;
+  if (splits < 0) return ATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  return dispatch_decode(ds, q, k, v, out, lse, B, H, Nk, d, scale, dtype, splits,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+             int Nq, int Nk, int d, int causal, float scale, int dtype, attn_stream_t stream) {
+  if (int rc = validate(q, k, v, out, lse, B, H, Nq, Nk, d, causal, scale, dtype)) return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  // One query row: under the bottom-right causal reading it sees every key, so
+  // the causal flag changes nothing and the split-KV decode path applies.
+  if (Nq == 1)
+    return dispatch_decode(ds, q, k, v, out, lse, B, H, Nk, d, scale, dtype, 0,
+                           reinterpret_cast<cudaStream_t>(stream));
+  return dispatch_prefill(ds, q, k, v, out, lse, B, H, Nq, Nk, d, causal, scale, dtype,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_get_status(attn_stream_t stream) {
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  int value = 0;
+  if (cudaMemcpy(&value, ds->status_ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(ds->status_ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return value;
+}
+
+const char* attn_error_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK: success";
+    case ATTN_ERR_INVALID_ARG:
+      return "ATTN_ERR_INVALID_ARG: null pointer, non-positive size, misaligned or overlapping "
+             "buffer, non-finite scale or size beyond a limit";
+    case ATTN_ERR_UNSUPPORTED:
+      return "ATTN_ERR_UNSUPPORTED: head_dim must be 64 or 128, dtype f16/bf16, device sm_100";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA runtime or driver call failed";
+    case ATTN_ERR_TIMEOUT:
+      return "ATTN_ERR_TIMEOUT: a bounded device-side pipeline wait expired; outputs undefined";
+    default: return "unknown attn status code";
+  }
+}
+
+int attn_version(void) { return kVersion; }
+
+int attn_debug_set(int inject, unsigned long long wait_timeout_ns) {
+  g_inject.store(inject);
+  g_timeout_ns.store(wait_timeout_ns ? wait_timeout_ns : kDefaultTimeoutNs);
+  return ATTN_OK;
+}
+
+}  // extern "C"

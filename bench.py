@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention forward on B200.  Rank 0 prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload causal4k] [--no-extra]
+
+A step is one call of the whole forward (the tiled prefill kernel for the
+prefill workloads; the split-KV partial and combine kernels for decode) over
+one batch of seeded synthetic inputs already resident in HBM.  Timing: W
+untimed warm-up steps, then exactly K steps bracketed by a barrier and a device
+synchronise, CUDA events on the launching stream, max over ranks.  Every rank
+runs an independent replica of the workload (the forward of one (b, h) never
+talks to another, so there is no data-path collective): scaling is weak.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the method available here) on bounded samples of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOP/s & % of B200 fp16 tensor peak; decode K+V GB/s vs HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_source_sha():
+    """Hash of the CUDA sources: ties a committed ncu traffic figure to the kernel it measured."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "attention_forward_tiled_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel."""
+    sha = kernel_source_sha()
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for name in sorted(os.listdir(pdir)):
+        if not name.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                if line.startswith("bench-traffic:"):
+                    kv = dict(tok.split("=", 1) for tok in line.split()[1:] if "=" in tok)
+                    if kv.get("workload") == workload and kv.get("source_sha") == sha:
+                        return float(kv["bytes_per_launch"])
+    return None
+
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    NAMES = {
+        "nvmlClocksEventReasonGpuIdle": "gpu_idle",
+        "nvmlClocksEventReasonApplicationsClocksSetting": "applications_clocks_setting",
+        "nvmlClocksEventReasonSwPowerCap": "sw_power_cap",
+        "nvmlClocksEventReasonHwSlowdown": "hw_slowdown",
+        "nvmlClocksEventReasonSyncBoost": "sync_boost",
+        "nvmlClocksEventReasonSwThermalSlowdown": "sw_thermal_slowdown",
+        "nvmlClocksEventReasonHwThermalSlowdown": "hw_thermal_slowdown",
+        "nvmlClocksEventReasonHwPowerBrakeSlowdown": "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.nvml = None
+            self.error = str(e)
+
+    def sample_once(self):
+        n = self.nvml
+        self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+        bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        for attr, name in self.NAMES.items():
+            if bits & getattr(n, attr, 0):
+                self.reasons.add(name)
+
+    def run(self):
+        if self.nvml is None:
+            return
+        while not self._stop.is_set():
+            try:
+                self.sample_once()
+            except Exception as e:  # pragma: no cover
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        self.join(timeout=5)
+        if self.nvml is not None and not self.samples:
+            try:
+                self.sample_once()
+            except Exception:
+                pass
+
+    def summary(self):
+        d = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+             "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+             "samples": len(self.samples), "source": "nvml"}
+        if self.error:
+            d["error"] = self.error
+        return d
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def workload_config(name, w):
+    q_bytes = w["B"] * w["Nq"] * w["H"] * w["d"] * 2
+    kv_bytes = 2 * w["B"] * w["Nk"] * w["H"] * w["d"] * 2
+    total = 2 * q_bytes + kv_bytes
+    l2 = ("inputs larger than L2 (%.0f MB of Q, K, V, O per step vs 126 MB L2): no flush"
+          % (total / 1e6)) if total > L2_BYTES else "L2 flushed between steps (256 MB memset)"
+    return {"workload": name, "B": w["B"], "H": w["H"], "Nq": w["Nq"], "Nk": w["Nk"], "d": w["d"],
+            "causal": w["causal"], "dtype": w["dtype"], "scale": w["scale"], "seed": w["seed"],
+            "k_mult": w["k_mult"], "layout": "[B,N,H,d]", "l2": l2, "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def time_gpu_steps(step, K, stream, flush=None):
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for i in range(K):
+            if flush is not None:
+                flush()
+            step()
+            evs[i + 1].record(stream)
+    stream.synchronize()
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+
+
+def measure_workload(name, K, W, world, device, peaks, want_e2e=True):
+    import torch
+
+    import attention_forward_tiled_b200 as attn
+    from attention_forward_tiled_b200.inputs import WORKLOADS, flops, kv_bytes, make_inputs
+
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(**w)
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    out = torch.empty_like(qd)
+    lse = torch.empty((w["B"], w["H"], w["Nq"]), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    total_bytes = 2 * qd.numel() * 2 + 2 * kd.numel() * 2
+    flush_buf = None
+    if total_bytes <= L2_BYTES:
+        flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def step():
+        attn.attn_fwd(qd, kd, vd, causal=w["causal"], scale=w["scale"], out=out, lse=lse,
+                      stream=stream)
+
+    flush = (lambda: flush_buf.zero_()) if flush_buf is not None else None
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(device)
+    if attn.get_status(device=device) != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    t_steps = time_gpu_steps(step, K, stream, flush)
+    sampler.stop()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    if attn.get_status(device=device) != 0:
+        raise RuntimeError("device status error during the timed region")
+    elapsed_ms = max_over_ranks(sum(t_steps), world)
+
+    is_decode = w["Nq"] == 1
+    res = {"elapsed_ms": elapsed_ms, "ms_per_step": elapsed_ms / K, "clocks": sampler.summary()}
+    if is_decode:
+        nbytes = kv_bytes(**w)
+        res["value"] = world * K * nbytes / (elapsed_ms * 1e-3) / 1e9
+        res["unit"] = "GB/s"
+        # each step: partial kernel (dominant) + combine kernel; the step time bounds the partial
+        per_launch = statistics.mean(t_steps)
+        achieved = nbytes / (per_launch * 1e-3) / 1e9
+        res["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                           "traffic": committed_traffic(name),
+                           "algorithmic_bytes_per_launch": nbytes,
+                           "note": "launch time includes the combine kernel"}
+        res["gpu_launches"] = 2 * K
+    else:
+        f = flops(**w)
+        res["value"] = world * K * f / (elapsed_ms * 1e-3) / 1e12
+        res["unit"] = "TFLOP/s"
+        per_launch = statistics.mean(t_steps)
+        achieved = f / (per_launch * 1e-3) / 1e12
+        res["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                           "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                           "traffic": committed_traffic(name),
+                           "algorithmic_flops_per_launch": f,
+                           "peak_note": "%s burst bf16 dense GEMM peak (fp16:bf16 nominal ratio 1:1); "
+                                        "sustained %.1f" % (peaks["source"], peaks["bf16_tflops_sustained"])}
+        res["gpu_launches"] = K
+    res["min_ms"] = min(t_steps)
+
+    if want_e2e:
+        runner = attn.HostRunner(w["B"], w["H"], w["Nq"], w["Nk"], w["d"], q.dtype, device=device,
+                                 causal=w["causal"], scale=w["scale"])
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        runner(qh, kh, vh)
+        torch.cuda.synchronize(device)
+        barrier(world)
+        t_e2e = time_gpu_steps(lambda: runner(qh, kh, vh, stream=stream), K, stream)
+        barrier(world)
+        e_ms = max_over_ranks(sum(t_e2e), world)
+        unit_work = kv_bytes(**w) / 1e9 if is_decode else flops(**w) / 1e12
+        res["e2e"] = {"value": world * K * unit_work / (e_ms * 1e-3), "unit": res["unit"],
+                      "h2d_bytes_per_step": runner.h2d_bytes, "d2h_bytes_per_step": runner.d2h_bytes,
+                      "ms_per_step": e_ms / K}
+        # the result of the last e2e step must match the device-resident run
+        if not torch.equal(runner.out_host, out.cpu()):
+            raise RuntimeError("end-to-end result differs from the device-resident result")
+    del qd, kd, vd, out, lse, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline_sample(name, budget_s=12.0):
+    """Time the oracle, as it stands, on a bounded sample of the workload (rank 0, host cores)."""
+    import oracle
+    from attention_forward_tiled_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(**w)
+    threads = oracle.num_threads()
+    heads = min(w["H"], max(1, threads))
+
+    def run(rows):
+        qs = q[0:1, w["Nq"] - rows:, :heads]
+        ks, vs = k[0:1, :, :heads], v[0:1, :, :heads]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qs, ks, vs, causal=w["causal"], scale=w["scale"])
+        return time.perf_counter() - t0
+
+    def work(rows):  # exact allowed (query, key) pairs x 4 d (bottom-right causal slice)
+        nq, nk = w["Nq"], w["Nk"]
+        if not w["causal"]:
+            pairs = rows * nk
+        else:
+            pairs = sum(max(0, min(nk, i + nk - nq + 1)) for i in range(nq - rows, nq))
+        return 4.0 * w["d"] * pairs * heads
+
+    rows = min(w["Nq"], 32)
+    t = run(rows)
+    if rows < w["Nq"]:
+        rows = int(min(w["Nq"], max(rows, rows * budget_s / max(t, 1e-3))))
+        t = run(rows)
+    is_decode = w["Nq"] == 1
+    if is_decode:
+        value = 2 * heads * w["Nk"] * w["d"] * 2 / t / 1e9
+        unit = "GB/s"
+    else:
+        value = work(rows) / t / 1e12
+        unit = "TFLOP/s"
+    return {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": "batch 0, heads 0..%d, last %d query rows x all %d keys (%s), %.1f s"
+                      % (heads - 1, rows, w["Nk"], "causal, bottom-right" if w["causal"] else "non-causal", t)}
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_setup(args)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    K, W = args.steps, max(3, args.warmup)
+
+    from attention_forward_tiled_b200.inputs import WORKLOADS
+    main = measure_workload(args.workload, K, W, world, device, peaks, want_e2e=True)
+    extra = {}
+    if not args.no_extra:
+        for name in ("decode", "causal8k", "bf16_k3"):
+            if name == args.workload:
+                continue
+            r = measure_workload(name, K, W, world, device, peaks, want_e2e=False)
+            extra[name] = {"value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
+                           "roofline": r["roofline"], "clocks": r["clocks"],
+                           "config": workload_config(name, WORKLOADS[name])}
+    line = {
+        "metric": METRIC,
+        "value": main["value"],
+        "unit": main["unit"],
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": main["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": WORKLOADS[args.workload]["dtype"],
+        "data": "synthetic (seeded randn, the article's [batch, seq, heads, head_dim] shapes)",
+        "config": workload_config(args.workload, WORKLOADS[args.workload]),
+        "roofline": main["roofline"],
+        "e2e": main["e2e"],
+        "gpu_launches": main["gpu_launches"],
+        "clocks": main["clocks"],
+        "impl": "ours",
+    }
+    if extra:
+        line["extra"] = extra
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample(args.workload)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on bounded samples of the same workload
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    import oracle
+    from attention_forward_tiled_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    K, W = args.steps, max(3, args.warmup)
+    q, k, v = make_inputs(**w)
+    threads = oracle.num_threads()
+    heads = min(w["H"], max(1, threads))
+    budget = max(0.2, 150.0 / (K + W))  # seconds per step, whole run within a few minutes
+
+    def run(rows):
+        qs = q[0:1, w["Nq"] - rows:, :heads]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qs, k[0:1, :, :heads], v[0:1, :, :heads], causal=w["causal"], scale=w["scale"])
+        return time.perf_counter() - t0
+
+    rows = min(w["Nq"], 8)
+    t = run(rows)
+    rows = int(min(w["Nq"], max(1, rows * budget / max(t, 1e-4))))
+    for _ in range(W):
+        run(rows)
+    times = [run(rows) for _ in range(K)]
+    nq, nk = w["Nq"], w["Nk"]
+    if w["Nq"] == 1:
+        unit = "GB/s"
+        per_step = 2 * heads * nk * w["d"] * 2 / 1e9
+    else:
+        unit = "TFLOP/s"
+        pairs = (rows * nk if not w["causal"] else
+                 sum(max(0, min(nk, i + nk - nq + 1)) for i in range(nq - rows, nq)))
+        per_step = 4.0 * w["d"] * pairs * heads / 1e12
+    total = sum(times)
+    value = K * per_step / total
+    sample = ("per step: batch 0, heads 0..%d, last %d query rows x all %d keys"
+              % (heads - 1, rows, nk))
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": 1e3 * total / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded randn)",
+        "config": workload_config(args.workload, w), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="causal4k")
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode/causal8k/bf16 lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

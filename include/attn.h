@@ -1,0 +1,127 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) fused attention forward library (libattn.so).
+ *
+ * Operation (FlashAttention/ops-transformer article on ai6s.net):
+ *   O = softmax(scale * Q K^T [+ causal mask]) V, per batch b and head h,
+ * as defined in the section "传统注意力的显存陷阱" (scores = Q K^T / sqrt(d_k),
+ * softmax over the key axis, output = probabilities . V), computed the way the
+ * section "FlashAttention的核心逻辑" describes: Q blocks against streamed K/V
+ * blocks with an online softmax (running row max and row sum, rescaling of the
+ * partial output), one normalisation at the end, so the Nq x Nk score matrix
+ * never exists in device memory.  The causal flag is the one of the article's
+ * API example (section "如何使用", causal=True for GPT-style models).
+ *
+ * Readings where the article is silent:
+ *   - the scale is an explicit argument (1/sqrt(d) is the caller's default);
+ *   - causal with Nq != Nk is aligned to the bottom-right corner: key j is
+ *     allowed for query i iff j <= i + (Nk - Nq);
+ *   - a query row with no allowed key yields O = 0 and lse = -inf;
+ *   - lse is the natural-log row log-sum-exp of the scaled, masked scores.
+ *
+ * Nothing here allocates host memory or keeps a pointer after a call returns.
+ * All pointers except `stream` are DEVICE pointers on the current CUDA device.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL means the legacy default stream. */
+typedef struct CUstream_st* attn_stream_t;
+
+/* Element type of q, k, v and out. */
+typedef enum {
+    ATTN_F16 = 0,   /* IEEE binary16 */
+    ATTN_BF16 = 1   /* bfloat16 */
+} attn_dtype_t;
+
+/* Return codes.  Every entry point returns one of these (negative = error). */
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = -1, /* null pointer, dimension <= 0, misaligned or overlapping
+                                  buffers, non-finite scale, size beyond a stated limit */
+    ATTN_ERR_UNSUPPORTED = -2, /* head_dim not in {64, 128}, unknown dtype, device not sm_100 */
+    ATTN_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed (launch, allocation...) */
+    ATTN_ERR_TIMEOUT = -4      /* device side: a bounded pipeline wait gave up (see attn_get_status) */
+} attn_status_t;
+
+/*
+ * attn_fwd -- fused scaled-dot-product attention forward.
+ *
+ *   q    [B, Nq, H, d]  contiguous, dtype        (read)
+ *   k    [B, Nk, H, d]  contiguous, dtype        (read)
+ *   v    [B, Nk, H, d]  contiguous, dtype        (read)
+ *   out  [B, Nq, H, d]  contiguous, dtype        (written; must not overlap q, k, v, lse)
+ *   lse  [B, H, Nq]     contiguous, float32      (written) or NULL = not written
+ *   B, H, Nq, Nk >= 1;  d (head_dim) in {64, 128};  causal 0/1;  scale finite;
+ *   dtype one of attn_dtype_t;  stream: the caller's stream.
+ *
+ * Alignment: q, k, v, out must be 16-byte aligned (tensor-memory-accelerator
+ * copies); lse 4-byte aligned.
+ *
+ * Paths: Nq == 1 runs the split-KV decode kernels (partials + combine, with a
+ * workspace of B*H*splits*(d+2)*4 bytes taken stream-ordered from the device's
+ * default memory pool and returned on the same stream); every other shape runs
+ * the tiled prefill kernel.  Both give the same result up to fp32 rounding.
+ *
+ * Asynchronous: the call validates its arguments on the host, enqueues the
+ * kernels on `stream` and returns.  Argument errors return before anything is
+ * enqueued.  A device-side failure (a bounded wait that expired) does not
+ * trap: it is recorded in a per-device status word read by attn_get_status().
+ *
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int B, int H, int Nq, int Nk, int d, int causal, float scale,
+             int dtype, attn_stream_t stream);
+
+/*
+ * attn_fwd_prefill / attn_fwd_decode -- the two paths of attn_fwd, callable
+ * directly (same arguments, same contract).  attn_fwd_decode requires Nq == 1
+ * (ATTN_ERR_INVALID_ARG otherwise); `splits` = number of key ranges per
+ * (b, h) row, 0 = automatic, otherwise 1 <= splits <= ceil(Nk / 128).
+ */
+ATTN_API int attn_fwd_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                     int dtype, attn_stream_t stream);
+ATTN_API int attn_fwd_decode(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int B, int H, int Nk, int d, float scale, int dtype, int splits,
+                    attn_stream_t stream);
+
+/*
+ * attn_get_status -- synchronises `stream`, then returns and clears the
+ * current device's status word: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel
+ * since the last call gave up on a pipeline wait (its outputs are then
+ * undefined), or ATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+ATTN_API int attn_get_status(attn_stream_t stream);
+
+/* attn_error_string -- static, human-readable text for a return code. */
+ATTN_API const char* attn_error_string(int status);
+
+/* attn_version -- library version as 10000*major + 100*minor + patch. */
+ATTN_API int attn_version(void);
+
+/*
+ * attn_debug_set -- test hook for the failure-detection path.
+ *   wait_timeout_ns: limit of every bounded device wait (0 = default, 2 s).
+ *   inject: 0 = off; 1 = the prefill producer skips its first Q-tile load, so
+ *   the matrix-multiply issuer's wait on it expires, the kernel records
+ *   ATTN_ERR_TIMEOUT and every role exits without trapping.  Applies to the
+ *   calls that follow on this host process; returns ATTN_OK.
+ */
+ATTN_API int attn_debug_set(int inject, unsigned long long wait_timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

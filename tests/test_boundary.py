@@ -1,0 +1,126 @@
+"""C-ABI boundary checks that need no GPU.
+
+The library must load, export every entry point include/attn.h declares, and
+reject bad arguments on the host with the documented code before any CUDA call
+(the pointers below are never dereferenced: validation fails first).
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import attention_forward_tiled_b200 as attn
+from attention_forward_tiled_b200 import build as abuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    abuild.build()
+    return attn.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:ATTN_API\s+)?(?:const\s+)?\w+\s*\*?\s*(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_get_status", "attn_error_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
+    assert set(declared_functions()) == set(attn.SIGNATURES), "binding and header disagree"
+
+
+def test_only_the_c_abi_is_exported():
+    """-fvisibility=hidden: nothing but the attn_* entry points leaks out of the library."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", attn.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert syms and all(s.startswith("attn_") for s in syms), sorted(syms)[:20]
+
+
+def test_version_and_error_strings(lib):
+    assert lib.attn_version() == 10000
+    for code in (0, -1, -2, -3, -4):
+        assert len(lib.attn_error_string(code)) > 10
+    assert b"unknown" in lib.attn_error_string(-99)
+
+
+# fake, 256-byte aligned, non-overlapping device addresses (never dereferenced)
+Q, K, V, O, L = (ctypes.c_void_p(0x100000000 * (i + 1)) for i in range(5))
+NULL = ctypes.c_void_p(0)
+
+
+def call(lib, q=Q, k=K, v=V, o=O, lse=L, B=1, H=2, Nq=128, Nk=128, d=64, causal=0,
+         scale=0.125, dtype=0):
+    return lib.attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dtype, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(k=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(v=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(o=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(H=-1), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Nq=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Nk=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(d=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=math.nan), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=math.inf), attn.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(dtype=2), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(q=ctypes.c_void_p(0x100000008)), attn.ATTN_ERR_INVALID_ARG),   # 8-byte aligned only
+    (dict(o=ctypes.c_void_p(0x500000004)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(lse=ctypes.c_void_p(0x500000002)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(o=ctypes.c_void_p(0x100000000 + 4096)), attn.ATTN_ERR_INVALID_ARG),  # out overlaps q
+    (dict(o=ctypes.c_void_p(0x200000000)), attn.ATTN_ERR_INVALID_ARG),         # out aliases k
+    (dict(lse=ctypes.c_void_p(0x400000000 + 64)), attn.ATTN_ERR_INVALID_ARG),  # lse inside out
+    (dict(Nk=1 << 30, H=64, d=128), attn.ATTN_ERR_INVALID_ARG),                # batch stride >= 2^40
+])
+def test_invalid_arguments_rejected_on_host(lib, kw, code):
+    assert call(lib, **kw) == code
+
+
+def test_decode_entry_validation(lib):
+    assert lib.attn_fwd_decode(Q, K, V, O, L, 1, 2, 128, 64, 0.1, 0, -1, NULL) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_decode(NULL, K, V, O, L, 1, 2, 128, 64, 0.1, 0, 0, NULL) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_decode(Q, K, V, O, L, 1, 2, 128, 80, 0.1, 0, 0, NULL) == attn.ATTN_ERR_UNSUPPORTED
+
+
+def test_prefill_entry_validation(lib):
+    assert lib.attn_fwd_prefill(Q, K, V, NULL, L, 1, 2, 64, 64, 64, 0, 0.1, 0, NULL) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_prefill(Q, K, V, O, L, 1, 2, 64, 64, 32, 0, 0.1, 1, NULL) == attn.ATTN_ERR_UNSUPPORTED
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 8, 1, 64, dtype=torch.float16)
+    with pytest.raises(TypeError):
+        attn.attn_fwd(q, q, q)
+
+
+def test_package_import_is_lazy_and_loud_without_library(tmp_path):
+    """A missing library raises instead of silently falling back."""
+    from attention_forward_tiled_b200 import _binding
+    saved = _binding._lib
+    _binding._lib = None
+    try:
+        with pytest.raises(RuntimeError):
+            _binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        _binding._lib = saved

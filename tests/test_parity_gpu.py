@@ -1,0 +1,147 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small shapes are compared element by element on every output; the full-size
+workloads run exactly as the benchmark launches them and are compared on whole
+sampled (batch, head) slices (heads are independent, which the oracle tests
+pin) plus properties checked on every output element.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_forward_tiled_b200 import attn_fwd, get_status
+from attention_forward_tiled_b200.inputs import WORKLOADS, make_inputs
+from tests.parity import assert_convex_hull, assert_lse_close, assert_o_close
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def run_and_compare(B, H, Nq, Nk, d, dtype, causal, scale, seed, k_mult=1.0, path="auto",
+                    splits=0, heads=None):
+    q, k, v = make_inputs(B, H, Nq, Nk, d, dtype=dtype, seed=seed, k_mult=k_mult)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    out, lse = attn_fwd(qd, kd, vd, causal=causal, scale=scale, path=path, splits=splits)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    if heads is None:
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal=causal, scale=scale)
+        assert_o_close(out, o_ref, DT[dtype], f"{B}x{H}x{Nq}x{Nk}x{d}")
+        assert_lse_close(lse, lse_ref, "lse")
+    else:
+        for b, h in heads:
+            sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+            o_ref, lse_ref = oracle.attn_fwd(q[sl], k[sl], v[sl], causal=causal, scale=scale)
+            assert_o_close(out[sl], o_ref, DT[dtype], f"head ({b},{h})")
+            assert_lse_close(lse[b:b + 1, h:h + 1], lse_ref, f"lse head ({b},{h})")
+    return q, k, v, out, lse
+
+
+SMALL = [
+    # (B, H, Nq, Nk, d, dtype, causal)
+    (1, 2, 128, 128, 64, "f16", False),
+    (1, 2, 128, 128, 128, "f16", False),
+    (2, 3, 256, 256, 128, "f16", True),
+    (1, 2, 64, 64, 64, "f16", True),
+    (1, 2, 63, 63, 128, "f16", False),
+    (1, 2, 65, 65, 64, "f16", True),
+    (1, 2, 127, 129, 128, "f16", False),
+    (1, 2, 129, 127, 128, "f16", True),
+    (1, 1, 200, 200, 128, "f16", True),
+    (2, 2, 1000, 1000, 64, "f16", True),
+    (1, 2, 1000, 1000, 128, "bf16", False),
+    (1, 2, 300, 700, 128, "f16", True),     # Nq < Nk, bottom-right diagonal not on a tile edge
+    (1, 2, 700, 300, 64, "f16", True),      # Nq > Nk: leading rows see no key
+    (1, 2, 513, 1, 128, "f16", False),      # a single key
+    (1, 2, 513, 1, 64, "bf16", True),       # single key, causal: only the last row has it
+    (1, 3, 2, 517, 128, "f16", True),       # two query rows
+    (3, 1, 384, 384, 64, "bf16", True),     # three Q tiles -> one half-used pair
+    (1, 4, 128, 1024, 128, "bf16", True),
+    (1, 2, 1, 300, 64, "f16", False),       # one query row on the decode path
+    (2, 2, 1, 129, 128, "bf16", True),      # decode path, causal flag is a no-op
+]
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,dtype,causal", SMALL)
+def test_small_shapes(B, H, Nq, Nk, d, dtype, causal):
+    run_and_compare(B, H, Nq, Nk, d, dtype, causal, 1.0 / math.sqrt(d), seed=Nq * 31 + Nk)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.09, 0.5])
+def test_scale_values(scale):
+    run_and_compare(1, 2, 200, 333, 128, "f16", True, scale, seed=77)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_path_with_one_query_row(d):
+    run_and_compare(2, 3, 1, 777, d, "f16", False, 0.1, seed=5, path="prefill")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 32])
+def test_decode_split_counts(splits):
+    run_and_compare(2, 4, 1, 4000, 128, "f16", False, 1 / math.sqrt(128), seed=9, path="decode",
+                    splits=splits)
+
+
+def test_large_logits_bf16():
+    run_and_compare(1, 4, 384, 512, 64, "bf16", False, 1 / 8, seed=3, k_mult=3.0)
+
+
+def test_lse_optional_and_deterministic():
+    q, k, v = (t.cuda() for t in make_inputs(2, 4, 300, 300, 128, seed=8))
+    o1, _ = attn_fwd(q, k, v, causal=True, return_lse=False)
+    o2, l2 = attn_fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    assert l2 is not None
+
+
+def test_side_stream():
+    q, k, v = (t.cuda() for t in make_inputs(1, 2, 256, 256, 64, seed=12))
+    ref, _ = attn_fwd(q, k, v)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        out, _ = attn_fwd(q, k, v, stream=s)
+    s.synchronize()
+    assert torch.equal(out, ref)
+
+
+# ---------------------------------------------------------------------------
+# the named workloads, at full size, in the launch configuration the bench uses
+# ---------------------------------------------------------------------------
+def _workload(name, heads):
+    w = WORKLOADS[name]
+    q, k, v, out, lse = run_and_compare(w["B"], w["H"], w["Nq"], w["Nk"], w["d"], w["dtype"],
+                                        w["causal"], w["scale"], w["seed"], w["k_mult"],
+                                        heads=heads)
+    assert_convex_hull(out, v.cuda(), w["causal"], w["Nq"], w["Nk"])
+    assert torch.isfinite(lse).all()
+
+
+def test_workload_tiny():
+    _workload("tiny", heads=None)
+
+
+def test_workload_causal4k():
+    _workload("causal4k", heads=[(0, 0), (1, 13), (3, 31)])
+
+
+def test_workload_bf16_k3():
+    _workload("bf16_k3", heads=[(0, 0), (4, 9), (7, 15)])
+
+
+def test_workload_causal8k():
+    _workload("causal8k", heads=[(0, 0), (0, 31)])
+
+
+def test_workload_causal8000():
+    _workload("causal8000", heads=[(0, 5), (0, 30)])
+
+
+def test_workload_decode():
+    _workload("decode", heads=None)
