@@ -16,11 +16,13 @@
 //       O_t += P_t V_j    (A = P from TMEM, B = V from shared memory)
 //     alternating the two Q tiles so one tile's softmax overlaps the other
 //     tile's matrix multiplies;
+//   * warps 10-11 (bf16 inputs only) convert each V tile to fp16 in place, so
+//     P V runs with P in fp16 (11-bit significand) rather than bf16 (8-bit);
 //   * warps 0-3 and 4-7 (softmax warpgroups, one per Q tile, one thread per
 //     query row) read a 128-column S row from TMEM, apply the tail/causal mask,
 //     update the running max m and sum l (base-2 exponent with scale*log2(e)
 //     folded into one FMA, lazy rescale of O only when the max grows by more
-//     than 2^8), write P back to TMEM as fp16/bf16 over the consumed S columns,
+//     than 2^8), write P back to TMEM as fp16 over the consumed S columns,
 //     and finally normalise O by 1/l, store it with TMA and write the row LSE.
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
@@ -62,9 +64,10 @@ struct PrefillCfg {
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // +1024: manual 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
+  static constexpr int kThreads = 384;  // 2 softmax warpgroups, producer, MMA, 2 converter warps
   static constexpr int kProducerWarp = 8;
   static constexpr int kMmaWarp = 9;
+  static constexpr int kConvWarp0 = 10;  // warps 10-11: bf16 -> fp16 conversion of V tiles
   // barrier indices
   static constexpr int kBarQFull = 0;    // [2]
   static constexpr int kBarSFull = 2;    // [2]
@@ -73,7 +76,8 @@ struct PrefillCfg {
   static constexpr int kBarMmaDone = 8;  // [1]
   static constexpr int kBarKVFull = 9;   // [kStages]
   static constexpr int kBarKVEmpty = 9 + kStages;
-  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int kBarVConv = 9 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
+  static constexpr int kNumBars = 9 + 3 * kStages;
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area too small");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -148,6 +152,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(BAR(C::kBarKVFull + s), 1);
       mbar_init(BAR(C::kBarKVEmpty + s), 1);
+      mbar_init(BAR(C::kBarVConv + s), 2);  // one arrive per converter warp
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -207,7 +212,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     // ======================= tcgen05 MMA issuer =======================
     if (lane == 0 && nmax > 0) {
       constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
-      constexpr uint32_t idesc_o = make_idesc_f16(128, D, BF16, true);     // P V, V is MN-major
+      // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
+      constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
       const int nkv[2] = {nkv0, nkv1};
       const uint32_t colS[2] = {0u, 128u};
       const uint32_t colO[2] = {256u, 256u + D};
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       for (int j = 0; j < nmax; ++j) {
         const int iv = 2 * j + 1;  // ring item of V_j
         const int sv = iv % C::kStages;
-        mbar_wait(BAR(C::kBarKVFull + sv), (iv / C::kStages) & 1, wctx);
+        mbar_wait(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + sv), (iv / C::kStages) & 1, wctx);
         const int ik = 2 * j + 2;  // ring item of K_{j+1}
         const int sk = ik % C::kStages;
         bool k_ready = false;
@@ -278,6 +284,30 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       // every MMA (and every commit arrive) has landed before TMEM is released
       tc_commit(BAR(C::kBarMmaDone));
       mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+    }
+  } else if (warp >= C::kConvWarp0) {
+    // ======================= bf16 -> fp16 conversion of V tiles (bf16 inputs) ===============
+    if constexpr (BF16) {
+      const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
+      for (int j = 0; j < nmax; ++j) {
+        const int iv = 2 * j + 1;
+        const int sv = iv % C::kStages;
+        mbar_wait(BAR(C::kBarKVFull + sv), (iv / C::kStages) & 1, wctx);
+        __syncwarp();
+        uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + sv * C::kTileBytes);
+#pragma unroll 4
+        for (int c = ct; c < C::kTileBytes / 16; c += 64) {
+          uint4 w = tile[c];
+          w.x = bf16x2_to_f16x2_sat(w.x);
+          w.y = bf16x2_to_f16x2_sat(w.y);
+          w.z = bf16x2_to_f16x2_sat(w.z);
+          w.w = bf16x2_to_f16x2_sat(w.w);
+          tile[c] = w;
+        }
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        __syncwarp();
+        if ((ct & 31) == 0) mbar_arrive(BAR(C::kBarVConv + sv));
+      }
     }
   } else {
     // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ===========
@@ -360,7 +390,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
                 ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), cs, -m_use));
             rs0 += p0;
             rs1 += p1;
-            pk[c >> 6][(c >> 1) & 31] = pack2<BF16>(p0, p1);
+            pk[c >> 6][(c >> 1) & 31] = pack2<false>(p0, p1);
           }
         } else {
 #pragma unroll
@@ -372,7 +402,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             p1 = c + 1 < lim ? p1 : 0.f;
             rs0 += p0;
             rs1 += p1;
-            pk[c >> 6][(c >> 1) & 31] = pack2<BF16>(p0, p1);
+            pk[c >> 6][(c >> 1) & 31] = pack2<false>(p0, p1);
           }
         }
         l_run += rs0 + rs1;

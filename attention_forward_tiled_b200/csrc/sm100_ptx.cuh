@@ -65,6 +65,15 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
   }
 }
 
+// bf16 pair -> fp16 pair (round to nearest even, saturating to +-65504).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
+  const float lo = __uint_as_float(w << 16);
+  const float hi = __uint_as_float(w & 0xFFFF0000u);
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

@@ -97,7 +97,7 @@ class ClockSampler(threading.Thread):
         self.reasons = set()
         self.max_mhz = None
         self.error = None
-        self._stop = threading.Event()
+        self._halt = threading.Event()
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -119,7 +119,7 @@ class ClockSampler(threading.Thread):
     def run(self):
         if self.nvml is None:
             return
-        while not self._stop.is_set():
+        while not self._halt.is_set():
             try:
                 self.sample_once()
             except Exception as e:  # pragma: no cover
@@ -128,7 +128,7 @@ class ClockSampler(threading.Thread):
             time.sleep(self.period)
 
     def stop(self):
-        self._stop.set()
+        self._halt.set()
         self.join(timeout=5)
         if self.nvml is not None and not self.samples:
             try:
