@@ -183,17 +183,28 @@ def workload_config(name, w):
 # our arm
 # ---------------------------------------------------------------------------
 def time_gpu_steps(step, K, stream, flush=None):
+    """Per-step device times (ms) from CUDA events on `stream`; an L2 flush, when
+    given, runs between steps outside the timed intervals."""
     import torch
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    if flush is None:  # back-to-back steps: one event between consecutive steps
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+        with torch.cuda.stream(stream):
+            evs[0].record(stream)
+            for i in range(K):
+                step()
+                evs[i + 1].record(stream)
+        stream.synchronize()
+        return [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     with torch.cuda.stream(stream):
-        evs[0].record(stream)
         for i in range(K):
-            if flush is not None:
-                flush()
+            flush()
+            starts[i].record(stream)
             step()
-            evs[i + 1].record(stream)
+            ends[i].record(stream)
     stream.synchronize()
-    return [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+    return [starts[i].elapsed_time(ends[i]) for i in range(K)]
 
 
 def measure_workload(name, K, W, world, device, peaks, want_e2e=True):
