@@ -24,6 +24,12 @@ using namespace attn_b200;
 // Device status word: kernels record ATTN_ERR_TIMEOUT here instead of trapping.
 __device__ int g_attn_status = 0;
 
+// Fixed scratch of attn_fwd_decode_noalloc: the split partials live here instead of in
+// a per-call allocation.  Every GPU that loads this library holds these 4 MiB until the
+// process exits.  All calls share it and it keeps the last call's contents.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
@@ -43,6 +49,25 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
+
+// Device address of g_noalloc_scratch, looked up once per device (with it current).
+float* g_noalloc_scratch_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+int noalloc_scratch_ptr(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return ATTN_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return ATTN_OK;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -255,6 +280,49 @@ int launch_decode(DeviceState* ds, const void* q, const void* k, const void* v, 
   return rc;
 }
 
+// Same kernels as launch_decode, with the partials in g_noalloc_scratch: no allocation.
+template <int D, bool BF16>
+int launch_decode_noalloc(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
+                          float* lse, int B, int H, int Nk, float scale, int splits_req,
+                          cudaStream_t stream) {
+  using C = DecodeCfg<D>;
+  auto kernel = attn_decode_partial_kernel<D, BF16>;
+  const int slot = 4 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  const int ntiles = (Nk + 127) / 128;
+  const long long BH = (long long)B * H;
+  int splits = splits_req > 0 ? splits_req : choose_splits(BH, ntiles, ds->sm_count);
+  if (splits < 1 || splits > ntiles) return ATTN_ERR_INVALID_ARG;
+  const int tps = (ntiles + splits - 1) / splits;
+  splits = (ntiles + tps - 1) / tps;
+  const long long items = BH * splits;
+  if ((unsigned long long)items * (D + 2) > kNoAllocScratchFloats) return ATTN_ERR_INVALID_ARG;
+  float* part = nullptr;
+  if (int rc = noalloc_scratch_ptr(&part)) return rc;
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+
+  DecodeParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  if (int rc = encode_bnhd(&p.tm_k, k, B, Nk, H, D, dtype)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v, B, Nk, H, D, dtype)) return rc;
+  p.q = q;
+  p.part = part;  // every slot the combine kernel reads is written first by this call
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Nk = Nk;
+  p.splits = splits;
+  p.tiles_per_split = tps;
+  p.n_items = (int)items;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  const int grid = (int)std::min<long long>(items, ds->sm_count);
+  kernel<<<dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  attn_decode_combine_kernel<D, BF16>
+      <<<dim3((unsigned)((BH + 3) / 4)), dim3(128), 0, stream>>>(part, out, lse, (int)BH, splits);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 int dispatch_prefill(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
                      float* lse, int B, int H, int Nq, int Nk, int d, int causal, float scale,
                      int dtype, cudaStream_t stream) {
@@ -314,6 +382,22 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                            reinterpret_cast<cudaStream_t>(stream));
   return dispatch_prefill(ds, q, k, v, out, lse, B, H, Nq, Nk, d, causal, scale, dtype,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int H, int Nk, int d, float scale, int dtype, int splits,
+                            attn_stream_t stream) {
+  if (int rc = validate(q, k, v, out, lse, B, H, 1, Nk, d, 0, scale, dtype)) return rc;
+  if (splits < 0) return ATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_BF16;
+  if (d == 128)
+    return bf16 ? launch_decode_noalloc<128, true>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st)
+                : launch_decode_noalloc<128, false>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st);
+  return bf16 ? launch_decode_noalloc<64, true>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st)
+              : launch_decode_noalloc<64, false>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st);
 }
 
 int attn_get_status(attn_stream_t stream) {

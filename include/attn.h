@@ -97,6 +97,38 @@ ATTN_API int attn_fwd_decode(const void* q, const void* k, const void* v, void* 
                     attn_stream_t stream);
 
 /*
+ * attn_fwd_decode_noalloc -- attn_fwd_decode without any device-memory allocation.
+ * (An addition of this library; the article has no counterpart.)
+ *
+ * For callers that must not allocate device memory while they run: code hosted
+ * inside another framework that owns all device memory and hands a plug-in only
+ * its input and output buffers, serving loops that forbid allocation after
+ * start-up so latency and footprint stay fixed, and processes at their memory
+ * limit, where a per-call allocation could fail in the middle of a step.
+ * attn_fwd_decode takes its split workspace from the stream-ordered pool; this
+ * variant keeps the split partials in a fixed array compiled into the library
+ * instead, and calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layouts and results are those of attn_fwd_decode; the caller
+ * still passes q, k, v, out and lse.  Limit: B * H * splits * (d + 2) must not
+ * exceed 1,048,576 floats (the array is 4 MiB; `splits` after the automatic
+ * choice or the caller's value), otherwise the call returns
+ * ATTN_ERR_INVALID_ARG and launches nothing.  Every GPU that loads the
+ * library holds the 4 MiB array until the process exits.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents; nothing in it has to start at zero, because every slot the
+ * combining kernel reads is written earlier in the same call.  Calls whose
+ * kernels overlap on the GPU (other streams, other host threads) race on the
+ * array and corrupt each other's results: serialise them.
+ */
+ATTN_API int attn_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* out,
+                                     float* lse, int B, int H, int Nk, int d, float scale,
+                                     int dtype, int splits, attn_stream_t stream);
+
+/*
  * attn_get_status -- synchronises `stream`, then returns and clears the
  * current device's status word: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel
  * since the last call gave up on a pipeline wait (its outputs are then
