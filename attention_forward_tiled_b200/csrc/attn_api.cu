@@ -431,6 +431,14 @@ const char* attn_error_string(int status) {
 
 int attn_version(void) { return kVersion; }
 
+#ifdef ATTN_TRACE
+// Timeline read-back of the instrumented build (not part of the regular library).
+ATTN_API int attn_trace_read(void* dst, unsigned long long bytes) {
+  if (bytes > sizeof(g_prefill_trace)) bytes = sizeof(g_prefill_trace);
+  return cudaMemcpyFromSymbol(dst, g_prefill_trace, bytes) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+#endif
+
 int attn_debug_set(int inject, unsigned long long wait_timeout_ns) {
   g_inject.store(inject);
   g_timeout_ns.store(wait_timeout_ns ? wait_timeout_ns : kDefaultTimeoutNs);

@@ -5,25 +5,33 @@
 // (FlashAttention/ops-transformer article, sections "FlashAttention的核心逻辑"
 // and "传统注意力的显存陷阱").  The article's Ascend tiling (Cube unit for the
 // matmuls, Vector unit for the softmax, 128x64 blocks staged in the Unified
-// Buffer) is prior art; this kernel maps the same algorithm onto B200:
+// Buffer) is prior art; this kernel maps the same algorithm onto B200.
 //
-//   * one CTA owns a work unit = (batch b, head h, a pair of 128-row Q tiles);
-//   * warp 8 (producer) streams Q once and then K_0, V_0, K_1, V_1, ... into a
-//     ring of shared-memory stages with TMA (128-byte swizzle), each stage
-//     guarded by a full/empty mbarrier pair;
-//   * warp 9 (MMA issuer, one thread) issues tcgen05.mma:
+// Work unit = (batch b, head h, a pair of 128-row Q tiles).  The grid has one CTA
+// per unit, but a resident CTA (one per SM) keeps going: while it works on a unit
+// it claims the next not-yet-started CTA with cluster launch control
+// (clusterlaunchcontrol.try_cancel) and does that CTA's unit as well, so units are
+// handed out dynamically in launch order (heaviest causal units first, heads in
+// groups so their K/V stay in L2) and TMEM, barriers and the load pipeline stay up
+// across units.  Roles inside a CTA (384 threads):
+//   * warp 8, producer: claims units and publishes them to the other roles through
+//     a two-slot ring in shared memory; loads Q_t once per unit and streams K_0,
+//     V_0, K_1, V_1, ... into a ring of shared-memory stages with TMA (128-byte
+//     swizzle), each stage guarded by a full/empty mbarrier pair;
+//   * warp 9, MMA issuer (whole warp, one elected lane issues) runs tcgen05.mma:
 //       S_t = Q_t K_j^T   (A, B from shared memory, fp32 accumulator in TMEM)
 //       O_t += P_t V_j    (A = P from TMEM, B = V from shared memory)
 //     alternating the two Q tiles so one tile's softmax overlaps the other
 //     tile's matrix multiplies;
 //   * warps 10-11 (bf16 inputs only) convert each V tile to fp16 in place, so
 //     P V runs with P in fp16 (11-bit significand) rather than bf16 (8-bit);
-//   * warps 0-3 and 4-7 (softmax warpgroups, one per Q tile, one thread per
-//     query row) read a 128-column S row from TMEM, apply the tail/causal mask,
+//   * warps 0-3 and 4-7, softmax warpgroups (one per Q tile, one thread per query
+//     row): read the 128-column S row from TMEM, apply the tail/causal mask,
 //     update the running max m and sum l (base-2 exponent with scale*log2(e)
-//     folded into one FMA, lazy rescale of O only when the max grows by more
-//     than 2^8), write P back to TMEM as fp16 over the consumed S columns,
-//     and finally normalise O by 1/l, store it with TMA and write the row LSE.
+//     folded into one packed FMA, lazy rescale of O only when the max grows by more
+//     than 2^8), write P back to TMEM as fp16 over the consumed S columns, and at
+//     the end of the unit normalise O by 1/l, stage it in shared memory, store it
+//     with TMA and write the row LSE.
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [256+D, 256+2D).  P_t occupies columns [64,128) of S_t.
@@ -46,39 +54,46 @@ struct PrefillParams {
   int n_qpairs;      // ceil(Nq / 256)
   int group_heads;   // heads per scheduling group (L2 locality of K/V)
   float scale_log2;  // scale * log2(e)
-  int inject;        // test hook: 1 = skip the first Q-tile load
+  int inject;        // test hook: 1 = skip the Q-tile-0 loads
   unsigned long long timeout_ns;
 };
 
 template <int D>
 struct PrefillCfg {
   static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
-  static constexpr int kRows = 128;                    // rows per Q tile and per K/V tile
   static constexpr int kBoxBytes = 128 * 128;          // 128 rows x 64 elements x 2 bytes
   static constexpr int kBoxes = D / 64;
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = 2 * kTileBytes;
-  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row Q, K, V or O tile
+  static constexpr int kStages = (D == 128) ? 3 : 8;    // K/V ring depth
+  static constexpr int kOffQ = 0;                                    // Q_0, Q_1
+  static constexpr int kOffKV = 2 * kTileBytes;                      // K/V ring
+  static constexpr int kOffO = kOffKV + kStages * kTileBytes;        // O staging, one per tile
+  static constexpr int kOffBar = kOffO + 2 * kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // +1024: manual 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 384;  // 2 softmax warpgroups, producer, MMA, 2 converter warps
+  static constexpr int kThreads = 384;
   static constexpr int kProducerWarp = 8;
   static constexpr int kMmaWarp = 9;
-  static constexpr int kConvWarp0 = 10;  // warps 10-11: bf16 -> fp16 conversion of V tiles
+  static constexpr int kConvWarp0 = 10;
+  static constexpr int kUnitReaders = 11;  // warps that read each published unit: 8 softmax, MMA, 2 converter
   // barrier indices
-  static constexpr int kBarQFull = 0;    // [2]
-  static constexpr int kBarSFull = 2;    // [2]
-  static constexpr int kBarPReady = 4;   // [2]
-  static constexpr int kBarOFull = 6;    // [2]
-  static constexpr int kBarMmaDone = 8;  // [1]
-  static constexpr int kBarKVFull = 9;   // [kStages]
-  static constexpr int kBarKVEmpty = 9 + kStages;
-  static constexpr int kBarVConv = 9 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
-  static constexpr int kNumBars = 9 + 3 * kStages;
-  static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area too small");
+  static constexpr int kBarQFull = 0;      // [2] Q_t landed
+  static constexpr int kBarQEmpty = 2;     // [2] last S_t of the unit done: Q_t buffer free
+  static constexpr int kBarSFull = 4;      // [2] S_t in TMEM
+  static constexpr int kBarPReady = 6;     // [2] P_t in TMEM (and O_t rescaled)
+  static constexpr int kBarOFull = 8;      // [2] last P_t V of the unit done
+  static constexpr int kBarMmaDone = 10;   // [1] teardown
+  static constexpr int kBarClc = 11;       // [1] launch-control response landed
+  static constexpr int kBarUnitFull = 12;  // [2] unit ring slot written
+  static constexpr int kBarUnitEmpty = 14; // [2] unit ring slot read by every reader warp
+  static constexpr int kBarKVFull = 16;    // [kStages]
+  static constexpr int kBarKVEmpty = 16 + kStages;
+  static constexpr int kBarVConv = 16 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
+  static constexpr int kNumBars = 16 + 3 * kStages;
+  static constexpr int kOffMisc = kNumBars * 8;  // tmem slot, abort flag, unit slots[2]
+  static constexpr int kOffClc = ((kOffMisc + 16 + 15) / 16) * 16;  // 16-byte launch-control response
+  static_assert(kOffClc + 16 <= kBarBytes, "barrier area too small");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -95,28 +110,19 @@ __device__ __forceinline__ int prefill_kv_tiles(int row0, int Nq, int Nk, int ca
   return (int)(last_key / 128) + 1;
 }
 
-template <int D, bool BF16>
-__global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
-    attn_prefill_kernel(const __grid_constant__ PrefillParams p) {
-  using C = PrefillCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (sbase - raw_addr);
+// Work unit index -> (b, h, Q-tile rows, K/V tile counts).  Units run in groups of
+// `group_heads` heads; inside a group, causal units go heaviest (last Q rows) first.
+struct PrefillUnit {
+  int b, h;
+  int row0[2];
+  int nkv[2];
+  int nmax;
+};
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  // ---- work unit: (b, h, q-pair), heads grouped for K/V reuse in L2, heavy causal pairs first
+__device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int unit) {
   const int BH = p.B * p.H;
   const int nqp = p.n_qpairs;
   const int G = p.group_heads;
-  const long long unit = blockIdx.x;
   const long long full_units = (long long)(BH / G) * G * nqp;
   int g, idx, Gc;
   if (unit < full_units) {
@@ -131,28 +137,156 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   const int qrank = idx / Gc;
   const int bh = g * G + (idx - qrank * Gc);
   const int qp = p.causal ? (nqp - 1 - qrank) : qrank;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-  const int row0_0 = qp * 256, row0_1 = qp * 256 + 128;
-  const int nkv0 = prefill_kv_tiles(row0_0, p.Nq, p.Nk, p.causal);
-  const int nkv1 = prefill_kv_tiles(row0_1, p.Nq, p.Nk, p.causal);
-  const int nmax = max(nkv0, nkv1);
+  PrefillUnit u;
+  u.b = bh / p.H;
+  u.h = bh - u.b * p.H;
+  u.row0[0] = qp * 256;
+  u.row0[1] = qp * 256 + 128;
+  u.nkv[0] = prefill_kv_tiles(u.row0[0], p.Nq, p.Nk, p.causal);
+  u.nkv[1] = prefill_kv_tiles(u.row0[1], p.Nq, p.Nk, p.causal);
+  u.nmax = max(u.nkv[0], u.nkv[1]);
+  return u;
+}
 
+// Every ATTN_EXP_EMU_PERIOD-th pair of softmax exponentials is evaluated with the
+// FMA-pipe polynomial instead of the MUFU unit (0 = all on MUFU).  At d = 128 the
+// exponentials of one K/V step need as many MUFU cycles as its four MMAs need
+// tensor cycles, so moving a share of them to the FMA pipe shortens the softmax.
+#ifndef ATTN_EXP_EMU_PERIOD
+#define ATTN_EXP_EMU_PERIOD 0
+#endif
+
+// Max over one 64-column half of an S row (columns 64*kHalf + c), sign-flipped for a
+// negative scale, restricted to columns < lim when kMask; four 3-input max chains.
+template <bool kMask, bool kNeg, int kHalf>
+__device__ __forceinline__ float half_max(const uint32_t (&h)[2][32], int lim) {
+  float m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float s0 = __uint_as_float(h[c >> 5][c & 31]);
+    float s1 = __uint_as_float(h[(c + 1) >> 5][(c + 1) & 31]);
+    if (kNeg) {
+      s0 = -s0;
+      s1 = -s1;
+    }
+    if (kMask) {
+      s0 = (64 * kHalf + c) < lim ? s0 : -INFINITY;
+      s1 = (64 * kHalf + c + 1) < lim ? s1 : -INFINITY;
+    }
+    m[(c >> 1) & 3] = fmax3(m[(c >> 1) & 3], s0, s1);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p = 2^(cs * s - m_use) for one 64-column half (0 at columns >= lim when kMask),
+// packed into 32 fp16 pairs (pk[c / 2], low half = even column c of the half).
+// Returns the half's row sum.  Unmasked halves run on the packed fp32x2 pipe.
+template <bool kMask, int kHalf>
+__device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float cs, float m_use,
+                                               int lim, uint32_t (&pk)[32]) {
+  if constexpr (!kMask) {
+    uint64_t acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
+    const uint64_t cs2 = f2_make(cs, cs), negm2 = f2_make(-m_use, -m_use);
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+      const uint64_t x2 = f2_fma(f2_make(__uint_as_float(h[c >> 5][c & 31]),
+                                         __uint_as_float(h[(c + 1) >> 5][(c + 1) & 31])),
+                                 cs2, negm2);
+      float2 pp;
+      if (ATTN_EXP_EMU_PERIOD > 0 && ((c >> 1) % (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD : 1)) ==
+                                         (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD - 1 : 0)) {
+        pp = exp2_poly2(x2);
+      } else {
+        const float2 x = f2_split(x2);
+        pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+      acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_make(pp.x, pp.y));
+      pk[c >> 1] = pack2<false>(pp.x, pp.y);
+    }
+    const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
+    return a.x + a.y;
+  } else {
+    float acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+      const float x0 = fmaf(__uint_as_float(h[c >> 5][c & 31]), cs, -m_use);
+      const float x1 = fmaf(__uint_as_float(h[(c + 1) >> 5][(c + 1) & 31]), cs, -m_use);
+      const float p0 = (64 * kHalf + c) < lim ? ex2_approx(x0) : 0.f;
+      const float p1 = (64 * kHalf + c + 1) < lim ? ex2_approx(x1) : 0.f;
+      acc[(c >> 1) & 3] += p0 + p1;
+      pk[c >> 1] = pack2<false>(p0, p1);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  }
+}
+
+// Optional timeline instrumentation (build with -DATTN_TRACE): the first
+// kTraceCtas CTAs record clock64() at fixed points of every role of their first
+// unit into g_prefill_trace, read back with attn_trace_read().  Compiled out otherwise.
+#ifdef ATTN_TRACE
+constexpr int kTraceCtas = 4;
+constexpr int kTraceSlots = 1024;
+__device__ long long g_prefill_trace[kTraceCtas][kTraceSlots];
+#define ATTN_TRACE_POINT(slot)                                                        \
+  do {                                                                                \
+    if (blockIdx.x < kTraceCtas && (slot) < kTraceSlots)                              \
+      g_prefill_trace[blockIdx.x][(slot)] = clock64();                                \
+  } while (0)
+#else
+#define ATTN_TRACE_POINT(slot) \
+  do {                         \
+  } while (0)
+#endif
+// trace slot layout (first unit only): 0 start; 1 + 64*t + j: MMA saw P_t(j) ready;
+// 129 + 64*t + j: MMA issued S_t(j+1); 257 + 64*t + j: softmax t saw S_t(j);
+// 385 + ...: S loaded; 513 + ...: max done; 641 + ...: P computed; 769 + ...: P ready
+// arrived; 897 + i: producer issued ring item i.
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
+    attn_prefill_kernel(const __grid_constant__ PrefillParams p) {
+  using C = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_addr);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [2]
+  const uint32_t clc_resp = sbase + C::kOffBar + C::kOffClc;
+  auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
 
   // ---- one-time setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(C::kBarQFull + i), 1);
+      mbar_init(BAR(C::kBarQEmpty + i), 1);
       mbar_init(BAR(C::kBarSFull + i), 1);
       mbar_init(BAR(C::kBarPReady + i), 4);  // one arrive per softmax warp
       mbar_init(BAR(C::kBarOFull + i), 1);
+      mbar_init(BAR(C::kBarUnitFull + i), 1);
+      mbar_init(BAR(C::kBarUnitEmpty + i), C::kUnitReaders);
     }
     mbar_init(BAR(C::kBarMmaDone), 1);
+    mbar_init(BAR(C::kBarClc), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(BAR(C::kBarKVFull + s), 1);
-      mbar_init(BAR(C::kBarKVEmpty + s), 1);
-      mbar_init(BAR(C::kBarVConv + s), 2);  // one arrive per converter warp
+      // bf16: the two converter warps also observe and release every ring item, so no
+      // waiter on these barriers can ever be two phases behind or ahead
+      mbar_init(BAR(C::kBarKVEmpty + s), BF16 ? 3 : 1);
+      mbar_init(BAR(C::kBarVConv + s), 2);  // one arrive per converter warp, every ring item
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -165,158 +299,235 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) ATTN_TRACE_POINT(0);
 
+  // Every role walks the same unit sequence, published by the producer.  Returns the
+  // k-th unit (-1 = no more) after this warp has read it and released its slot.
+  auto next_unit = [&](int k) -> int {
+    mbar_wait(BAR(C::kBarUnitFull + (k & 1)), (k >> 1) & 1, wctx);
+    __syncwarp();
+    const int u = __shfl_sync(0xffffffffu, unit_slot[k & 1], 0);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(C::kBarUnitEmpty + (k & 1)));
+    return u;
+  };
+
+  static_assert(C::kProducerWarp == 8 && C::kMmaWarp == 9 && C::kConvWarp0 == 10 && C::kThreads == 384,
+                "warpgroup 2 = producer, MMA issuer, two converter warps");
   if (warp == C::kProducerWarp) {
-    // ======================= TMA producer =======================
+    // ======================= producer: unit claims + TMA loads ======================
     if (lane == 0) {
       tma_prefetch_map(&p.tm_q);
       tma_prefetch_map(&p.tm_k);
       tma_prefetch_map(&p.tm_v);
       tma_prefetch_map(&p.tm_o);
-      const int nkv[2] = {nkv0, nkv1};
-      const int row0[2] = {row0_0, row0_1};
-      bool q_issued[2] = {false, false};
+    }
+    __syncwarp();
+    int unit = blockIdx.x;  // the first unit is this CTA's own
+    int nq[2] = {0, 0};     // Q loads issued per tile
+    bool q_pending[2] = {false, false};
+    int g = 0;              // ring items issued
+    int nclaim = 0;
+    for (int k = 0;; ++k) {
+      if (k >= 2) mbar_wait(BAR(C::kBarUnitEmpty + (k & 1)), ((k >> 1) - 1) & 1, wctx);
+      __syncwarp();
+      if (lane == 0) {
+        unit_slot[k & 1] = unit;
+        mbar_arrive(BAR(C::kBarUnitFull + (k & 1)));
+      }
+      __syncwarp();
+      if (unit < 0) break;
+      const bool claim = !warp_flag(abort_flag);
+      if (claim) {
+        mbar_arrive_expect_tx_w(BAR(C::kBarClc), 16);
+        clc_try_cancel_w(clc_resp, BAR(C::kBarClc));
+      }
+      const PrefillUnit u = prefill_unit(p, unit);
       for (int t = 0; t < 2; ++t) {
-        if (nkv[t] == 0) continue;
-        if (p.inject == 1 && t == 0) continue;  // test hook: the MMA issuer's wait must expire
-        mbar_arrive_expect_tx(BAR(C::kBarQFull + t), C::kTileBytes);
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_4d(sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
-                      BAR(C::kBarQFull + t), bx * 64, h, row0[t], b);
-        q_issued[t] = true;
+        if (u.nkv[t] == 0) continue;
+        if (nq[t] > 0) mbar_wait(BAR(C::kBarQEmpty + t), (nq[t] - 1) & 1, wctx);
+        __syncwarp();
+        if (!(p.inject == 1 && t == 0) && !warp_flag(abort_flag)) {
+          mbar_arrive_expect_tx_w(BAR(C::kBarQFull + t), C::kTileBytes);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_4d_w(sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
+                          BAR(C::kBarQFull + t), bx * 64, u.h, u.row0[t], u.b);
+          q_pending[t] = true;
+        }
+        ++nq[t];
       }
-      int issued = 0;
-      for (int i = 0; i < 2 * nmax; ++i) {
-        const int stage = i % C::kStages;
-        const int round = i / C::kStages;
+      for (int i = 0; i < 2 * u.nmax; ++i, ++g) {
+        const int stage = g % C::kStages;
+        const int round = g / C::kStages;
         if (round > 0) mbar_wait(BAR(C::kBarKVEmpty + stage), (round - 1) & 1, wctx);
-        if (*abort_flag) break;
-        mbar_arrive_expect_tx(BAR(C::kBarKVFull + stage), C::kTileBytes);
+        __syncwarp();
+        if (warp_flag(abort_flag)) continue;
+        mbar_arrive_expect_tx_w(BAR(C::kBarKVFull + stage), C::kTileBytes);
         const CUtensorMap* map = (i & 1) ? &p.tm_v : &p.tm_k;
-        const int key0 = (i >> 1) * 128;
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_4d(sbase + C::kOffKV + stage * C::kTileBytes + bx * C::kBoxBytes, map,
-                      BAR(C::kBarKVFull + stage), bx * 64, h, key0, b);
-        issued = i + 1;
+          tma_load_4d_w(sbase + C::kOffKV + stage * C::kTileBytes + bx * C::kBoxBytes, map,
+                        BAR(C::kBarKVFull + stage), bx * 64, u.h, (i >> 1) * 128, u.b);
+        if (lane == 0 && k == 0) ATTN_TRACE_POINT(897 + i);
       }
-      if (*abort_flag) {
-        // Let every copy this thread started land before the CTA can exit.
-        for (int t = 0; t < 2; ++t)
-          if (q_issued[t]) mbar_wait_drain(BAR(C::kBarQFull + t), 0, p.timeout_ns);
-        const int first = issued > C::kStages ? issued - C::kStages : 0;
-        for (int i = first; i < issued; ++i)
-          mbar_wait_drain(BAR(C::kBarKVFull + i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+      int next = -1;
+      if (claim) {
+        if (mbar_wait(BAR(C::kBarClc), nclaim & 1, wctx)) next = clc_response_ctaid_x(clc_resp);
+        else mbar_wait_drain(BAR(C::kBarClc), nclaim & 1, p.timeout_ns);
+        ++nclaim;
       }
+      __syncwarp();
+      unit = __shfl_sync(0xffffffffu, next, 0);
+    }
+    if (warp_flag(abort_flag)) {
+      // Let every copy this warp started land before the CTA can exit.
+      for (int t = 0; t < 2; ++t)
+        if (q_pending[t]) mbar_wait_drain(BAR(C::kBarQFull + t), (nq[t] - 1) & 1, p.timeout_ns);
+      const int first = g > C::kStages ? g - C::kStages : 0;
+      for (int i = first; i < g; ++i)
+        mbar_wait_drain(BAR(C::kBarKVFull + i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+      __syncwarp();
     }
   } else if (warp == C::kMmaWarp) {
-    // ======================= tcgen05 MMA issuer =======================
-    if (lane == 0 && nmax > 0) {
-      constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
-      // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
-      constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
-      const int nkv[2] = {nkv0, nkv1};
-      const uint32_t colS[2] = {0u, 128u};
-      const uint32_t colO[2] = {256u, 256u + D};
-      const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
-      bool ok = true;
-      for (int t = 0; t < 2; ++t)
-        if (nkv[t] > 0) ok = mbar_wait(BAR(C::kBarQFull + t), 0, wctx) && ok;
-
-      // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
-      auto issue_s = [&](int t, uint32_t sK) {
+    // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
+    constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
+    // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
+    constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
+    const uint32_t colS[2] = {0u, 128u};
+    const uint32_t colO[2] = {256u, 256u + D};
+    const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+    // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
+    auto issue_s = [&](int t, uint32_t sK) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + colS[t], make_sdesc_sw128(sQ[t] + off, 16, 1024),
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+        mma_f16_ss_w(tmem + colS[t], make_sdesc_sw128(sQ[t] + off, 16, 1024),
                      make_sdesc_sw128(sK + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-      };
-      // O_t += P_t V_j over 8 k-steps of 16 keys; P_t is in TMEM columns [64,128) of S_t.
-      auto issue_pv = [&](int t, uint32_t sV, bool accumulate_first) {
+      }
+    };
+    // O_t += P_t V_j over 8 k-steps of 16 keys; P_t is in TMEM columns [64,128) of S_t.
+    auto issue_pv = [&](int t, uint32_t sV, bool accumulate_first) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_f16_ts(tmem + colO[t], tmem + colS[t] + 64 + kk * 8,
+      for (int kk = 0; kk < 8; ++kk) {
+        mma_f16_ts_w(tmem + colO[t], tmem + colS[t] + 64 + kk * 8,
                      make_sdesc_sw128(sV + kk * 2048, C::kBoxBytes, 1024), idesc_o,
                      (accumulate_first || kk > 0) ? 1u : 0u);
-        }
-      };
-
-      // prologue: S_t(0) for both tiles from K_0 (ring item 0)
-      ok = mbar_wait(BAR(C::kBarKVFull + 0), 0, wctx) && ok;
-      if (ok && !*abort_flag) {
-        for (int t = 0; t < 2; ++t)
-          if (nkv[t] > 0) {
-            issue_s(t, sbase + C::kOffKV);
-            tc_commit(BAR(C::kBarSFull + t));
-          }
-        tc_commit(BAR(C::kBarKVEmpty + 0));
       }
-      for (int j = 0; j < nmax; ++j) {
-        const int iv = 2 * j + 1;  // ring item of V_j
-        const int sv = iv % C::kStages;
-        mbar_wait(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + sv), (iv / C::kStages) & 1, wctx);
-        const int ik = 2 * j + 2;  // ring item of K_{j+1}
-        const int sk = ik % C::kStages;
+    };
+    auto stage_addr = [&](int item) -> uint32_t {
+      return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;
+    };
+    int nq[2] = {0, 0};  // units seen per tile (q_full / q_empty phases)
+    int np[2] = {0, 0};  // P tiles consumed per tile (p_ready phases)
+    int g = 0;           // ring items consumed
+    for (int k = 0;; ++k) {
+      const int unit = next_unit(k);
+      if (unit < 0) break;
+      const PrefillUnit u = prefill_unit(p, unit);
+      if (u.nmax == 0) continue;
+      for (int t = 0; t < 2; ++t)
+        if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
+      // prologue: S_t(0) for both tiles from K_0
+      mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      if (!warp_flag(abort_flag)) {
+        for (int t = 0; t < 2; ++t)
+          if (u.nkv[t] > 0) {
+            issue_s(t, stage_addr(g));
+            tc_commit_w(BAR(C::kBarSFull + t));
+            if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
+          }
+        tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
+      }
+      for (int j = 0; j < u.nmax; ++j) {
+        const int iv = g + 2 * j + 1;  // ring item of V_j
+        mbar_wait(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + iv % C::kStages), (iv / C::kStages) & 1,
+                  wctx);
+        __syncwarp();
+        const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
-          if (j >= nkv[t]) continue;
-          mbar_wait(BAR(C::kBarPReady + t), j & 1, wctx);
+          if (j >= u.nkv[t]) continue;
+          mbar_wait(BAR(C::kBarPReady + t), np[t] & 1, wctx);
+          ++np[t];
+          __syncwarp();
+          if (lane == 0 && k == 0) ATTN_TRACE_POINT(1 + 64 * t + j);
           tc_fence_after_sync();
-          if (*abort_flag) continue;
-          issue_pv(t, sbase + C::kOffKV + sv * C::kTileBytes, j > 0);
-          if (j + 1 < nkv[t]) {
+          if (warp_flag(abort_flag)) continue;
+          issue_pv(t, stage_addr(iv), j > 0);
+          if (j + 1 < u.nkv[t]) {
             if (!k_ready) {
-              mbar_wait(BAR(C::kBarKVFull + sk), (ik / C::kStages) & 1, wctx);
+              mbar_wait(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
+              __syncwarp();
               k_ready = true;
             }
-            if (*abort_flag) continue;
-            issue_s(t, sbase + C::kOffKV + sk * C::kTileBytes);
-            tc_commit(BAR(C::kBarSFull + t));
+            if (warp_flag(abort_flag)) continue;
+            issue_s(t, stage_addr(ik));
+            tc_commit_w(BAR(C::kBarSFull + t));
+            if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
+            if (lane == 0 && k == 0) ATTN_TRACE_POINT(129 + 64 * t + j);
           } else {
-            tc_commit(BAR(C::kBarOFull + t));
+            tc_commit_w(BAR(C::kBarOFull + t));
           }
         }
-        if (!*abort_flag) {
-          tc_commit(BAR(C::kBarKVEmpty + sv));
-          if (k_ready) tc_commit(BAR(C::kBarKVEmpty + sk));
+        if (!warp_flag(abort_flag)) {
+          tc_commit_w(BAR(C::kBarKVEmpty + iv % C::kStages));
+          if (k_ready) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
         }
       }
-      // every MMA (and every commit arrive) has landed before TMEM is released
-      tc_commit(BAR(C::kBarMmaDone));
-      mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+      g += 2 * u.nmax;
+      for (int t = 0; t < 2; ++t)
+        if (u.nkv[t] > 0) ++nq[t];
     }
+    // every MMA (and every commit arrive) has landed before TMEM is released
+    tc_commit_w(BAR(C::kBarMmaDone));
+    mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+    __syncwarp();
   } else if (warp >= C::kConvWarp0) {
-    // ======================= bf16 -> fp16 conversion of V tiles (bf16 inputs) ===============
-    if constexpr (BF16) {
-      const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
-      for (int j = 0; j < nmax; ++j) {
-        const int iv = 2 * j + 1;
-        const int sv = iv % C::kStages;
-        mbar_wait(BAR(C::kBarKVFull + sv), (iv / C::kStages) & 1, wctx);
-        __syncwarp();
-        uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + sv * C::kTileBytes);
+    // ======================= bf16 -> fp16 conversion of V tiles (bf16 inputs) ======
+    // Walks every ring item in order: waits for it to land, converts it if it is a V
+    // tile, then arrives on its v_conv barrier (the MMA issuer waits on that for V
+    // tiles) and on its empty barrier (the producer refills a stage only after both the
+    // tensor core and the converters are done with it).
+    const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
+    int g = 0;
+    for (int k = 0;; ++k) {
+      const int unit = next_unit(k);
+      if (unit < 0) break;
+      const PrefillUnit u = prefill_unit(p, unit);
+      if constexpr (BF16) {
+        for (int i = 0; i < 2 * u.nmax; ++i) {
+          const int item = g + i;
+          const int st = item % C::kStages;
+          mbar_wait(BAR(C::kBarKVFull + st), (item / C::kStages) & 1, wctx);
+          __syncwarp();
+          if (i & 1) {
+            uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + st * C::kTileBytes);
 #pragma unroll 4
-        for (int c = ct; c < C::kTileBytes / 16; c += 64) {
-          uint4 w = tile[c];
-          w.x = bf16x2_to_f16x2_sat(w.x);
-          w.y = bf16x2_to_f16x2_sat(w.y);
-          w.z = bf16x2_to_f16x2_sat(w.z);
-          w.w = bf16x2_to_f16x2_sat(w.w);
-          tile[c] = w;
+            for (int c = ct; c < C::kTileBytes / 16; c += 64) {
+              uint4 w = tile[c];
+              w.x = bf16x2_to_f16x2_sat(w.x);
+              w.y = bf16x2_to_f16x2_sat(w.y);
+              w.z = bf16x2_to_f16x2_sat(w.z);
+              w.w = bf16x2_to_f16x2_sat(w.w);
+              tile[c] = w;
+            }
+            fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(BAR(C::kBarVConv + st));
+            mbar_arrive(BAR(C::kBarKVEmpty + st));
+          }
         }
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-        __syncwarp();
-        if ((ct & 31) == 0) mbar_arrive(BAR(C::kBarVConv + sv));
       }
+      g += 2 * u.nmax;
     }
   } else {
-    // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ===========
+    // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ======
     const int t = warp >> 2;
-    const int quarter = warp & 3;           // TMEM lane quarter this warp may access
-    const int r = quarter * 32 + lane;      // row inside the Q tile
-    const int row0 = t ? row0_1 : row0_0;
-    const int nkv = t ? nkv1 : nkv0;
-    const int grow = row0 + r;              // global query row
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;  // row inside the Q tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + (t ? 128u : 0u);
     const uint32_t tO = tmem + lane_base + (t ? 256u + D : 256u);
@@ -324,22 +535,36 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     const bool neg = cs < 0.f;
     const float cs_abs = fabsf(cs);
     const long long diag = (long long)p.Nk - p.Nq;
+    uint8_t* ostage = smem + C::kOffO + t * C::kTileBytes;
+    int ns = 0;  // S tiles consumed (s_full phases)
+    int no = 0;  // units finished (o_full phases)
+    for (int k = 0;; ++k) {
+      const int unit = next_unit(k);
+      if (unit < 0) break;
+      const PrefillUnit u = prefill_unit(p, unit);
+      const int row0 = u.row0[t];
+      const int nkv = u.nkv[t];
+      const int grow = row0 + r;  // global query row
+      if (nkv == 0) {
+        // every row of this tile is left without a key (causal, Nq > Nk): O = 0, lse = -inf
+        if (row0 < p.Nq && grow < p.Nq) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
+                                                ((((long long)u.b * p.Nq + grow) * p.H + u.h) * D) * 2);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (p.lse != nullptr) p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = -INFINITY;
+        }
+        continue;
+      }
 
-    float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazy: may lag the true max by <= 8)
-    float l_run = 0.f;        // running sum of 2^(cs*s - m_run)
-
-    if (nkv > 0) {
+      float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazy: may lag the true max by <= 8)
+      float l_run = 0.f;        // running sum of 2^(cs*s - m_run)
       for (int j = 0; j < nkv; ++j) {
-        mbar_wait(BAR(C::kBarSFull + t), j & 1, wctx);
+        mbar_wait(BAR(C::kBarSFull + t), ns & 1, wctx);
+        ++ns;
         __syncwarp();  // lanes may leave the bounded wait on different polls
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(257 + 64 * t + j);
         tc_fence_after_sync();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_order_after_wait(sr[c]);
-
         // mask needed on the key tail and on tiles crossing the causal diagonal
         const long long key0 = (long long)j * 128;
         const bool need_mask = (key0 + 128 > p.Nk) ||
@@ -352,23 +577,24 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
           lim = (int)max(0LL, min(128LL, l));
         }
 
-        // tile max of the sign-adjusted raw scores (scale folded in afterwards)
-        float mx = -INFINITY;
-        if (!need_mask) {
-          if (!neg) {
-#pragma unroll
-            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, -__uint_as_float(sr[c >> 5][c & 31]));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float s = __uint_as_float(sr[c >> 5][c & 31]);
-            mx = fmaxf(mx, c < lim ? (neg ? -s : s) : -INFINITY);
-          }
-        }
+        // pass 1: row max over the two 64-column halves (half 1 stays in registers)
+        uint32_t hv[2][32];
+        tmem_ld32(tS + 0, hv[0]);
+        tmem_ld32(tS + 32, hv[1]);
+        tmem_ld_wait();
+        reg_order_after_wait(hv[0]);
+        reg_order_after_wait(hv[1]);
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(385 + 64 * t + j);
+        float mx = need_mask ? (neg ? half_max<true, true, 0>(hv, lim) : half_max<true, false, 0>(hv, lim))
+                             : (neg ? half_max<false, true, 0>(hv, lim) : half_max<false, false, 0>(hv, lim));
+        tmem_ld32(tS + 64, hv[0]);
+        tmem_ld32(tS + 96, hv[1]);
+        tmem_ld_wait();
+        reg_order_after_wait(hv[0]);
+        reg_order_after_wait(hv[1]);
+        mx = fmaxf(mx, need_mask ? (neg ? half_max<true, true, 1>(hv, lim) : half_max<true, false, 1>(hv, lim))
+                                 : (neg ? half_max<false, true, 1>(hv, lim) : half_max<false, false, 1>(hv, lim)));
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(513 + 64 * t + j);
         const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cs_abs;
         const float m_new = fmaxf(m_run, m_tile);
         const bool rescale = m_new > m_run + 8.0f;
@@ -379,35 +605,25 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
 
-        // P = 2^(cs*s - m), row sum, pack to 16-bit pairs
-        uint32_t pk[2][32];
-        float rs0 = 0.f, rs1 = 0.f;
-        if (!need_mask) {
-#pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), cs, -m_use));
-            const float p1 =
-                ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), cs, -m_use));
-            rs0 += p0;
-            rs1 += p1;
-            pk[c >> 6][(c >> 1) & 31] = pack2<false>(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            float p0 = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), cs, -m_use));
-            float p1 =
-                ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), cs, -m_use));
-            p0 = c < lim ? p0 : 0.f;
-            p1 = c + 1 < lim ? p1 : 0.f;
-            rs0 += p0;
-            rs1 += p1;
-            pk[c >> 6][(c >> 1) & 31] = pack2<false>(p0, p1);
-          }
-        }
-        l_run += rs0 + rs1;
-        tmem_st32(tS + 64, pk[0]);
-        tmem_st32(tS + 96, pk[1]);
+        // pass 2: P for half 1 (keys 64..127, from registers) into TMEM columns 96..127,
+        // which held S columns 96..127 -- already read; then half 0 re-read from TMEM
+        // (columns 0..63, untouched) into P columns 64..95.
+        uint32_t pk[32];
+        float rs = need_mask ? half_exp_pack<true, 1>(hv, cs, m_use, lim, pk)
+                             : half_exp_pack<false, 1>(hv, cs, m_use, lim, pk);
+        __syncwarp();
+        tmem_st32(tS + 96, pk);
+        tmem_ld32(tS + 0, hv[0]);
+        tmem_ld32(tS + 32, hv[1]);
+        tmem_ld_wait();
+        reg_order_after_wait(hv[0]);
+        reg_order_after_wait(hv[1]);
+        rs += need_mask ? half_exp_pack<true, 0>(hv, cs, m_use, lim, pk)
+                        : half_exp_pack<false, 0>(hv, cs, m_use, lim, pk);
+        l_run += rs;
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
+        __syncwarp();
+        tmem_st32(tS + 64, pk);
 
         // lazy rescale of O (the previous P V of this tile completed before S_t(j) did)
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
@@ -426,14 +642,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kBarPReady + t));
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
       }
 
-      // ---- epilogue: O / l -> 16-bit -> swizzled smem (this tile's Q buffer) -> TMA store
-      mbar_wait(BAR(C::kBarOFull + t), 0, wctx);
+      // ---- epilogue: O / l -> 16-bit -> swizzled staging buffer -> TMA store
+      mbar_wait(BAR(C::kBarOFull + t), no & 1, wctx);
+      ++no;
       __syncwarp();
       tc_fence_after_sync();
+      named_bar_sync(1 + t, 128);  // the previous store from this staging buffer has read it
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-      uint8_t* stage = smem + C::kOffQ + t * C::kTileBytes;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -449,31 +667,22 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
           w.w = pack2<BF16>(__uint_as_float(o[q4 * 8 + 6]) * inv_l, __uint_as_float(o[q4 * 8 + 7]) * inv_l);
           const int chunk = c * 4 + q4;  // 16-byte chunk index along the row
           const int bx = chunk >> 3, cc = chunk & 7;
-          *reinterpret_cast<uint4*>(stage + bx * C::kBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+          *reinterpret_cast<uint4*>(ostage + bx * C::kBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
         }
       }
       fence_proxy_async_smem();
       named_bar_sync(1 + t, 128);
       if (r == 0 && !*abort_flag) {
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_store_4d(&p.tm_o, sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64,
-                       h, row0, b);
+          tma_store_4d(&p.tm_o, sbase + C::kOffO + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64,
+                       u.h, row0, u.b);
         bulk_commit_group();
         bulk_wait_group_read0();
       }
       if (p.lse != nullptr && grow < p.Nq) {
         const float lse = l_run > 0.f ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                       : -INFINITY;
-        p.lse[((long long)b * p.H + h) * p.Nq + grow] = lse;
-      }
-    } else if (row0 < p.Nq) {
-      // every row of this tile is left without a key (causal, Nq > Nk): O = 0, lse = -inf
-      if (grow < p.Nq) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
-                                              ((((long long)b * p.Nq + grow) * p.H + h) * D) * 2);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-        if (p.lse != nullptr) p.lse[((long long)b * p.H + h) * p.Nq + grow] = -INFINITY;
+        p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
       }
     }
   }

@@ -10,6 +10,8 @@
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 
+#include "exp2_poly.cuh"
+
 namespace attn_b200 {
 
 // Status codes shared with include/attn.h (device-side subset).
@@ -42,6 +44,66 @@ __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA/ALU pipes (no MUFU): Cody-Waite reduction 2^x = 2^j * 2^f with
+// j = round(x) taken from the low mantissa bits of x + 1.5*2^23 and f = x - j in
+// [-1/2, 1/2], a minimax cubic for 2^f (exp2_poly.cuh), and 2^j applied by adding
+// j to the exponent field.  Inputs are clamped to >= -125 so the result stays a
+// normal float; intended for the softmax exponents (x <= ~8).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23
+  const float j = t - 12582912.0f;  // round-to-nearest-even(x)
+  const float f = x - j;
+  float p = fmaf(kExp2PolyC3, f, kExp2PolyC2);
+  p = fmaf(p, f, kExp2PolyC1);
+  p = fmaf(p, f, kExp2PolyC0);
+  // bits(t) = bits(1.5*2^23) + j, and bits(1.5*2^23) << 23 == 0 (mod 2^32)
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// ---- packed fp32x2 arithmetic (sm_100): one instruction for two lanes of work
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// exp2_poly on a packed pair (range reduction and cubic on the packed fp32x2 pipe).
+__device__ __forceinline__ float2 exp2_poly2(uint64_t x2) {
+  const float2 xc = f2_split(x2);
+  x2 = f2_make(fmaxf(xc.x, -125.0f), fmaxf(xc.y, -125.0f));
+  const uint64_t magic = f2_make(12582912.0f, 12582912.0f);      // 1.5 * 2^23
+  const uint64_t t2 = f2_add(x2, magic);
+  const uint64_t j2 = f2_add(t2, f2_make(-12582912.0f, -12582912.0f));
+  const uint64_t f2 = f2_fma(j2, f2_make(-1.0f, -1.0f), x2);     // x - round(x)
+  uint64_t p2 = f2_fma(f2_make(kExp2PolyC3, kExp2PolyC3), f2, f2_make(kExp2PolyC2, kExp2PolyC2));
+  p2 = f2_fma(p2, f2, f2_make(kExp2PolyC1, kExp2PolyC1));
+  p2 = f2_fma(p2, f2, f2_make(kExp2PolyC0, kExp2PolyC0));
+  const float2 p = f2_split(p2), t = f2_split(t2);
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Pack two fp32 values (lo -> bits 0..15, hi -> bits 16..31) with round-to-nearest-even.
@@ -95,8 +157,23 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// Optional upper bound (ns) on how long one try_wait may suspend the thread; 0 = the
+// hardware's default.
+#ifndef ATTN_WAIT_HINT_NS
+#define ATTN_WAIT_HINT_NS 0
+#endif
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+#if ATTN_WAIT_HINT_NS > 0
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(ATTN_WAIT_HINT_NS)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -104,6 +181,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 
@@ -260,6 +338,110 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
                                                      uint32_t sbo_bytes) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// ---------------------------------------------------------------------------
+// Warp-collective issue: the whole (converged) warp executes these, one lane
+// elected by elect.sync issues the instruction.  Keeping the issuing warp
+// converged lets the compiler hold descriptors and addresses in uniform
+// registers; issuing from a single divergent lane costs hundreds of cycles per
+// instruction.  elect.sync picks the same (lowest) lane every time, so all
+// tcgen05 operations of a warp come from one thread, as tcgen05.commit needs.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_f16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_f16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_w(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}\n" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_w(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                              int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];\n\t}\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// Register re-balancing between warpgroups (all four warps of a warpgroup execute it).
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+// Cluster launch control: ask the hardware to cancel the launch of a not-yet-started
+// CTA of this grid; the 16-byte response lands in shared memory with complete_tx on
+// `bar`.  Whole warp calls; one elected lane issues.
+__device__ __forceinline__ void clc_try_cancel_w(uint32_t resp_smem, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];\n\t}\n" ::"r"(resp_smem),
+      "r"(bar)
+      : "memory");
+}
+
+// Decode a launch-control response: the x index of the cancelled CTA, or -1 if none
+// was cancelled (no CTA of the grid is left to start).
+__device__ __forceinline__ int clc_response_ctaid_x(uint32_t resp_smem) {
+  uint32_t valid, x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 res;\n\t"
+      "ld.shared.b128 res, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, res;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "mov.u32 %1, 0;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, res;\n\t}\n"
+      : "=r"(valid), "=r"(x)
+      : "r"(resp_smem)
+      : "memory");
+  return valid ? (int)x : -1;
+}
+
+// Warp-uniform read of a shared flag (lane 0's view, broadcast).
+__device__ __forceinline__ bool warp_flag(const volatile int* flag) {
+  return __shfl_sync(0xffffffffu, *flag, 0) != 0;
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane
