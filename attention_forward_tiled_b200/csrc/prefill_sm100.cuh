@@ -64,11 +64,11 @@ struct PrefillCfg {
   static constexpr int kBoxBytes = 128 * 128;          // 128 rows x 64 elements x 2 bytes
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row Q, K, V or O tile
-  static constexpr int kStages = (D == 128) ? 3 : 8;    // K/V ring depth
+  static constexpr int kStages = (D == 128) ? 4 : 8;    // K/V ring depth
   static constexpr int kOffQ = 0;                                    // Q_0, Q_1
   static constexpr int kOffKV = 2 * kTileBytes;                      // K/V ring
-  static constexpr int kOffO = kOffKV + kStages * kTileBytes;        // O staging, one per tile
-  static constexpr int kOffBar = kOffO + 2 * kTileBytes;
+  static constexpr int kOffO = kOffKV + kStages * kTileBytes;        // O staging, shared by the tiles
+  static constexpr int kOffBar = kOffO + kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // +1024: manual 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
@@ -87,10 +87,11 @@ struct PrefillCfg {
   static constexpr int kBarClc = 11;       // [1] launch-control response landed
   static constexpr int kBarUnitFull = 12;  // [2] unit ring slot written
   static constexpr int kBarUnitEmpty = 14; // [2] unit ring slot read by every reader warp
-  static constexpr int kBarKVFull = 16;    // [kStages]
-  static constexpr int kBarKVEmpty = 16 + kStages;
-  static constexpr int kBarVConv = 16 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
-  static constexpr int kNumBars = 16 + 3 * kStages;
+  static constexpr int kBarOStage = 16;    // [2] tile t's turn with the O staging buffer is over
+  static constexpr int kBarKVFull = 18;    // [kStages]
+  static constexpr int kBarKVEmpty = 18 + kStages;
+  static constexpr int kBarVConv = 18 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
+  static constexpr int kNumBars = 18 + 3 * kStages;
   static constexpr int kOffMisc = kNumBars * 8;  // tmem slot, abort flag, unit slots[2]
   static constexpr int kOffClc = ((kOffMisc + 16 + 15) / 16) * 16;  // 16-byte launch-control response
   static_assert(kOffClc + 16 <= kBarBytes, "barrier area too small");
@@ -153,7 +154,7 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
 // exponentials of one K/V step need as many MUFU cycles as its four MMAs need
 // tensor cycles, so moving a share of them to the FMA pipe shortens the softmax.
 #ifndef ATTN_EXP_EMU_PERIOD
-#define ATTN_EXP_EMU_PERIOD 0
+#define ATTN_EXP_EMU_PERIOD 4
 #endif
 
 // Max over one 64-column half of an S row (columns 64*kHalf + c), sign-flipped for a
@@ -231,7 +232,7 @@ __device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float
 // unit into g_prefill_trace, read back with attn_trace_read().  Compiled out otherwise.
 #ifdef ATTN_TRACE
 constexpr int kTraceCtas = 4;
-constexpr int kTraceSlots = 1024;
+constexpr int kTraceSlots = 2048;
 __device__ long long g_prefill_trace[kTraceCtas][kTraceSlots];
 #define ATTN_TRACE_POINT(slot)                                                        \
   do {                                                                                \
@@ -246,7 +247,9 @@ __device__ long long g_prefill_trace[kTraceCtas][kTraceSlots];
 // trace slot layout (first unit only): 0 start; 1 + 64*t + j: MMA saw P_t(j) ready;
 // 129 + 64*t + j: MMA issued S_t(j+1); 257 + 64*t + j: softmax t saw S_t(j);
 // 385 + ...: S loaded; 513 + ...: max done; 641 + ...: P computed; 769 + ...: P ready
-// arrived; 897 + i: producer issued ring item i.
+// arrived; 897 + i: producer issued ring item i.  Per unit k < 64 (all units):
+// 1024 + k: MMA read unit k; 1088 + k: MMA issued its first S; 1152 + 64*t + k: softmax t
+// read unit k; 1280 + 64*t + k: softmax t saw O_t final; 1408 + 64*t + k: softmax t epilogue done.
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
@@ -278,6 +281,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       mbar_init(BAR(C::kBarOFull + i), 1);
       mbar_init(BAR(C::kBarUnitFull + i), 1);
       mbar_init(BAR(C::kBarUnitEmpty + i), C::kUnitReaders);
+      mbar_init(BAR(C::kBarOStage + i), 1);
     }
     mbar_init(BAR(C::kBarMmaDone), 1);
     mbar_init(BAR(C::kBarClc), 1);
@@ -422,6 +426,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     for (int k = 0;; ++k) {
       const int unit = next_unit(k);
       if (unit < 0) break;
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1024 + k);
       const PrefillUnit u = prefill_unit(p, unit);
       if (u.nmax == 0) continue;
       for (int t = 0; t < 2; ++t)
@@ -437,6 +442,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tc_commit_w(BAR(C::kBarSFull + t));
             if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
           }
+        if (lane == 0 && k < 64) ATTN_TRACE_POINT(1088 + k);
         tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
       }
       for (int j = 0; j < u.nmax; ++j) {
@@ -535,17 +541,28 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     const bool neg = cs < 0.f;
     const float cs_abs = fabsf(cs);
     const long long diag = (long long)p.Nk - p.Nq;
-    uint8_t* ostage = smem + C::kOffO + t * C::kTileBytes;
+    uint8_t* ostage = smem + C::kOffO;
+    // The two tiles take turns with the one O staging buffer, in the order tile 0 of
+    // unit 0, tile 1 of unit 0, tile 0 of unit 1, ...: a turn starts when the previous
+    // turn's TMA store has finished reading the buffer (an inactive tile passes its turn).
+    auto ostage_acquire = [&](int k) {
+      if (t == 0 && k > 0) mbar_wait(BAR(C::kBarOStage + 1), (k - 1) & 1, wctx);
+      if (t == 1) mbar_wait(BAR(C::kBarOStage + 0), k & 1, wctx);
+      __syncwarp();
+    };
     int ns = 0;  // S tiles consumed (s_full phases)
     int no = 0;  // units finished (o_full phases)
     for (int k = 0;; ++k) {
       const int unit = next_unit(k);
       if (unit < 0) break;
+      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1152 + 64 * t + k);
       const PrefillUnit u = prefill_unit(p, unit);
       const int row0 = u.row0[t];
       const int nkv = u.nkv[t];
       const int grow = row0 + r;  // global query row
       if (nkv == 0) {
+        ostage_acquire(k);  // pass this tile's turn with the staging buffer
+        if (threadIdx.x == 128 * t) mbar_arrive(BAR(C::kBarOStage + t));
         // every row of this tile is left without a key (causal, Nq > Nk): O = 0, lse = -inf
         if (row0 < p.Nq && grow < p.Nq) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
@@ -649,8 +666,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       mbar_wait(BAR(C::kBarOFull + t), no & 1, wctx);
       ++no;
       __syncwarp();
+      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1280 + 64 * t + k);
       tc_fence_after_sync();
-      named_bar_sync(1 + t, 128);  // the previous store from this staging buffer has read it
+      ostage_acquire(k);  // the previous store from the staging buffer has read it
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -674,16 +692,19 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       named_bar_sync(1 + t, 128);
       if (r == 0 && !*abort_flag) {
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_store_4d(&p.tm_o, sbase + C::kOffO + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64,
-                       u.h, row0, u.b);
+          tma_store_4d(&p.tm_o, sbase + C::kOffO + bx * C::kBoxBytes, bx * 64, u.h, row0, u.b);
         bulk_commit_group();
+      }
+      if (r == 0) {
         bulk_wait_group_read0();
+        mbar_arrive(BAR(C::kBarOStage + t));  // hand the staging buffer to the other tile
       }
       if (p.lse != nullptr && grow < p.Nq) {
         const float lse = l_run > 0.f ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                       : -INFINITY;
         p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
       }
+      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1408 + 64 * t + k);
     }
   }
 

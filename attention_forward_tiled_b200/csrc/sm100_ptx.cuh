@@ -197,17 +197,24 @@ struct WaitCtx {
 // gives up after timeout_ns (wall clock, %globaltimer) or once any thread of the
 // CTA has raised the abort flag.  Returns false on give-up; the first thread
 // that times out records kStatusTimeout in the status word and raises the flag.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The first poll is inline; the polling loop is out of line with its arguments in
+// registers.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            int* status, uint64_t timeout_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0; it < (1u << 26); ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*w.abort_flag) return false;
-    if (global_timer_ns() - t0 > w.timeout_ns) break;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > timeout_ns) break;
   }
-  *w.abort_flag = 1;
-  atomicCAS(w.status, 0, kStatusTimeout);
+  *abort_flag = 1;
+  atomicCAS(status, 0, kStatusTimeout);
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, w.abort_flag, w.status, w.timeout_ns);
 }
 
 // Drain wait used on the way out after an abort: ignores the abort flag but is
