@@ -1,0 +1,62 @@
+"""Multi-rank logic of the benchmark on CPU (gloo, world size 2).
+
+The forward has no data-path collective (every (b, h) row is independent), so the
+only cross-rank steps are the barrier around the timed region and the max over
+ranks of the elapsed time; the reference arm runs on rank 0 only.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        elapsed = 10.0 + 5.0 * rank  # each rank's own timed region (ms)
+        m = bench.max_over_ranks(elapsed, world, device="cpu")
+        w, r, lr = bench.dist_setup(None)
+        q.put((rank, m, w, r, lr))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_barrier_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    assert [g[1] for g in got] == [15.0, 15.0]          # both ranks see the slowest rank's time
+    assert [(g[2], g[3], g[4]) for g in got] == [(2, 0, 0), (2, 1, 1)]
+
+
+def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+
+    class A:
+        workload, steps, warmup = "tiny", 1, 3
+
+    bench.run_reference(A())        # rank 1: returns at once, prints nothing
+    assert capsys.readouterr().out == ""
