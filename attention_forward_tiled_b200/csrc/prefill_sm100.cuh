@@ -20,21 +20,26 @@
 //     swizzle), each stage guarded by a full/empty mbarrier pair;
 //   * warp 9, MMA issuer (whole warp, one elected lane issues) runs tcgen05.mma:
 //       S_t = Q_t K_j^T   (A, B from shared memory, fp32 accumulator in TMEM)
-//       O_t += P_t V_j    (A = P from TMEM, B = V from shared memory)
-//     alternating the two Q tiles so one tile's softmax overlaps the other
-//     tile's matrix multiplies;
+//       O_t += P_t V_j    (A = P_t from TMEM, B = V from shared memory)
+//     alternating the two Q tiles so one tile's softmax overlaps the other tile's
+//     matrix multiplies.  d = 128: P_t is written over the consumed S_t columns, so
+//     S_t(j+1) follows P_t(j) V_j.  d = 64: TMEM has room for separate P buffers, so
+//     S_t(j+1) is issued as soon as the softmax has read S_t(j) and is computed while
+//     that softmax runs;
 //   * warps 10-11 (bf16 inputs only) convert each V tile to fp16 in place, so
 //     P V runs with P in fp16 (11-bit significand) rather than bf16 (8-bit);
 //   * warps 0-3 and 4-7, softmax warpgroups (one per Q tile, one thread per query
-//     row): read the 128-column S row from TMEM, apply the tail/causal mask,
-//     update the running max m and sum l (base-2 exponent with scale*log2(e)
+//     row): read the 128-column S row from TMEM, release it, apply the tail/causal
+//     mask, update the running max m and sum l (base-2 exponent with scale*log2(e)
 //     folded into one packed FMA, lazy rescale of O only when the max grows by more
-//     than 2^8), write P back to TMEM as fp16 over the consumed S columns, and at
-//     the end of the unit normalise O by 1/l, stage it in shared memory, store it
-//     with TMA and write the row LSE.
+//     than 2^8), write P as fp16 into TMEM, and at the end of the unit normalise O
+//     by 1/l, stage it in shared memory, store it with TMA and write the row LSE.
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).  P_t occupies columns [64,128) of S_t.
+// O_1 [256+D, 256+2D); P_t in columns [64,128) of S_t (d = 128) or in its own
+// columns P_0 [384,448), P_1 [448,512) (d = 64).
+// Shared memory: Q_0, Q_1 | K/V ring | O staging (one buffer the two tiles take
+// turns with for d = 128, one per tile for d = 64).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -61,17 +66,22 @@ struct PrefillParams {
 template <int D>
 struct PrefillCfg {
   static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
-  static constexpr int kBoxBytes = 128 * 128;          // 128 rows x 64 elements x 2 bytes
+  // d = 64: separate P columns in TMEM, S released as soon as the softmax has read it.
+  // d = 128: TMEM is full (2 S + 2 O tiles = 512 columns), P aliases the consumed S columns.
+  static constexpr bool kDecoupled = (D == 64);
+  static constexpr int kBoxBytes = 128 * 128;            // 128 rows x 64 elements x 2 bytes
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row Q, K, V or O tile
   static constexpr int kStages = (D == 128) ? 4 : 8;    // K/V ring depth
+  static constexpr int kNumOStage = kDecoupled ? 2 : 1;  // O staging buffers
   static constexpr int kOffQ = 0;                                    // Q_0, Q_1
   static constexpr int kOffKV = 2 * kTileBytes;                      // K/V ring
-  static constexpr int kOffO = kOffKV + kStages * kTileBytes;        // O staging, shared by the tiles
-  static constexpr int kOffBar = kOffO + kTileBytes;
+  static constexpr int kOffO = kOffKV + kStages * kTileBytes;        // O staging
+  static constexpr int kOffBar = kOffO + kNumOStage * kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // +1024: manual 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColP = 384;  // d = 64: P_t at kColP + 64 t
   static constexpr int kThreads = 384;
   static constexpr int kProducerWarp = 8;
   static constexpr int kMmaWarp = 9;
@@ -81,17 +91,18 @@ struct PrefillCfg {
   static constexpr int kBarQFull = 0;      // [2] Q_t landed
   static constexpr int kBarQEmpty = 2;     // [2] last S_t of the unit done: Q_t buffer free
   static constexpr int kBarSFull = 4;      // [2] S_t in TMEM
-  static constexpr int kBarPReady = 6;     // [2] P_t in TMEM (and O_t rescaled)
-  static constexpr int kBarOFull = 8;      // [2] last P_t V of the unit done
-  static constexpr int kBarMmaDone = 10;   // [1] teardown
-  static constexpr int kBarClc = 11;       // [1] launch-control response landed
-  static constexpr int kBarUnitFull = 12;  // [2] unit ring slot written
-  static constexpr int kBarUnitEmpty = 14; // [2] unit ring slot read by every reader warp
-  static constexpr int kBarOStage = 16;    // [2] tile t's turn with the O staging buffer is over
-  static constexpr int kBarKVFull = 18;    // [kStages]
-  static constexpr int kBarKVEmpty = 18 + kStages;
-  static constexpr int kBarVConv = 18 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
-  static constexpr int kNumBars = 18 + 3 * kStages;
+  static constexpr int kBarSFree = 6;      // [2] (d = 64) the softmax has read S_t (4 warps)
+  static constexpr int kBarPFull = 8;      // [2] P_t written and O_t rescaled (4 warps)
+  static constexpr int kBarPVDone = 10;    // [2] d = 64: every P_t V done; d = 128: the unit's last one
+  static constexpr int kBarOStage = 12;    // [2] (d = 128) tile t's turn with the O staging buffer is over
+  static constexpr int kBarMmaDone = 14;   // [1] teardown
+  static constexpr int kBarClc = 15;       // [1] launch-control response landed
+  static constexpr int kBarUnitFull = 16;  // [2] unit ring slot written
+  static constexpr int kBarUnitEmpty = 18; // [2] unit ring slot read by every reader warp
+  static constexpr int kBarKVFull = 20;    // [kStages]
+  static constexpr int kBarKVEmpty = 20 + kStages;
+  static constexpr int kBarVConv = 20 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
+  static constexpr int kNumBars = 20 + 3 * kStages;
   static constexpr int kOffMisc = kNumBars * 8;  // tmem slot, abort flag, unit slots[2]
   static constexpr int kOffClc = ((kOffMisc + 16 + 15) / 16) * 16;  // 16-byte launch-control response
   static_assert(kOffClc + 16 <= kBarBytes, "barrier area too small");
@@ -227,6 +238,79 @@ __device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float
   }
 }
 
+// Max over the 128 scores of an S row (sign-flipped for a negative scale),
+// restricted to columns < lim when kMask; four 3-input max chains.
+template <bool kMask, bool kNeg>
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32], int lim) {
+  float m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 128; c += 2) {
+    float s0 = __uint_as_float(sr[c >> 5][c & 31]);
+    float s1 = __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]);
+    if (kNeg) {
+      s0 = -s0;
+      s1 = -s1;
+    }
+    if (kMask) {
+      s0 = c < lim ? s0 : -INFINITY;
+      s1 = c + 1 < lim ? s1 : -INFINITY;
+    }
+    m[(c >> 1) & 3] = fmax3(m[(c >> 1) & 3], s0, s1);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p for the column pair (c, c+1): 2^(cs * s - m_use); the FMA-pipe polynomial for every
+// ATTN_EXP_EMU_PERIOD-th pair, MUFU ex2 otherwise; 0 at columns >= lim when kMask.
+template <bool kMask>
+__device__ __forceinline__ float2 pair_exp(const uint32_t (&sr)[4][32], int c, uint64_t cs2,
+                                           uint64_t negm2, int lim) {
+  const uint64_t x2 = f2_fma(f2_make(__uint_as_float(sr[c >> 5][c & 31]),
+                                     __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31])),
+                             cs2, negm2);
+  float2 pp;
+  if (!kMask && ATTN_EXP_EMU_PERIOD > 0 &&
+      ((c >> 1) % (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD : 1)) ==
+          (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD - 1 : 0)) {
+    pp = exp2_poly2(x2);
+  } else {
+    const float2 x = f2_split(x2);
+    pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+  }
+  if (kMask) {
+    pp.x = c < lim ? pp.x : 0.f;
+    pp.y = c + 1 < lim ? pp.y : 0.f;
+  }
+  return pp;
+}
+
+// The 128 p values of the row, packed to fp16 pairs, stored into 64 TMEM columns at
+// tP (lane = row) in four 16-column pieces.  Returns the row sum.
+template <bool kMask>
+__device__ __forceinline__ float row_exp_to_tmem(const uint32_t (&sr)[4][32], float cs, float m_use,
+                                                 int lim, uint32_t tP) {
+  const uint64_t cs2 = f2_make(cs, cs), negm2 = f2_make(-m_use, -m_use);
+  uint64_t acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
+#pragma unroll
+  for (int q32 = 0; q32 < 4; ++q32) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = q32 * 32 + 2 * i;
+      const float2 pp = pair_exp<kMask>(sr, c, cs2, negm2, lim);
+      acc[i & 3] = f2_add(acc[i & 3], f2_make(pp.x, pp.y));
+      w[i] = pack2<false>(pp.x, pp.y);
+    }
+    tmem_st16(tP + q32 * 16, w);
+  }
+  const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
+  return a.x + a.y;
+}
+
 // Optional timeline instrumentation (build with -DATTN_TRACE): the first
 // kTraceCtas CTAs record clock64() at fixed points of every role of their first
 // unit into g_prefill_trace, read back with attn_trace_read().  Compiled out otherwise.
@@ -277,8 +361,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       mbar_init(BAR(C::kBarQFull + i), 1);
       mbar_init(BAR(C::kBarQEmpty + i), 1);
       mbar_init(BAR(C::kBarSFull + i), 1);
-      mbar_init(BAR(C::kBarPReady + i), 4);  // one arrive per softmax warp
-      mbar_init(BAR(C::kBarOFull + i), 1);
+      mbar_init(BAR(C::kBarSFree + i), 4);  // one arrive per softmax warp
+      mbar_init(BAR(C::kBarPFull + i), 4);  // one arrive per softmax warp
+      mbar_init(BAR(C::kBarPVDone + i), 1);
       mbar_init(BAR(C::kBarUnitFull + i), 1);
       mbar_init(BAR(C::kBarUnitEmpty + i), C::kUnitReaders);
       mbar_init(BAR(C::kBarOStage + i), 1);
@@ -392,6 +477,112 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       __syncwarp();
     }
   } else if (warp == C::kMmaWarp) {
+    if constexpr (C::kDecoupled) {
+    // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
+    constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
+    // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
+    constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
+    const uint32_t colS[2] = {0u, 128u};
+    const uint32_t colO[2] = {256u, 256u + D};
+    const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+    // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
+    auto issue_s = [&](int t, uint32_t sK) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+        mma_f16_ss_w(tmem + colS[t], make_sdesc_sw128(sQ[t] + off, 16, 1024),
+                     make_sdesc_sw128(sK + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+      }
+    };
+    // O_t += P_t V_j over 8 k-steps of 16 keys; P_t in its own TMEM columns.
+    auto issue_pv = [&](int t, uint32_t sV, bool accumulate_first) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t bdesc = make_sdesc_sw128(sV + kk * 2048, C::kBoxBytes, 1024);
+        const uint32_t acc = (accumulate_first || kk > 0) ? 1u : 0u;
+        mma_f16_ts_w(tmem + colO[t], tmem + C::kColP + 64 * t + kk * 8, bdesc, idesc_o, acc);
+      }
+    };
+    auto stage_addr = [&](int item) -> uint32_t {
+      return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;
+    };
+    int nq[2] = {0, 0};   // units seen per tile (q_full / q_empty phases)
+    int nsf[2] = {0, 0};  // S tiles released by the softmax (s_free phases)
+    int npf[2] = {0, 0};  // P tiles written by the softmax (p_full phases)
+    int g = 0;            // ring items consumed
+    for (int k = 0;; ++k) {
+      const int unit = next_unit(k);
+      if (unit < 0) break;
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1024 + k);
+      const PrefillUnit u = prefill_unit(p, unit);
+      if (u.nmax == 0) continue;
+      for (int t = 0; t < 2; ++t)
+        if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
+      // prologue: S_t(0) for both tiles from K_0
+      mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      if (!warp_flag(abort_flag)) {
+        for (int t = 0; t < 2; ++t)
+          if (u.nkv[t] > 0) {
+            issue_s(t, stage_addr(g));
+            tc_commit_w(BAR(C::kBarSFull + t));
+            if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
+          }
+        tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
+      }
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1088 + k);
+      for (int j = 0; j < u.nmax; ++j) {
+        // next score tiles: S_t(j+1) as soon as the softmax has read S_t(j) out of TMEM
+        const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
+        bool k_ready = false;
+        for (int t = 0; t < 2; ++t) {
+          if (j >= u.nkv[t]) continue;
+          mbar_wait(BAR(C::kBarSFree + t), nsf[t] & 1, wctx);
+          ++nsf[t];
+          __syncwarp();
+          if (j + 1 < u.nkv[t]) {
+            if (!k_ready) {
+              mbar_wait(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
+              __syncwarp();
+              k_ready = true;
+            }
+            tc_fence_after_sync();
+            if (warp_flag(abort_flag)) continue;
+            issue_s(t, stage_addr(ik));
+            tc_commit_w(BAR(C::kBarSFull + t));
+            if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
+            if (lane == 0 && k == 0) ATTN_TRACE_POINT(129 + 64 * t + j);
+          }
+        }
+        if (k_ready && !warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
+        // O_t += P_t(j) V_j once the softmax has written P_t(j)
+        const int iv = g + 2 * j + 1;  // ring item of V_j
+        mbar_wait(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + iv % C::kStages), (iv / C::kStages) & 1,
+                  wctx);
+        __syncwarp();
+        for (int t = 0; t < 2; ++t) {
+          if (j >= u.nkv[t]) continue;
+          mbar_wait(BAR(C::kBarPFull + t), npf[t] & 1, wctx);
+          ++npf[t];
+          __syncwarp();
+          if (lane == 0 && k == 0) ATTN_TRACE_POINT(1 + 64 * t + j);
+          tc_fence_after_sync();
+          if (warp_flag(abort_flag)) continue;
+          issue_pv(t, stage_addr(iv), j > 0);
+          tc_commit_w(BAR(C::kBarPVDone + t));
+        }
+        if (!warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + iv % C::kStages));
+      }
+      g += 2 * u.nmax;
+      for (int t = 0; t < 2; ++t)
+        if (u.nkv[t] > 0) ++nq[t];
+    }
+    // every MMA (and every commit arrive) has landed before TMEM is released
+    tc_commit_w(BAR(C::kBarMmaDone));
+    mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+    __syncwarp();
+    } else {
     // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
     constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
     // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
@@ -454,7 +645,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= u.nkv[t]) continue;
-          mbar_wait(BAR(C::kBarPReady + t), np[t] & 1, wctx);
+          mbar_wait(BAR(C::kBarPFull + t), np[t] & 1, wctx);
           ++np[t];
           __syncwarp();
           if (lane == 0 && k == 0) ATTN_TRACE_POINT(1 + 64 * t + j);
@@ -473,7 +664,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
             if (lane == 0 && k == 0) ATTN_TRACE_POINT(129 + 64 * t + j);
           } else {
-            tc_commit_w(BAR(C::kBarOFull + t));
+            tc_commit_w(BAR(C::kBarPVDone + t));
           }
         }
         if (!warp_flag(abort_flag)) {
@@ -489,6 +680,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     tc_commit_w(BAR(C::kBarMmaDone));
     mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
     __syncwarp();
+    }
   } else if (warp >= C::kConvWarp0) {
     // ======================= bf16 -> fp16 conversion of V tiles (bf16 inputs) ======
     // Walks every ring item in order: waits for it to land, converts it if it is a V
@@ -530,6 +722,160 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       g += 2 * u.nmax;
     }
   } else {
+    if constexpr (C::kDecoupled) {
+    // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ======
+    const int t = warp >> 2;
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;  // row inside the Q tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (t ? 128u : 0u);
+    const uint32_t tO = tmem + lane_base + (t ? 256u + D : 256u);
+    const uint32_t tP = tmem + lane_base + C::kColP + 64u * t;  // d = 64 only
+    const float cs = p.scale_log2;
+    const bool neg = cs < 0.f;
+    const float cs_abs = fabsf(cs);
+    const long long diag = (long long)p.Nk - p.Nq;
+    uint8_t* ptile = smem + C::kOffO + t * C::kTileBytes;  // O staging of tile t
+    int ns = 0;   // S tiles consumed (s_full phases)
+    int npv = 0;  // P V operations of this tile completed before the current unit (pv_done phases)
+    for (int k = 0;; ++k) {
+      const int unit = next_unit(k);
+      if (unit < 0) break;
+      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1152 + 64 * t + k);
+      const PrefillUnit u = prefill_unit(p, unit);
+      const int row0 = u.row0[t];
+      const int nkv = u.nkv[t];
+      const int grow = row0 + r;  // global query row
+      if (nkv == 0) {
+        // every row of this tile is left without a key (causal, Nq > Nk): O = 0, lse = -inf
+        if (row0 < p.Nq && grow < p.Nq) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
+                                                ((((long long)u.b * p.Nq + grow) * p.H + u.h) * D) * 2);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (p.lse != nullptr) p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = -INFINITY;
+        }
+        continue;
+      }
+
+      float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazy: may lag the true max by <= 8)
+      float l_run = 0.f;        // running sum of 2^(cs*s - m_run)
+      for (int j = 0; j < nkv; ++j) {
+        mbar_wait(BAR(C::kBarSFull + t), ns & 1, wctx);
+        ++ns;
+        __syncwarp();  // lanes may leave the bounded wait on different polls
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(257 + 64 * t + j);
+        tc_fence_after_sync();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_order_after_wait(sr[c]);
+        // S_t is in registers: the tensor core may compute S_t(j+1) into the same columns
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::kBarSFree + t));
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(385 + 64 * t + j);
+
+        // mask needed on the key tail and on tiles crossing the causal diagonal
+        const long long key0 = (long long)j * 128;
+        const bool need_mask = (key0 + 128 > p.Nk) ||
+                               (p.causal && key0 + 127 > (long long)row0 + diag);
+        int lim = 128;  // keys [key0, key0+lim) are allowed for this row
+        if (need_mask) {
+          long long l = (long long)p.Nk;
+          if (p.causal) l = min(l, (long long)grow + diag + 1);
+          l -= key0;
+          lim = (int)max(0LL, min(128LL, l));
+        }
+        const float mx = need_mask ? (neg ? row_max<true, true>(sr, lim) : row_max<true, false>(sr, lim))
+                                   : (neg ? row_max<false, true>(sr, lim) : row_max<false, false>(sr, lim));
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(513 + 64 * t + j);
+        const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cs_abs;
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool rescale = m_new > m_run + 8.0f;
+        const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
+        if (rescale) {
+          m_run = m_new;
+          l_run *= alpha;
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+
+        if (j > 0) {
+          // P_t(j-1) V must be done: its P buffer is about to be overwritten and O_t may be rescaled
+          mbar_wait(BAR(C::kBarPVDone + t), (npv + j - 1) & 1, wctx);
+          __syncwarp();
+          tc_fence_after_sync();
+          if (__any_sync(0xffffffffu, rescale)) {  // lazy rescale of O (rare after the first tiles)
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_ld_wait();
+              reg_order_after_wait(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+        }
+
+        l_run += need_mask ? row_exp_to_tmem<true>(sr, cs, m_use, lim, tP)
+                           : row_exp_to_tmem<false>(sr, cs, m_use, lim, tP);
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
+      }
+
+      // ---- epilogue: O / l -> 16-bit -> swizzled staging (this tile's buffer) -> TMA store
+      mbar_wait(BAR(C::kBarPVDone + t), (npv + nkv - 1) & 1, wctx);
+      npv += nkv;
+      __syncwarp();
+      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1280 + 64 * t + k);
+      tc_fence_after_sync();
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_ld_wait();
+        reg_order_after_wait(o);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {  // four 16-byte chunks of 8 elements
+          uint4 w;
+          w.x = pack2<BF16>(__uint_as_float(o[q4 * 8 + 0]) * inv_l, __uint_as_float(o[q4 * 8 + 1]) * inv_l);
+          w.y = pack2<BF16>(__uint_as_float(o[q4 * 8 + 2]) * inv_l, __uint_as_float(o[q4 * 8 + 3]) * inv_l);
+          w.z = pack2<BF16>(__uint_as_float(o[q4 * 8 + 4]) * inv_l, __uint_as_float(o[q4 * 8 + 5]) * inv_l);
+          w.w = pack2<BF16>(__uint_as_float(o[q4 * 8 + 6]) * inv_l, __uint_as_float(o[q4 * 8 + 7]) * inv_l);
+          const int chunk = c * 4 + q4;  // 16-byte chunk index along the row
+          const int bx = chunk >> 3, cc = chunk & 7;
+          *reinterpret_cast<uint4*>(ptile + bx * C::kBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (r == 0) {
+        if (!*abort_flag) {
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_store_4d(&p.tm_o, sbase + C::kOffO + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64,
+                         u.h, row0, u.b);
+          bulk_commit_group();
+        }
+        bulk_wait_group_read0();
+      }
+      if (p.lse != nullptr && grow < p.Nq) {
+        const float lse = l_run > 0.f ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
+                                      : -INFINITY;
+        p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
+      }
+      named_bar_sync(1 + t, 128);  // the staging buffer is free again for the next unit
+      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1408 + 64 * t + k);
+    }
+    } else {
     // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ======
     const int t = warp >> 2;
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
@@ -658,12 +1004,12 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(C::kBarPReady + t));
+        if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
         if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
       }
 
       // ---- epilogue: O / l -> 16-bit -> swizzled staging buffer -> TMA store
-      mbar_wait(BAR(C::kBarOFull + t), no & 1, wctx);
+      mbar_wait(BAR(C::kBarPVDone + t), no & 1, wctx);
       ++no;
       __syncwarp();
       if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1280 + 64 * t + k);
@@ -705,6 +1051,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
       }
       if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1408 + 64 * t + k);
+    }
     }
   }
 
