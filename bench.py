@@ -90,7 +90,7 @@ class ClockSampler(threading.Thread):
         "nvmlClocksEventReasonHwPowerBrakeSlowdown": "hw_power_brake_slowdown",
     }
 
-    def __init__(self, device_index, period_s=0.002):
+    def __init__(self, device_index, period_s=0.0005):
         super().__init__(daemon=True)
         self.period = period_s
         self.samples = []
@@ -300,7 +300,7 @@ def measure_workload(name, K, W, world, device, peaks, want_e2e=True):
     return res
 
 
-def cpu_baseline_sample(name, budget_s=12.0):
+def cpu_baseline_sample(name, budget_s=20.0):
     """Time the oracle, as it stands, on a bounded sample of the workload (rank 0, host cores)."""
     import oracle
     from attention_forward_tiled_b200.inputs import WORKLOADS, make_inputs
