@@ -35,7 +35,13 @@ namespace {
 constexpr int kVersion = 10000;  // 1.0.0
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 constexpr int kMaxDevices = 64;
-constexpr int kHeadsPerGroup = 8;  // prefill scheduling group (K/V of 8 heads stay in L2)
+// Prefill scheduling group: units of 16 heads are handed out together (heaviest causal
+// units first), so the K/V being read stay in L2 (16 heads x 4096 keys x d 128 x 2 x 2 B
+// = 32 MB) while the group is long enough to even out the causal unit sizes over SMs.
+#ifndef ATTN_HEADS_PER_GROUP
+#define ATTN_HEADS_PER_GROUP 16
+#endif
+constexpr int kHeadsPerGroup = ATTN_HEADS_PER_GROUP;
 
 std::atomic<int> g_inject{0};
 std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
@@ -436,6 +442,10 @@ int attn_version(void) { return kVersion; }
 ATTN_API int attn_trace_read(void* dst, unsigned long long bytes) {
   if (bytes > sizeof(g_prefill_trace)) bytes = sizeof(g_prefill_trace);
   return cudaMemcpyFromSymbol(dst, g_prefill_trace, bytes) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+ATTN_API int attn_trace_spans(void* dst, unsigned long long bytes) {
+  if (bytes > sizeof(g_cta_span)) bytes = sizeof(g_cta_span);
+  return cudaMemcpyFromSymbol(dst, g_cta_span, bytes) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 #endif
 

@@ -63,6 +63,8 @@ struct PrefillParams {
   unsigned long long timeout_ns;
 };
 
+constexpr int kUnitInts = 8;  // ints per published work unit (PrefillUnit)
+
 template <int D>
 struct PrefillCfg {
   static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
@@ -73,6 +75,11 @@ struct PrefillCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row Q, K, V or O tile
   static constexpr int kStages = (D == 128) ? 4 : 8;    // K/V ring depth
+#ifdef ATTN_CLAIM_LEAD
+  static constexpr int kClaimLead = ATTN_CLAIM_LEAD;
+#else
+  static constexpr int kClaimLead = 2 * kStages;  // ring items before a unit's last load
+#endif
   static constexpr int kNumOStage = kDecoupled ? 2 : 1;  // O staging buffers
   static constexpr int kOffQ = 0;                                    // Q_0, Q_1
   static constexpr int kOffKV = 2 * kTileBytes;                      // K/V ring
@@ -92,19 +99,23 @@ struct PrefillCfg {
   static constexpr int kBarQEmpty = 2;     // [2] last S_t of the unit done: Q_t buffer free
   static constexpr int kBarSFull = 4;      // [2] S_t in TMEM
   static constexpr int kBarSFree = 6;      // [2] (d = 64) the softmax has read S_t (4 warps)
-  static constexpr int kBarPFull = 8;      // [2] P_t written and O_t rescaled (4 warps)
+  static constexpr int kBarPFull = 8;      // [2] P_t written (d = 128: keys 0..63 last), O_t rescaled (4 warps)
   static constexpr int kBarPVDone = 10;    // [2] d = 64: every P_t V done; d = 128: the unit's last one
   static constexpr int kBarOStage = 12;    // [2] (d = 128) tile t's turn with the O staging buffer is over
   static constexpr int kBarMmaDone = 14;   // [1] teardown
   static constexpr int kBarClc = 15;       // [1] launch-control response landed
   static constexpr int kBarUnitFull = 16;  // [2] unit ring slot written
   static constexpr int kBarUnitEmpty = 18; // [2] unit ring slot read by every reader warp
-  static constexpr int kBarKVFull = 20;    // [kStages]
-  static constexpr int kBarKVEmpty = 20 + kStages;
-  static constexpr int kBarVConv = 20 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
-  static constexpr int kNumBars = 20 + 3 * kStages;
-  static constexpr int kOffMisc = kNumBars * 8;  // tmem slot, abort flag, unit slots[2]
-  static constexpr int kOffClc = ((kOffMisc + 16 + 15) / 16) * 16;  // 16-byte launch-control response
+  static constexpr int kBarOReady = 20;   // [2] tile t's rows are in its O staging buffer (4 warps)
+  static constexpr int kBarOFree = 22;    // [2] (d = 64) tile t's previous O store has read its buffer
+  static constexpr int kBarPHalf = 24;    // [2] (d = 128) P_t for keys 64..127 written, O_t rescaled (4 warps)
+  static constexpr int kBarKVFull = 26;    // [kStages]
+  static constexpr int kBarKVEmpty = 26 + kStages;
+  static constexpr int kBarVConv = 26 + 2 * kStages;  // [kStages] V tile converted (bf16 only)
+  static constexpr int kNumBars = 26 + 3 * kStages;
+  static constexpr int kOffMisc = kNumBars * 8;  // tmem slot, abort flag, pad, unit slots[2][kUnitInts]
+  static constexpr int kMiscBytes = 16 + 2 * kUnitInts * 4;
+  static constexpr int kOffClc = ((kOffMisc + kMiscBytes + 15) / 16) * 16;  // 16-byte launch-control response
   static_assert(kOffClc + 16 <= kBarBytes, "barrier area too small");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -124,32 +135,37 @@ __device__ __forceinline__ int prefill_kv_tiles(int row0, int Nq, int Nk, int ca
 
 // Work unit index -> (b, h, Q-tile rows, K/V tile counts).  Units run in groups of
 // `group_heads` heads; inside a group, causal units go heaviest (last Q rows) first.
+// The producer decodes each unit once and publishes the result to the other roles.
 struct PrefillUnit {
+  int id;  // unit index (-1: no more units)
   int b, h;
   int row0[2];
   int nkv[2];
   int nmax;
 };
 
+// All quantities fit in 32 bits: the launcher rejects grids of 2^31 units or more.
 __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int unit) {
   const int BH = p.B * p.H;
   const int nqp = p.n_qpairs;
   const int G = p.group_heads;
-  const long long full_units = (long long)(BH / G) * G * nqp;
+  const int per_group = G * nqp;
+  const int full_units = (BH / G) * per_group;
   int g, idx, Gc;
   if (unit < full_units) {
-    g = (int)(unit / ((long long)G * nqp));
-    idx = (int)(unit - (long long)g * G * nqp);
+    g = unit / per_group;
+    idx = unit - g * per_group;
     Gc = G;
   } else {
     g = BH / G;
-    idx = (int)(unit - full_units);
+    idx = unit - full_units;
     Gc = BH - g * G;
   }
   const int qrank = idx / Gc;
   const int bh = g * G + (idx - qrank * Gc);
   const int qp = p.causal ? (nqp - 1 - qrank) : qrank;
   PrefillUnit u;
+  u.id = unit;
   u.b = bh / p.H;
   u.h = bh - u.b * p.H;
   u.row0[0] = qp * 256;
@@ -323,6 +339,8 @@ __device__ long long g_prefill_trace[kTraceCtas][kTraceSlots];
     if (blockIdx.x < kTraceCtas && (slot) < kTraceSlots)                              \
       g_prefill_trace[blockIdx.x][(slot)] = clock64();                                \
   } while (0)
+// per-CTA wall-clock span (globaltimer at start and end) and units done, first 4096 CTAs
+__device__ unsigned long long g_cta_span[4096][3];
 #else
 #define ATTN_TRACE_POINT(slot) \
   do {                         \
@@ -347,7 +365,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* unit_slot = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [2]
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(tmem_slot + 4);  // [2][kUnitInts]
   const uint32_t clc_resp = sbase + C::kOffBar + C::kOffClc;
   auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
 
@@ -367,6 +385,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       mbar_init(BAR(C::kBarUnitFull + i), 1);
       mbar_init(BAR(C::kBarUnitEmpty + i), C::kUnitReaders);
       mbar_init(BAR(C::kBarOStage + i), 1);
+      mbar_init(BAR(C::kBarOReady + i), 4);  // one arrive per softmax warp
+      mbar_init(BAR(C::kBarOFree + i), 1);
+      mbar_init(BAR(C::kBarPHalf + i), 4);  // one arrive per softmax warp
     }
     mbar_init(BAR(C::kBarMmaDone), 1);
     mbar_init(BAR(C::kBarClc), 1);
@@ -389,13 +410,26 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) ATTN_TRACE_POINT(0);
+#ifdef ATTN_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][0] = global_timer_ns();
+#endif
 
-  // Every role walks the same unit sequence, published by the producer.  Returns the
-  // k-th unit (-1 = no more) after this warp has read it and released its slot.
-  auto next_unit = [&](int k) -> int {
+  // Every role walks the same unit sequence, decoded and published by the producer.
+  // Returns the k-th unit (nmax < 0: no more) after this warp has read it and released
+  // its slot.
+  auto next_unit = [&](int k) -> PrefillUnit {
     mbar_wait(BAR(C::kBarUnitFull + (k & 1)), (k >> 1) & 1, wctx);
     __syncwarp();
-    const int u = __shfl_sync(0xffffffffu, unit_slot[k & 1], 0);
+    const volatile int* us = unit_slot + (k & 1) * kUnitInts;
+    PrefillUnit u;
+    u.id = us[0];
+    u.b = us[1];
+    u.h = us[2];
+    u.row0[0] = us[3];
+    u.row0[1] = us[4];
+    u.nkv[0] = us[5];
+    u.nkv[1] = us[6];
+    u.nmax = us[7];
     __syncwarp();
     if (lane == 0) mbar_arrive(BAR(C::kBarUnitEmpty + (k & 1)));
     return u;
@@ -418,20 +452,42 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     int g = 0;              // ring items issued
     int nclaim = 0;
     for (int k = 0;; ++k) {
+      PrefillUnit u;
+      if (unit >= 0) {
+        u = prefill_unit(p, unit);
+      } else {
+        u.id = -1;
+        u.b = u.h = u.row0[0] = u.row0[1] = u.nkv[0] = u.nkv[1] = 0;
+        u.nmax = -1;
+      }
       if (k >= 2) mbar_wait(BAR(C::kBarUnitEmpty + (k & 1)), ((k >> 1) - 1) & 1, wctx);
       __syncwarp();
       if (lane == 0) {
-        unit_slot[k & 1] = unit;
+        volatile int* us = unit_slot + (k & 1) * kUnitInts;
+        us[0] = u.id;
+        us[1] = u.b;
+        us[2] = u.h;
+        us[3] = u.row0[0];
+        us[4] = u.row0[1];
+        us[5] = u.nkv[0];
+        us[6] = u.nkv[1];
+        us[7] = u.nmax;
         mbar_arrive(BAR(C::kBarUnitFull + (k & 1)));
       }
       __syncwarp();
       if (unit < 0) break;
-      const bool claim = !warp_flag(abort_flag);
-      if (claim) {
-        mbar_arrive_expect_tx_w(BAR(C::kBarClc), 16);
-        clc_try_cancel_w(clc_resp, BAR(C::kBarClc));
-      }
-      const PrefillUnit u = prefill_unit(p, unit);
+      // The next unit is claimed late in this one (kClaimLead ring items before its last
+      // load), so units go to the CTAs that are about to run out of work: claiming a
+      // whole unit ahead leaves a tail of up to one long causal unit between SMs.
+      bool claimed = false;
+      const int claim_at = max(0, 2 * u.nmax - C::kClaimLead);
+      auto claim_next = [&]() {
+        if (!claimed && !warp_flag(abort_flag)) {
+          mbar_arrive_expect_tx_w(BAR(C::kBarClc), 16);
+          clc_try_cancel_w(clc_resp, BAR(C::kBarClc));
+          claimed = true;
+        }
+      };
       for (int t = 0; t < 2; ++t) {
         if (u.nkv[t] == 0) continue;
         if (nq[t] > 0) mbar_wait(BAR(C::kBarQEmpty + t), (nq[t] - 1) & 1, wctx);
@@ -442,10 +498,12 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tma_load_4d_w(sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
                           BAR(C::kBarQFull + t), bx * 64, u.h, u.row0[t], u.b);
           q_pending[t] = true;
+          if (lane == 0 && k < 64) ATTN_TRACE_POINT(1600 + 64 * t + k);
         }
         ++nq[t];
       }
       for (int i = 0; i < 2 * u.nmax; ++i, ++g) {
+        if (i == claim_at) claim_next();
         const int stage = g % C::kStages;
         const int round = g / C::kStages;
         if (round > 0) mbar_wait(BAR(C::kBarKVEmpty + stage), (round - 1) & 1, wctx);
@@ -457,9 +515,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
           tma_load_4d_w(sbase + C::kOffKV + stage * C::kTileBytes + bx * C::kBoxBytes, map,
                         BAR(C::kBarKVFull + stage), bx * 64, u.h, (i >> 1) * 128, u.b);
         if (lane == 0 && k == 0) ATTN_TRACE_POINT(897 + i);
+        if (lane == 0 && i == 0 && k < 64) ATTN_TRACE_POINT(1728 + k);
       }
+      claim_next();  // units without K/V tiles
       int next = -1;
-      if (claim) {
+      if (claimed) {
         if (mbar_wait(BAR(C::kBarClc), nclaim & 1, wctx)) next = clc_response_ctaid_x(clc_resp);
         else mbar_wait_drain(BAR(C::kBarClc), nclaim & 1, p.timeout_ns);
         ++nclaim;
@@ -511,15 +571,22 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     int npf[2] = {0, 0};  // P tiles written by the softmax (p_full phases)
     int g = 0;            // ring items consumed
     for (int k = 0;; ++k) {
-      const int unit = next_unit(k);
-      if (unit < 0) break;
+      const PrefillUnit u = next_unit(k);
+      if (u.nmax < 0) break;
       if (lane == 0 && k < 64) ATTN_TRACE_POINT(1024 + k);
-      const PrefillUnit u = prefill_unit(p, unit);
+#ifdef ATTN_TRACE
+      if (lane == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][2] = k + 1;
+#endif
+#ifdef ATTN_TRACE
+      if (lane == 0 && k < 64 && blockIdx.x < kTraceCtas) g_prefill_trace[blockIdx.x][1536 + k] = u.id;
+#endif
       if (u.nmax == 0) continue;
       for (int t = 0; t < 2; ++t)
         if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1792 + k);
       // prologue: S_t(0) for both tiles from K_0
       mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1856 + k);
       __syncwarp();
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
@@ -600,12 +667,14 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       }
     };
     // O_t += P_t V_j over 8 k-steps of 16 keys; P_t is in TMEM columns [64,128) of S_t.
-    auto issue_pv = [&](int t, uint32_t sV, bool accumulate_first) {
+    // k-steps kk0 .. kk0+3 of O_t += P_t V_j (keys 16*kk0 .. 16*kk0+63); the first k-step
+    // of the unit starts the accumulator.
+    auto issue_pv4 = [&](int t, uint32_t sV, int kk0, bool accumulate_first) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+      for (int kk = kk0; kk < kk0 + 4; ++kk) {
         mma_f16_ts_w(tmem + colO[t], tmem + colS[t] + 64 + kk * 8,
                      make_sdesc_sw128(sV + kk * 2048, C::kBoxBytes, 1024), idesc_o,
-                     (accumulate_first || kk > 0) ? 1u : 0u);
+                     (accumulate_first || kk > kk0) ? 1u : 0u);
       }
     };
     auto stage_addr = [&](int item) -> uint32_t {
@@ -615,15 +684,22 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     int np[2] = {0, 0};  // P tiles consumed per tile (p_ready phases)
     int g = 0;           // ring items consumed
     for (int k = 0;; ++k) {
-      const int unit = next_unit(k);
-      if (unit < 0) break;
+      const PrefillUnit u = next_unit(k);
+      if (u.nmax < 0) break;
       if (lane == 0 && k < 64) ATTN_TRACE_POINT(1024 + k);
-      const PrefillUnit u = prefill_unit(p, unit);
+#ifdef ATTN_TRACE
+      if (lane == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][2] = k + 1;
+#endif
+#ifdef ATTN_TRACE
+      if (lane == 0 && k < 64 && blockIdx.x < kTraceCtas) g_prefill_trace[blockIdx.x][1536 + k] = u.id;
+#endif
       if (u.nmax == 0) continue;
       for (int t = 0; t < 2; ++t)
         if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1792 + k);
       // prologue: S_t(0) for both tiles from K_0
       mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
+      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1856 + k);
       __syncwarp();
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
@@ -645,13 +721,18 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= u.nkv[t]) continue;
+          // keys 64..127 as soon as that half of P_t(j) is written, then keys 0..63
+          mbar_wait(BAR(C::kBarPHalf + t), np[t] & 1, wctx);
+          __syncwarp();
+          tc_fence_after_sync();
+          if (!warp_flag(abort_flag)) issue_pv4(t, stage_addr(iv), 4, j > 0);
           mbar_wait(BAR(C::kBarPFull + t), np[t] & 1, wctx);
           ++np[t];
           __syncwarp();
           if (lane == 0 && k == 0) ATTN_TRACE_POINT(1 + 64 * t + j);
           tc_fence_after_sync();
           if (warp_flag(abort_flag)) continue;
-          issue_pv(t, stage_addr(iv), j > 0);
+          issue_pv4(t, stage_addr(iv), 0, true);
           if (j + 1 < u.nkv[t]) {
             if (!k_ready) {
               mbar_wait(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
@@ -690,9 +771,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
     int g = 0;
     for (int k = 0;; ++k) {
-      const int unit = next_unit(k);
-      if (unit < 0) break;
-      const PrefillUnit u = prefill_unit(p, unit);
+      const PrefillUnit u = next_unit(k);
+      if (u.nmax < 0) break;
       if constexpr (BF16) {
         for (int i = 0; i < 2 * u.nmax; ++i) {
           const int item = g + i;
@@ -738,11 +818,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     uint8_t* ptile = smem + C::kOffO + t * C::kTileBytes;  // O staging of tile t
     int ns = 0;   // S tiles consumed (s_full phases)
     int npv = 0;  // P V operations of this tile completed before the current unit (pv_done phases)
+    int nout = 0;  // O tiles stored (o_free / o_ready phases)
     for (int k = 0;; ++k) {
-      const int unit = next_unit(k);
-      if (unit < 0) break;
+      const PrefillUnit u = next_unit(k);
+      if (u.nmax < 0) break;
       if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1152 + 64 * t + k);
-      const PrefillUnit u = prefill_unit(p, unit);
       const int row0 = u.row0[t];
       const int nkv = u.nkv[t];
       const int grow = row0 + r;  // global query row
@@ -838,43 +918,53 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1280 + 64 * t + k);
       tc_fence_after_sync();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-#pragma unroll 1
+      uint32_t o[D / 32][32];  // the whole O row: one TMEM round trip
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
+      // this tile's previous O store has read the staging buffer before it is rewritten
+      if (r == 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(BAR(C::kBarOFree + t));
+      }
+      mbar_wait(BAR(C::kBarOFree + t), nout & 1, wctx);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_order_after_wait(o[c]);
+#pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_ld_wait();
-        reg_order_after_wait(o);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {  // four 16-byte chunks of 8 elements
           uint4 w;
-          w.x = pack2<BF16>(__uint_as_float(o[q4 * 8 + 0]) * inv_l, __uint_as_float(o[q4 * 8 + 1]) * inv_l);
-          w.y = pack2<BF16>(__uint_as_float(o[q4 * 8 + 2]) * inv_l, __uint_as_float(o[q4 * 8 + 3]) * inv_l);
-          w.z = pack2<BF16>(__uint_as_float(o[q4 * 8 + 4]) * inv_l, __uint_as_float(o[q4 * 8 + 5]) * inv_l);
-          w.w = pack2<BF16>(__uint_as_float(o[q4 * 8 + 6]) * inv_l, __uint_as_float(o[q4 * 8 + 7]) * inv_l);
+          w.x = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 0]) * inv_l, __uint_as_float(o[c][q4 * 8 + 1]) * inv_l);
+          w.y = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 2]) * inv_l, __uint_as_float(o[c][q4 * 8 + 3]) * inv_l);
+          w.z = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 4]) * inv_l, __uint_as_float(o[c][q4 * 8 + 5]) * inv_l);
+          w.w = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 6]) * inv_l, __uint_as_float(o[c][q4 * 8 + 7]) * inv_l);
           const int chunk = c * 4 + q4;  // 16-byte chunk index along the row
           const int bx = chunk >> 3, cc = chunk & 7;
           *reinterpret_cast<uint4*>(ptile + bx * C::kBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
         }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1 + t, 128);
-      if (r == 0) {
-        if (!*abort_flag) {
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the TMA store
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::kBarOReady + t));
+      if (quarter == 0) {
+        mbar_wait(BAR(C::kBarOReady + t), nout & 1, wctx);
+        if (r == 0 && !*abort_flag) {
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_store_4d(&p.tm_o, sbase + C::kOffO + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64,
                          u.h, row0, u.b);
           bulk_commit_group();
         }
-        bulk_wait_group_read0();
       }
+      ++nout;
       if (p.lse != nullptr && grow < p.Nq) {
         const float lse = l_run > 0.f ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                       : -INFINITY;
         p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
       }
-      named_bar_sync(1 + t, 128);  // the staging buffer is free again for the next unit
       if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1408 + 64 * t + k);
     }
+    if (r == 0) bulk_wait_group_read0();  // the last O store has read the staging buffer
     } else {
     // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ======
     const int t = warp >> 2;
@@ -898,11 +988,18 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     };
     int ns = 0;  // S tiles consumed (s_full phases)
     int no = 0;  // units finished (o_full phases)
+    bool store_pending = false;  // (row 0's thread) this tile's last O store may still read the buffer
     for (int k = 0;; ++k) {
-      const int unit = next_unit(k);
-      if (unit < 0) break;
+      const PrefillUnit u = next_unit(k);
+      // The store issued at the end of the previous unit has had the unit switch to read
+      // the staging buffer; only now does row 0's thread wait for it and pass the turn on.
+      if (r == 0 && store_pending) {
+        bulk_wait_group_read0();
+        mbar_arrive(BAR(C::kBarOStage + t));
+        store_pending = false;
+      }
+      if (u.nmax < 0) break;
       if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1152 + 64 * t + k);
-      const PrefillUnit u = prefill_unit(p, unit);
       const int row0 = u.row0[t];
       const int nkv = u.nkv[t];
       const int grow = row0 + r;  // global query row
@@ -968,27 +1065,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
 
-        // pass 2: P for half 1 (keys 64..127, from registers) into TMEM columns 96..127,
-        // which held S columns 96..127 -- already read; then half 0 re-read from TMEM
-        // (columns 0..63, untouched) into P columns 64..95.
-        uint32_t pk[32];
-        float rs = need_mask ? half_exp_pack<true, 1>(hv, cs, m_use, lim, pk)
-                             : half_exp_pack<false, 1>(hv, cs, m_use, lim, pk);
-        __syncwarp();
-        tmem_st32(tS + 96, pk);
-        tmem_ld32(tS + 0, hv[0]);
-        tmem_ld32(tS + 32, hv[1]);
-        tmem_ld_wait();
-        reg_order_after_wait(hv[0]);
-        reg_order_after_wait(hv[1]);
-        rs += need_mask ? half_exp_pack<true, 0>(hv, cs, m_use, lim, pk)
-                        : half_exp_pack<false, 0>(hv, cs, m_use, lim, pk);
-        l_run += rs;
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
-        __syncwarp();
-        tmem_st32(tS + 64, pk);
-
-        // lazy rescale of O (the previous P V of this tile completed before S_t(j) did)
+        // lazy rescale of O, before any P_t(j) V_j can start (P_t(j-1) V_{j-1} completed
+        // before S_t(j) did)
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -1001,6 +1079,31 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tmem_st32(tO + c * 32, o);
           }
         }
+
+        // pass 2: P for half 1 (keys 64..127, from registers) into TMEM columns 96..127,
+        // which held S columns 96..127 -- already read -- and published at once, so the
+        // tensor core starts on keys 64..127 of P_t V_j; then half 0 re-read from TMEM
+        // (columns 0..63, untouched) into P columns 64..95.
+        uint32_t pk[32];
+        float rs = need_mask ? half_exp_pack<true, 1>(hv, cs, m_use, lim, pk)
+                             : half_exp_pack<false, 1>(hv, cs, m_use, lim, pk);
+        __syncwarp();
+        tmem_st32(tS + 96, pk);
+        tmem_ld32(tS + 0, hv[0]);
+        tmem_ld32(tS + 32, hv[1]);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::kBarPHalf + t));
+        tmem_ld_wait();
+        reg_order_after_wait(hv[0]);
+        reg_order_after_wait(hv[1]);
+        rs += need_mask ? half_exp_pack<true, 0>(hv, cs, m_use, lim, pk)
+                        : half_exp_pack<false, 0>(hv, cs, m_use, lim, pk);
+        l_run += rs;
+        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
+        __syncwarp();
+        tmem_st32(tS + 64, pk);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
@@ -1016,35 +1119,40 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       tc_fence_after_sync();
       ostage_acquire(k);  // the previous store from the staging buffer has read it
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_ld_wait();
-        reg_order_after_wait(o);
+      {
+        uint32_t o[D / 32][32];  // the whole O row: one TMEM round trip
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {  // four 16-byte chunks of 8 elements
-          uint4 w;
-          w.x = pack2<BF16>(__uint_as_float(o[q4 * 8 + 0]) * inv_l, __uint_as_float(o[q4 * 8 + 1]) * inv_l);
-          w.y = pack2<BF16>(__uint_as_float(o[q4 * 8 + 2]) * inv_l, __uint_as_float(o[q4 * 8 + 3]) * inv_l);
-          w.z = pack2<BF16>(__uint_as_float(o[q4 * 8 + 4]) * inv_l, __uint_as_float(o[q4 * 8 + 5]) * inv_l);
-          w.w = pack2<BF16>(__uint_as_float(o[q4 * 8 + 6]) * inv_l, __uint_as_float(o[q4 * 8 + 7]) * inv_l);
-          const int chunk = c * 4 + q4;  // 16-byte chunk index along the row
-          const int bx = chunk >> 3, cc = chunk & 7;
-          *reinterpret_cast<uint4*>(ostage + bx * C::kBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) reg_order_after_wait(o[c]);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {  // four 16-byte chunks of 8 elements
+            uint4 w;
+            w.x = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 0]) * inv_l, __uint_as_float(o[c][q4 * 8 + 1]) * inv_l);
+            w.y = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 2]) * inv_l, __uint_as_float(o[c][q4 * 8 + 3]) * inv_l);
+            w.z = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 4]) * inv_l, __uint_as_float(o[c][q4 * 8 + 5]) * inv_l);
+            w.w = pack2<BF16>(__uint_as_float(o[c][q4 * 8 + 6]) * inv_l, __uint_as_float(o[c][q4 * 8 + 7]) * inv_l);
+            const int chunk = c * 4 + q4;  // 16-byte chunk index along the row
+            const int bx = chunk >> 3, cc = chunk & 7;
+            *reinterpret_cast<uint4*>(ostage + bx * C::kBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+          }
         }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1 + t, 128);
-      if (r == 0 && !*abort_flag) {
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_store_4d(&p.tm_o, sbase + C::kOffO + bx * C::kBoxBytes, bx * 64, u.h, row0, u.b);
-        bulk_commit_group();
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the TMA store
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::kBarOReady + t));
+      if (quarter == 0) {
+        mbar_wait(BAR(C::kBarOReady + t), (no - 1) & 1, wctx);
+        if (r == 0 && !*abort_flag) {
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_store_4d(&p.tm_o, sbase + C::kOffO + bx * C::kBoxBytes, bx * 64, u.h, row0, u.b);
+          bulk_commit_group();
+        }
       }
-      if (r == 0) {
-        bulk_wait_group_read0();
-        mbar_arrive(BAR(C::kBarOStage + t));  // hand the staging buffer to the other tile
-      }
+      store_pending = true;  // completed (and the turn passed on) after the next unit is read
       if (p.lse != nullptr && grow < p.Nq) {
         const float lse = l_run > 0.f ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f
                                       : -INFINITY;
@@ -1058,6 +1166,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   // ---- teardown: every role is done with TMEM
   tc_fence_before_sync();
   __syncthreads();
+#ifdef ATTN_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][1] = global_timer_ns();
+#endif
   if (warp == C::kMmaWarp) {
     __syncwarp();
     tc_fence_after_sync();
