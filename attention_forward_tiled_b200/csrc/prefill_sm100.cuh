@@ -184,6 +184,13 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
 #define ATTN_EXP_EMU_PERIOD 4
 #endif
 
+// d = 128: unmasked tiles after the first are exponentiated against the running max in
+// the same pass that finds the tile max (P kept in registers, redone in the rare case a
+// score exceeds the running max by more than 8).
+#ifndef ATTN_SPECULATIVE
+#define ATTN_SPECULATIVE 1
+#endif
+
 // Max over one 64-column half of an S row (columns 64*kHalf + c), sign-flipped for a
 // negative scale, restricted to columns < lim when kMask; four 3-input max chains.
 template <bool kMask, bool kNeg, int kHalf>
@@ -252,6 +259,38 @@ __device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float
     }
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
+}
+
+// Unmasked half row (64 columns, registers h) against the running max m_use: packs
+// p = 2^(cs * s - m_use) into 32 fp16 pairs and returns the half's row sum; xmax gets the
+// largest exponent cs * s - m_use seen (the caller redoes the tile if it exceeds 8).
+__device__ __forceinline__ float half_exp_pack_spec(const uint32_t (&h)[2][32], float cs, float m_use,
+                                                    uint32_t (&pk)[32], float& xmax) {
+  uint64_t acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
+  float mx[2] = {xmax, -INFINITY};
+  const uint64_t cs2 = f2_make(cs, cs), negm2 = f2_make(-m_use, -m_use);
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const uint64_t x2 = f2_fma(f2_make(__uint_as_float(h[c >> 5][c & 31]),
+                                       __uint_as_float(h[(c + 1) >> 5][(c + 1) & 31])),
+                               cs2, negm2);
+    const float2 x = f2_split(x2);
+    mx[(c >> 1) & 1] = fmax3(mx[(c >> 1) & 1], x.x, x.y);
+    float2 pp;
+    if (ATTN_EXP_EMU_PERIOD > 0 && ((c >> 1) % (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD : 1)) ==
+                                       (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD - 1 : 0)) {
+      pp = exp2_poly2(x2);
+    } else {
+      pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    }
+    acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_make(pp.x, pp.y));
+    pk[c >> 1] = pack2<false>(pp.x, pp.y);
+  }
+  xmax = fmaxf(mx[0], mx[1]);
+  const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
+  return a.x + a.y;
 }
 
 // Max over the 128 scores of an S row (sign-flipped for a negative scale),
@@ -718,12 +757,14 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
                   wctx);
         __syncwarp();
         const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
+        if (lane == 0 && k == 0 && j < 32) ATTN_TRACE_POINT(1920 + j);
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= u.nkv[t]) continue;
           // keys 64..127 as soon as that half of P_t(j) is written, then keys 0..63
           mbar_wait(BAR(C::kBarPHalf + t), np[t] & 1, wctx);
           __syncwarp();
+          if (lane == 0 && k == 0 && j < 32) ATTN_TRACE_POINT(1952 + 32 * t + j);
           tc_fence_after_sync();
           if (!warp_flag(abort_flag)) issue_pv4(t, stage_addr(iv), 4, j > 0);
           mbar_wait(BAR(C::kBarPFull + t), np[t] & 1, wctx);
@@ -1035,6 +1076,49 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
           if (p.causal) l = min(l, (long long)grow + diag + 1);
           l -= key0;
           lim = (int)max(0LL, min(128LL, l));
+        }
+
+        // Speculative single pass: S read in two halves, exponentiated against m_run while
+        // the tile max is found; P stays in registers and is written only if no exponent
+        // exceeds 8 in any row of the warp (S is untouched until then), else the two-pass
+        // path below redoes the tile.
+        if (ATTN_SPECULATIVE && j > 0 && !need_mask && __all_sync(0xffffffffu, m_run != -INFINITY)) {
+          uint32_t pk[2][32];
+          float xmax = -INFINITY;
+          float rs;
+          {
+            uint32_t sv[2][32];
+            tmem_ld32(tS + 64, sv[0]);
+            tmem_ld32(tS + 96, sv[1]);
+            tmem_ld_wait();
+            reg_order_after_wait(sv[0]);
+            reg_order_after_wait(sv[1]);
+            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(385 + 64 * t + j);
+            rs = half_exp_pack_spec(sv, cs, m_run, pk[1], xmax);
+            tmem_ld32(tS + 0, sv[0]);
+            tmem_ld32(tS + 32, sv[1]);
+            tmem_ld_wait();
+            reg_order_after_wait(sv[0]);
+            reg_order_after_wait(sv[1]);
+            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(513 + 64 * t + j);
+            rs += half_exp_pack_spec(sv, cs, m_run, pk[0], xmax);
+          }
+          if (!__any_sync(0xffffffffu, xmax > 8.0f)) {
+            l_run += rs;
+            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
+            tmem_st32(tS + 96, pk[1]);  // keys 64..127
+            tmem_st_wait();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(C::kBarPHalf + t));
+            tmem_st32(tS + 64, pk[0]);  // keys 0..63
+            tmem_st_wait();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
+            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
+            continue;
+          }
         }
 
         // pass 1: row max over the two 64-column halves (half 1 stays in registers)
