@@ -697,24 +697,18 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     const uint32_t colO[2] = {256u, 256u + D};
     const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
     // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
+    // S_t = Q_t K_j^T: 8 k-steps of 16 elements, issued in one batch.
     auto issue_s = [&](int t, uint32_t sK) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-        mma_f16_ss_w(tmem + colS[t], make_sdesc_sw128(sQ[t] + off, 16, 1024),
-                     make_sdesc_sw128(sK + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-      }
+      mma_f16_ss_k128_w<C::kBoxBytes>(tmem + colS[t], make_sdesc_sw128(sQ[t], 16, 1024),
+                                      make_sdesc_sw128(sK, 16, 1024), idesc_s, 0u);
     };
-    // O_t += P_t V_j over 8 k-steps of 16 keys; P_t is in TMEM columns [64,128) of S_t.
-    // k-steps kk0 .. kk0+3 of O_t += P_t V_j (keys 16*kk0 .. 16*kk0+63); the first k-step
-    // of the unit starts the accumulator.
+    // k-steps kk0 .. kk0+3 of O_t += P_t V_j (keys 16*kk0 .. 16*kk0+63; P_t is in TMEM
+    // columns [64,128) of S_t), issued in one batch; the first k-step of the unit starts
+    // the accumulator.
     auto issue_pv4 = [&](int t, uint32_t sV, int kk0, bool accumulate_first) {
-#pragma unroll
-      for (int kk = kk0; kk < kk0 + 4; ++kk) {
-        mma_f16_ts_w(tmem + colO[t], tmem + colS[t] + 64 + kk * 8,
-                     make_sdesc_sw128(sV + kk * 2048, C::kBoxBytes, 1024), idesc_o,
-                     (accumulate_first || kk > kk0) ? 1u : 0u);
-      }
+      mma_f16_ts_k64_w<2048>(tmem + colO[t], tmem + colS[t] + 64 + kk0 * 8,
+                             make_sdesc_sw128(sV + kk0 * 2048, C::kBoxBytes, 1024), idesc_o,
+                             accumulate_first ? 1u : 0u);
     };
     auto stage_addr = [&](int item) -> uint32_t {
       return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;

@@ -377,6 +377,61 @@ __device__ __forceinline__ void mma_f16_ts_w(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// Eight k-steps of D = A B with A and B K-major in shared memory (128-byte swizzle, two
+// 64-element boxes of kBox bytes along K): one elected lane issues all eight, advancing both
+// descriptors' start address by 32 B per k-step inside a box and by one box after four.
+template <uint32_t kBoxBytes>
+__device__ __forceinline__ void mma_f16_ss_k128_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  constexpr uint64_t kStep = 32 >> 4, kBox = kBoxBytes >> 4;
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b64 a, b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 a, %1, %5;\n\tadd.s64 b, %2, %5;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %6;\n\tadd.s64 b, %2, %6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %7;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %8;\n\tadd.s64 b, %2, %8;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %9;\n\tadd.s64 b, %2, %9;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %10;\n\tadd.s64 b, %2, %10;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %11;\n\tadd.s64 b, %2, %11;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kStep), "n"(2 * kStep),
+      "n"(3 * kStep), "n"(kBox), "n"(kBox + kStep), "n"(kBox + 2 * kStep), "n"(kBox + 3 * kStep)
+      : "memory");
+}
+
+// Four k-steps of D += A B with A in TMEM (8 columns of packed 16-bit pairs per k-step) and
+// B MN-major in shared memory (kRowBytes per 16-row k-step): one elected lane issues all four.
+template <uint32_t kKStepBytes>
+__device__ __forceinline__ void mma_f16_ts_k64_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  constexpr uint64_t kStep = kKStepBytes >> 4;
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 a, %1, 8;\n\tadd.s64 b, %2, %5;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, %1, 16;\n\tadd.s64 b, %2, %6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, %1, 24;\n\tadd.s64 b, %2, %7;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kStep), "n"(2 * kStep),
+      "n"(3 * kStep)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_commit_w(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
