@@ -194,18 +194,25 @@ struct WaitCtx {
 };
 
 // Wait for the phase with the given parity to complete.  Never spins forever:
-// gives up after timeout_ns (wall clock, %globaltimer) or once any thread of the
-// CTA has raised the abort flag.  Returns false on give-up; the first thread
-// that times out records kStatusTimeout in the status word and raises the flag.
-// The first poll is inline; the polling loop is out of line with its arguments in
-// registers.
+// gives up after the time limit or once any thread of the CTA has raised the abort
+// flag.  Returns false on give-up; the first thread that times out records
+// kStatusTimeout in the status word and raises the flag.  The first poll is inline;
+// the polling loop is out of line with its arguments in registers.
+// The limit is counted in SM clock cycles (clock64, a cheap register read; %globaltimer
+// costs hundreds of cycles per read and delayed the wake-up after a phase completed) at
+// 2 cycles per ns, so below 2 GHz a wait may last proportionally longer than timeout_ns.
+__device__ __forceinline__ long long wait_limit_cycles(uint64_t timeout_ns) {
+  return (long long)(timeout_ns < (1ull << 40) ? timeout_ns : (1ull << 40)) * 2;
+}
+
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                             int* status, uint64_t timeout_ns) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0; it < (1u << 26); ++it) {
+  const long long limit = wait_limit_cycles(timeout_ns);
+  const long long c0 = clock64();
+  for (uint32_t it = 0; it < (1u << 30); ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > timeout_ns) break;
+    if (clock64() - c0 > limit) break;
   }
   *abort_flag = 1;
   atomicCAS(status, 0, kStatusTimeout);
@@ -220,10 +227,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 // Drain wait used on the way out after an abort: ignores the abort flag but is
 // still bounded by the time limit.
 __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0; it < (1u << 26); ++it) {
+  const long long limit = wait_limit_cycles(timeout_ns);
+  const long long c0 = clock64();
+  for (uint32_t it = 0; it < (1u << 30); ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > timeout_ns) return false;
+    if (clock64() - c0 > limit) return false;
   }
   return false;
 }
