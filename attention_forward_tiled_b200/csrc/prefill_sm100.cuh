@@ -1110,6 +1110,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
+            if (lane == 0 && k == 0 && j >= 8 && j < 12) ATTN_TRACE_POINT(2016 + (j - 8) * 8 + t * 4 + quarter);
             if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
             continue;
           }
