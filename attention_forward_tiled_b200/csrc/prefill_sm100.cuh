@@ -176,13 +176,21 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
   return u;
 }
 
-// Every ATTN_EXP_EMU_PERIOD-th pair of softmax exponentials is evaluated with the
-// FMA-pipe polynomial instead of the MUFU unit (0 = all on MUFU).  At d = 128 the
-// exponentials of one K/V step need as many MUFU cycles as its four MMAs need
-// tensor cycles, so moving a share of them to the FMA pipe shortens the softmax.
+// Every ATTN_EXP_EMU_PERIOD-th pair of softmax exponentials (d = 128;
+// ATTN_EXP_EMU_PERIOD_D64 at d = 64) is evaluated with the FMA-pipe polynomial instead
+// of the MUFU unit (0 = all on MUFU).  MUFU delivers 4 exp2 per clock per SM
+// sub-partition; the polynomial costs more issue slots per result, so the best share is
+// measured: every 8th pair at d = 128 (1 in 4 and 1 in 3 were slower), every 4th at d = 64.
 #ifndef ATTN_EXP_EMU_PERIOD
-#define ATTN_EXP_EMU_PERIOD 4
+#define ATTN_EXP_EMU_PERIOD 8
 #endif
+#ifndef ATTN_EXP_EMU_PERIOD_D64
+#define ATTN_EXP_EMU_PERIOD_D64 4
+#endif
+template <int kPeriod>
+__device__ __forceinline__ constexpr bool emu_pair(int pair) {
+  return kPeriod > 0 && (pair % (kPeriod > 0 ? kPeriod : 1)) == (kPeriod > 0 ? kPeriod - 1 : 0);
+}
 
 // d = 128: unmasked tiles after the first are exponentiated against the running max in
 // the same pass that finds the tile max (P kept in registers, redone in the rare case a
@@ -232,8 +240,7 @@ __device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float
                                          __uint_as_float(h[(c + 1) >> 5][(c + 1) & 31])),
                                  cs2, negm2);
       float2 pp;
-      if (ATTN_EXP_EMU_PERIOD > 0 && ((c >> 1) % (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD : 1)) ==
-                                         (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD - 1 : 0)) {
+      if (emu_pair<ATTN_EXP_EMU_PERIOD>(c >> 1)) {
         pp = exp2_poly2(x2);
       } else {
         const float2 x = f2_split(x2);
@@ -279,8 +286,7 @@ __device__ __forceinline__ float half_exp_pack_spec(const uint32_t (&h)[2][32], 
     const float2 x = f2_split(x2);
     mx[(c >> 1) & 1] = fmax3(mx[(c >> 1) & 1], x.x, x.y);
     float2 pp;
-    if (ATTN_EXP_EMU_PERIOD > 0 && ((c >> 1) % (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD : 1)) ==
-                                       (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD - 1 : 0)) {
+    if (emu_pair<ATTN_EXP_EMU_PERIOD>(c >> 1)) {
       pp = exp2_poly2(x2);
     } else {
       pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
@@ -318,7 +324,7 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32], int lim) {
 }
 
 // p for the column pair (c, c+1): 2^(cs * s - m_use); the FMA-pipe polynomial for every
-// ATTN_EXP_EMU_PERIOD-th pair, MUFU ex2 otherwise; 0 at columns >= lim when kMask.
+// ATTN_EXP_EMU_PERIOD_D64-th pair, MUFU ex2 otherwise; 0 at columns >= lim when kMask.
 template <bool kMask>
 __device__ __forceinline__ float2 pair_exp(const uint32_t (&sr)[4][32], int c, uint64_t cs2,
                                            uint64_t negm2, int lim) {
@@ -326,9 +332,7 @@ __device__ __forceinline__ float2 pair_exp(const uint32_t (&sr)[4][32], int c, u
                                      __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31])),
                              cs2, negm2);
   float2 pp;
-  if (!kMask && ATTN_EXP_EMU_PERIOD > 0 &&
-      ((c >> 1) % (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD : 1)) ==
-          (ATTN_EXP_EMU_PERIOD > 0 ? ATTN_EXP_EMU_PERIOD - 1 : 0)) {
+  if (!kMask && emu_pair<ATTN_EXP_EMU_PERIOD_D64>(c >> 1)) {
     pp = exp2_poly2(x2);
   } else {
     const float2 x = f2_split(x2);
