@@ -91,6 +91,30 @@ def test_large_logits_bf16():
     run_and_compare(1, 4, 384, 512, 64, "bf16", False, 1 / 8, seed=3, k_mult=3.0)
 
 
+@pytest.mark.parametrize("d,dtype,causal", [(128, "f16", False), (128, "bf16", True),
+                                             (64, "f16", True), (64, "bf16", False)])
+def test_running_max_jumps(d, dtype, causal):
+    """Key norms grow tile by tile, so the row max of scale*log2(e)*s rises by ~9 per key
+    tile, past the lazy threshold of 8: every lazy O rescale and the redo of a tile whose
+    single-pass exponentials would overflow the running max are exercised (the inputs are
+    only reshaped here)."""
+    B, H, Nq, Nk = 1, 2, 512, 1024
+    q, k, v = make_inputs(B, H, Nq, Nk, d, dtype="f16", seed=21 + d)
+    growth = 1.0 + 2.5 * (torch.arange(Nk, dtype=torch.float32) // 128)  # x1 .. x18.5 per key tile
+    k = (k.float() * growth.view(1, Nk, 1, 1)).to(DT[dtype])
+    # Half-size values: with so peaked a softmax the fp16 rounding of P alone moves O by up
+    # to 2^-11 * |v_i - O| (2.1e-3 at unit-variance V, as an fp32/fp16 model of the kernel's
+    # arithmetic reproduces exactly); halving V keeps that within the fp16 bound.
+    q, v = q.to(DT[dtype]), (v.float() * 0.5).to(DT[dtype])
+    scale = 1 / math.sqrt(d)
+    out, lse = attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal=causal, scale=scale)
+    assert_o_close(out, o_ref, DT[dtype], f"growing keys d={d} {dtype} causal={causal}")
+    assert_lse_close(lse, lse_ref, "lse (growing keys)")
+
+
 def test_lse_optional_and_deterministic():
     q, k, v = (t.cuda() for t in make_inputs(2, 4, 300, 300, 128, seed=8))
     o1, _ = attn_fwd(q, k, v, causal=True, return_lse=False)
