@@ -8,32 +8,36 @@
 // Buffer) is prior art; this kernel maps the same algorithm onto B200.
 //
 // Work unit = (batch b, head h, a pair of 128-row Q tiles).  The grid has one CTA
-// per unit, but a resident CTA (one per SM) keeps going: while it works on a unit
-// it claims the next not-yet-started CTA with cluster launch control
+// per unit, but a resident CTA (one per SM) keeps going: late in each unit it claims
+// the next not-yet-started CTA with cluster launch control
 // (clusterlaunchcontrol.try_cancel) and does that CTA's unit as well, so units are
-// handed out dynamically in launch order (heaviest causal units first, heads in
-// groups so their K/V stay in L2) and TMEM, barriers and the load pipeline stay up
-// across units.  Roles inside a CTA (384 threads):
-//   * warp 8, producer: claims units and publishes them to the other roles through
-//     a two-slot ring in shared memory; loads Q_t once per unit and streams K_0,
-//     V_0, K_1, V_1, ... into a ring of shared-memory stages with TMA (128-byte
-//     swizzle), each stage guarded by a full/empty mbarrier pair;
-//   * warp 9, MMA issuer (whole warp, one elected lane issues) runs tcgen05.mma:
+// handed out dynamically, in launch order (heaviest causal units first, heads in
+// groups so their K/V stay in L2), to the SMs about to run out of work, and TMEM,
+// barriers and the load pipeline stay up across units.  Roles inside a CTA (384
+// threads):
+//   * warp 8, producer: claims units, decodes them and publishes them to the other
+//     roles through a two-slot ring in shared memory; loads Q_t once per unit and
+//     streams K_0, V_0, K_1, V_1, ... into a ring of shared-memory stages with TMA
+//     (128-byte swizzle), each stage guarded by a full/empty mbarrier pair;
+//   * warp 9, MMA issuer (whole warp, one elected lane issues a batch of k-steps at
+//     a time) runs tcgen05.mma:
 //       S_t = Q_t K_j^T   (A, B from shared memory, fp32 accumulator in TMEM)
 //       O_t += P_t V_j    (A = P_t from TMEM, B = V from shared memory)
 //     alternating the two Q tiles so one tile's softmax overlaps the other tile's
 //     matrix multiplies.  d = 128: P_t is written over the consumed S_t columns, so
-//     S_t(j+1) follows P_t(j) V_j.  d = 64: TMEM has room for separate P buffers, so
-//     S_t(j+1) is issued as soon as the softmax has read S_t(j) and is computed while
-//     that softmax runs;
+//     S_t(j+1) follows P_t(j) V_j; the softmax publishes P for keys 64..127 first and
+//     that half of P V starts at once.  d = 64: TMEM has room for separate P buffers,
+//     so S_t(j+1) is issued as soon as the softmax has read S_t(j) and is computed
+//     while that softmax runs;
 //   * warps 10-11 (bf16 inputs only) convert each V tile to fp16 in place, so
 //     P V runs with P in fp16 (11-bit significand) rather than bf16 (8-bit);
 //   * warps 0-3 and 4-7, softmax warpgroups (one per Q tile, one thread per query
-//     row): read the 128-column S row from TMEM, release it, apply the tail/causal
-//     mask, update the running max m and sum l (base-2 exponent with scale*log2(e)
-//     folded into one packed FMA, lazy rescale of O only when the max grows by more
-//     than 2^8), write P as fp16 into TMEM, and at the end of the unit normalise O
-//     by 1/l, stage it in shared memory, store it with TMA and write the row LSE.
+//     row): read the 128-column S row from TMEM, apply the tail/causal mask, update
+//     the running max m and sum l (base-2 exponent with scale*log2(e) folded into one
+//     packed FMA, lazy rescale of O only when the max grows by more than 2^8; at
+//     d = 128 unmasked tiles after the first take a single pass against the running
+//     max), write P as fp16 into TMEM, and at the end of the unit normalise O by 1/l,
+//     stage it in shared memory, store it with TMA and write the row LSE.
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [256+D, 256+2D); P_t in columns [64,128) of S_t (d = 128) or in its own

@@ -17,6 +17,7 @@ the method available here) on bounded samples of the same workload.
 """
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -49,12 +50,19 @@ def load_peaks():
 
 
 def kernel_source_sha():
-    """Hash of the CUDA sources: ties a committed ncu traffic figure to the kernel it measured."""
+    """Hash of the CUDA sources' code (comments and blank space removed): ties a committed
+    ncu traffic figure to the kernel it measured, so editing a comment does not orphan it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_forward_tiled_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        if not name.endswith((".cu", ".cuh", ".h")):
+            continue
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        text = " ".join(text.split())
+        h.update(name.encode() + b"\0" + text.encode())
     return h.hexdigest()[:16]
 
 
