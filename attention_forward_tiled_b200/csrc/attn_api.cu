@@ -212,7 +212,12 @@ int launch_prefill(DeviceState* ds, const void* q, const void* k, const void* v,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.inject = g_inject.load();
   p.timeout_ns = g_timeout_ns.load();
-  const long long units = (long long)B * H * p.n_qpairs;
+  const long long pairs = (long long)B * H * p.n_qpairs;
+  // Equal-sized (non-causal) units end in a partial wave; when it would fill at most half
+  // of the SMs, its pairs run as single-tile units, two per pair, in about half the time.
+  const long long rem = pairs % ds->sm_count;
+  p.n_split = (!causal && pairs > ds->sm_count && 2 * rem <= ds->sm_count) ? (int)rem : 0;
+  const long long units = pairs + p.n_split;
   if (units >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
   kernel<<<dim3((unsigned)units), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

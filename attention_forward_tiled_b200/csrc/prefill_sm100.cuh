@@ -62,6 +62,7 @@ struct PrefillParams {
   int causal;
   int n_qpairs;      // ceil(Nq / 256)
   int group_heads;   // heads per scheduling group (L2 locality of K/V)
+  int n_split;       // the last n_split pair units run as two single-tile units each
   float scale_log2;  // scale * log2(e)
   int inject;        // test hook: 1 = skip the Q-tile-0 loads
   unsigned long long timeout_ns;
@@ -149,20 +150,28 @@ struct PrefillUnit {
 };
 
 // All quantities fit in 32 bits: the launcher rejects grids of 2^31 units or more.
+// Units past the first B*H*n_qpairs - n_split are single Q tiles: the last n_split pairs,
+// split in two, so the final wave of equal-sized (non-causal) units is half as long.
 __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int unit) {
   const int BH = p.B * p.H;
   const int nqp = p.n_qpairs;
   const int G = p.group_heads;
+  const int n_pairs = BH * nqp - p.n_split;
+  int pair = unit, single = -1;  // single: which tile of a split pair this unit runs
+  if (unit >= n_pairs) {
+    pair = n_pairs + ((unit - n_pairs) >> 1);
+    single = (unit - n_pairs) & 1;
+  }
   const int per_group = G * nqp;
   const int full_units = (BH / G) * per_group;
   int g, idx, Gc;
-  if (unit < full_units) {
-    g = unit / per_group;
-    idx = unit - g * per_group;
+  if (pair < full_units) {
+    g = pair / per_group;
+    idx = pair - g * per_group;
     Gc = G;
   } else {
     g = BH / G;
-    idx = unit - full_units;
+    idx = pair - full_units;
     Gc = BH - g * G;
   }
   const int qrank = idx / Gc;
@@ -174,6 +183,10 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
   u.h = bh - u.b * p.H;
   u.row0[0] = qp * 256;
   u.row0[1] = qp * 256 + 128;
+  if (single >= 0) {  // tile slot 1 idles: rows at or past Nq are neither computed nor stored
+    u.row0[0] = qp * 256 + 128 * single;
+    u.row0[1] = p.Nq;
+  }
   u.nkv[0] = prefill_kv_tiles(u.row0[0], p.Nq, p.Nk, p.causal);
   u.nkv[1] = prefill_kv_tiles(u.row0[1], p.Nq, p.Nk, p.causal);
   u.nmax = max(u.nkv[0], u.nkv[1]);

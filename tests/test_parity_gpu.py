@@ -58,6 +58,8 @@ SMALL = [
     (1, 2, 700, 300, 64, "f16", True),      # Nq > Nk: leading rows see no key
     (1, 2, 513, 1, 128, "f16", False),      # a single key
     (1, 2, 513, 1, 64, "bf16", True),       # single key, causal: only the last row has it
+    (2, 80, 384, 256, 64, "f16", False),    # 320 tile pairs: the last partial wave runs as single
+    (2, 80, 320, 200, 128, "bf16", False),  #   tiles (a pair's second tile may lie past Nq)
     (1, 3, 2, 517, 128, "f16", True),       # two query rows
     (3, 1, 384, 384, 64, "bf16", True),     # three Q tiles -> one half-used pair
     (1, 4, 128, 1024, 128, "bf16", True),
