@@ -76,6 +76,9 @@ typedef enum {
  * kernels on `stream` and returns.  Argument errors return before anything is
  * enqueued.  A device-side failure (a bounded wait that expired) does not
  * trap: it is recorded in a per-device status word read by attn_get_status().
+ * Since the call only enqueues work (and stream-ordered allocations) on
+ * `stream`, it can be captured into a CUDA graph once a first call on the
+ * device has run (that call sets the kernels' shared-memory attributes).
  *
  * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA.
  */
