@@ -51,7 +51,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int* status_ptr = nullptr;
-  bool attr_set[8] = {};  // per kernel instantiation: max dynamic shared memory raised
+  bool attr_set[12] = {};  // per kernel instantiation: max dynamic shared memory raised
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -133,14 +133,15 @@ int ensure_smem_attr(DeviceState* ds, int slot, Kernel kernel, int bytes) {
   return ATTN_OK;
 }
 
-// 4-D view (d, H, N, B) of a contiguous [B, N, H, d] tensor; box (64, 1, 128, 1), 128B swizzle.
-int encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, int dtype) {
+// 4-D view (d, H, N, B) of a contiguous [B, N, H, d] tensor; box (64, 1, box_rows, 1), 128B swizzle.
+int encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, int dtype,
+                int box_rows = 128) {
   EncodeTiledFn encode = get_encode_fn();
   if (!encode) return ATTN_ERR_CUDA;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
                                  (cuuint64_t)N * H * d * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapDataType ty =
       dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -291,6 +292,101 @@ int launch_decode(DeviceState* ds, const void* q, const void* k, const void* v, 
   return rc;
 }
 
+// Paged cache: the same two kernels, the partial one reading each request's keys and
+// values page by page through its block table (up to seq_lens[b] keys).
+template <int D, bool BF16>
+int launch_decode_paged(DeviceState* ds, const void* q, const void* k_cache, const void* v_cache,
+                        const int* block_table, const int* seq_lens, void* out, float* lse, int B,
+                        int H, int num_blocks, int page_size, int max_blocks, float scale,
+                        int splits_req, cudaStream_t stream) {
+  using C = DecodeCfg<D>;
+  auto kernel = attn_decode_partial_kernel<D, BF16, true>;
+  const int slot = 8 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  const int Nk = max_blocks * page_size;  // validated < 2^31
+  const int ntiles = (Nk + 127) / 128;
+  const long long BH = (long long)B * H;
+  int splits = splits_req > 0 ? splits_req : choose_splits(BH, ntiles, ds->sm_count);
+  if (splits < 1 || splits > ntiles) return ATTN_ERR_INVALID_ARG;
+  const int tps = (ntiles + splits - 1) / splits;
+  splits = (ntiles + tps - 1) / tps;
+  const long long items = BH * splits;
+  if (items >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+
+  DecodeParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  const int page_rows = page_size < 128 ? page_size : 128;
+  if (int rc = encode_bnhd(&p.tm_k, k_cache, 1, num_blocks * page_size, H, D, dtype, page_rows)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v_cache, 1, num_blocks * page_size, H, D, dtype, page_rows)) return rc;
+  float* part = nullptr;
+  const size_t ws_bytes = (size_t)items * (D + 2) * sizeof(float);
+  if (cudaMallocAsync(reinterpret_cast<void**>(&part), ws_bytes, stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  p.q = q;
+  p.part = part;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Nk = Nk;
+  p.splits = splits;
+  p.tiles_per_split = tps;
+  p.n_items = (int)items;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.max_blocks = max_blocks;
+  p.page_size = page_size;
+  p.page_rows = page_rows;
+  p.num_blocks = num_blocks;
+  const int grid = (int)std::min<long long>(items, ds->sm_count);
+  kernel<<<dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  int rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  if (rc == ATTN_OK) {
+    attn_decode_combine_kernel<D, BF16>
+        <<<dim3((unsigned)((BH + 3) / 4)), dim3(128), 0, stream>>>(part, out, lse, (int)BH, splits);
+    rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (cudaFreeAsync(part, stream) != cudaSuccess) rc = ATTN_ERR_CUDA;
+  return rc;
+}
+
+// Argument checks of attn_fwd_decode_paged (nothing is enqueued on failure).
+int validate_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                   const int* seq_lens, const void* out, const float* lse, int B, int H, int d,
+                   int num_blocks, int page_size, int max_blocks, float scale, int dtype, int splits) {
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || d <= 0 || num_blocks <= 0 || page_size <= 0 || max_blocks <= 0 || splits < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  // a page is a whole number of 128-key tiles, or a tile a whole number of >= 8-row pages
+  const bool page_ok = page_size < 128 ? (page_size % 8 == 0 && 128 % page_size == 0)
+                                       : (page_size % 128 == 0);
+  if (!page_ok) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * page_size >= (1LL << 31) || (long long)max_blocks * page_size >= (1LL << 31))
+    return ATTN_ERR_INVALID_ARG;
+  const unsigned long long row_bytes = (unsigned long long)H * d * 2;
+  if ((unsigned long long)num_blocks * page_size * row_bytes >= (1ull << 40)) return ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) != 0; };
+  if (misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) || misaligned(out, 16) ||
+      misaligned(block_table, 4) || misaligned(seq_lens, 4) || (lse && misaligned(lse, 4)))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = (size_t)B * row_bytes;
+  const size_t cache_bytes = (size_t)num_blocks * page_size * row_bytes;
+  if (overlaps(out, q_bytes, q, q_bytes) || overlaps(out, q_bytes, k_cache, cache_bytes) ||
+      overlaps(out, q_bytes, v_cache, cache_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  if (lse) {
+    const size_t lse_bytes = (size_t)B * H * sizeof(float);
+    if (overlaps(lse, lse_bytes, out, q_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
+        overlaps(lse, lse_bytes, k_cache, cache_bytes) || overlaps(lse, lse_bytes, v_cache, cache_bytes))
+      return ATTN_ERR_INVALID_ARG;
+  }
+  return ATTN_OK;
+}
+
 // Same kernels as launch_decode, with the partials in g_noalloc_scratch: no allocation.
 template <int D, bool BF16>
 int launch_decode_noalloc(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
@@ -409,6 +505,28 @@ int attn_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* o
                 : launch_decode_noalloc<128, false>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st);
   return bf16 ? launch_decode_noalloc<64, true>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st)
               : launch_decode_noalloc<64, false>(ds, q, k, v, out, lse, B, H, Nk, scale, splits, st);
+}
+
+int attn_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                          const int* block_table, const int* seq_lens, void* out, float* lse, int B,
+                          int H, int d, int num_blocks, int page_size, int max_blocks, float scale,
+                          int dtype, int splits, attn_stream_t stream) {
+  if (int rc = validate_paged(q, k_cache, v_cache, block_table, seq_lens, out, lse, B, H, d,
+                              num_blocks, page_size, max_blocks, scale, dtype, splits))
+    return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_BF16;
+#define ATTN_PAGED_ARGS                                                                          \
+  ds, q, k_cache, v_cache, block_table, seq_lens, out, lse, B, H, num_blocks, page_size, max_blocks, \
+      scale, splits, st
+  if (d == 128)
+    return bf16 ? launch_decode_paged<128, true>(ATTN_PAGED_ARGS)
+                : launch_decode_paged<128, false>(ATTN_PAGED_ARGS);
+  return bf16 ? launch_decode_paged<64, true>(ATTN_PAGED_ARGS)
+              : launch_decode_paged<64, false>(ATTN_PAGED_ARGS);
+#undef ATTN_PAGED_ARGS
 }
 
 int attn_get_status(attn_stream_t stream) {

@@ -22,18 +22,30 @@
 namespace attn_b200 {
 
 struct DecodeParams {
-  CUtensorMap tm_k;  // [B, Nk, H, D] as 4-D (D, H, Nk, B), box (64, 1, 128, 1), 128B swizzle
-  CUtensorMap tm_v;
+  CUtensorMap tm_k;  // [B, Nk, H, D] as 4-D (D, H, Nk, B), box (64, 1, 128, 1), 128B swizzle;
+  CUtensorMap tm_v;  // paged: the cache [num_blocks * page_size, H, D], box (64, 1, page_rows, 1)
   const void* q;     // [B, 1, H, D]
   float* part;       // [B*H*splits][D + 2]: o[0..D) unnormalised, m (base-2 units), l
   int* status;
-  int B, H, Nk;
+  int B, H, Nk;          // paged: Nk = max_blocks * page_size, the longest sequence the table holds
   int splits;            // key ranges per (b, h)
   int tiles_per_split;   // 128-key tiles per range
   int n_items;           // B * H * splits
   float scale_log2;      // scale * log2(e)
   unsigned long long timeout_ns;
+  // paged key/value cache (kPaged kernels only)
+  const int* block_table;  // [B, max_blocks]: page of the request's keys [i*page_size, (i+1)*page_size)
+  const int* seq_lens;     // [B]: keys of each request
+  int max_blocks, page_size, page_rows, num_blocks;  // page_rows = min(page_size, 128)
 };
+
+// Keys of request b the kernel reads: seq_lens[b] clamped to what its table can hold
+// (Nk = max_blocks * page_size), or Nk for a dense cache.
+template <bool kPaged>
+__device__ __forceinline__ int decode_seq_len(const DecodeParams& p, int b) {
+  if constexpr (kPaged) return min(max(__ldg(p.seq_lens + b), 0), p.Nk);
+  return p.Nk;
+}
 
 template <int D>
 struct DecodeCfg {
@@ -66,7 +78,7 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kPaged = false>
 __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 1)
     attn_decode_partial_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecodeCfg<D>;
@@ -106,8 +118,9 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 1)
         const int bh = item / p.splits;
         const int sp = item - bh * p.splits;
         const int b = bh / p.H, h = bh - b * p.H;
+        const int seq_len = decode_seq_len<kPaged>(p, b);
         const int t0 = sp * p.tiles_per_split;
-        const int t1 = min(ntiles, t0 + p.tiles_per_split);
+        const int t1 = min(min(ntiles, (seq_len + 127) / 128), t0 + p.tiles_per_split);
         for (int tile = t0; tile < t1; ++tile, ++g) {
           const int stage = g % C::kStages;
           const int round = g / C::kStages;
@@ -118,10 +131,30 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 1)
           }
           const uint32_t dst = sbase + stage * C::kStageBytes;
           mbar_arrive_expect_tx(FULL(stage), C::kStageBytes);
-          for (int bx = 0; bx < C::kBoxes; ++bx) {
-            tma_load_4d(dst + bx * C::kBoxBytes, &p.tm_k, FULL(stage), bx * 64, h, tile * 128, b);
-            tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes, &p.tm_v, FULL(stage), bx * 64, h,
-                        tile * 128, b);
+          if constexpr (kPaged) {
+            // the tile's 128 keys come in 128 / page_rows pieces, each from its page; a piece
+            // lands at a multiple of 8 rows, where the 128-byte swizzle pattern restarts
+            for (int key = tile * 128; key < tile * 128 + 128; key += p.page_rows) {
+              const int page = key / p.page_size;
+              // table entries outside [0, num_blocks) are clamped: every read stays in the cache
+              const int phys = key < seq_len
+                                   ? min(max(__ldg(p.block_table + (long long)b * p.max_blocks + page), 0),
+                                         p.num_blocks - 1)
+                                   : 0;
+              const int row = phys * p.page_size + (key - page * p.page_size);
+              const uint32_t off = (uint32_t)(key - tile * 128) * 128;
+              for (int bx = 0; bx < C::kBoxes; ++bx) {
+                tma_load_4d(dst + bx * C::kBoxBytes + off, &p.tm_k, FULL(stage), bx * 64, h, row, 0);
+                tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes + off, &p.tm_v, FULL(stage),
+                            bx * 64, h, row, 0);
+              }
+            }
+          } else {
+            for (int bx = 0; bx < C::kBoxes; ++bx) {
+              tma_load_4d(dst + bx * C::kBoxBytes, &p.tm_k, FULL(stage), bx * 64, h, tile * 128, b);
+              tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes, &p.tm_v, FULL(stage), bx * 64, h,
+                          tile * 128, b);
+            }
           }
         }
       }
@@ -141,8 +174,9 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 1)
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
       const int bh = item / p.splits;
       const int sp = item - bh * p.splits;
+      const int seq_len = decode_seq_len<kPaged>(p, bh / p.H);
       const int t0 = sp * p.tiles_per_split;
-      const int t1 = min(ntiles, t0 + p.tiles_per_split);
+      const int t1 = min(min(ntiles, (seq_len + 127) / 128), t0 + p.tiles_per_split);
 
       // the query row, pre-multiplied by scale*log2(e) (every lane holds all of it)
       float qf[D];
@@ -194,7 +228,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 1)
           a0 = fmaf(qf[c * 8 + 6], f3.x, a0);
           a1 = fmaf(qf[c * 8 + 7], f3.y, a1);
         }
-        const bool valid = tile * 128 + r < p.Nk;
+        const bool valid = tile * 128 + r < seq_len;
         const float s = valid ? (a0 + a1) : -INFINITY;
         const float m_new = fmaxf(m, warp_max(s));
         if (m_new != -INFINITY) {

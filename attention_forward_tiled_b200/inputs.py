@@ -33,6 +33,13 @@ WORKLOADS = {
                    scale=1.0 / math.sqrt(128), seed=5, k_mult=1.0),
 }
 
+# The decode workload over a paged cache: the same 16 requests x 4096 keys, stored in
+# randomly placed 16-key pages (a common serving page size).
+PAGED_WORKLOADS = {
+    "decode_paged16": dict(B=16, H=32, d=128, seq_lens=[4096] * 16, page_size=16, dtype="f16",
+                           scale=1.0 / math.sqrt(128), seed=6),
+}
+
 
 def make_inputs(B, H, Nq, Nk, d, dtype="f16", seed=0, k_mult=1.0, **_):
     """Return CPU tensors (q, k, v) in [B, N, H, d] layout and the given dtype."""
@@ -44,6 +51,31 @@ def make_inputs(B, H, Nq, Nk, d, dtype="f16", seed=0, k_mult=1.0, **_):
         k = k * k_mult
     dt = DTYPES[dtype]
     return q.to(dt), k.to(dt), v.to(dt)
+
+
+def make_paged_inputs(B, H, d, seq_lens, page_size, dtype="f16", seed=0, max_blocks=None,
+                      spare_pages=3):
+    """Seeded paged decode inputs (CPU tensors): q [B, 1, H, d]; k_cache, v_cache
+    [num_blocks, page_size, H, d]; block_table [B, max_blocks] int32 (-1 past each
+    sequence); seq_lens [B] int32.  The pages of all requests (plus `spare_pages`
+    unused ones) are a random permutation of the cache, so no request's pages are
+    contiguous.  Draw order: q, the page permutation, k_cache, v_cache."""
+    g = torch.Generator("cpu").manual_seed(int(seed))
+    npages = [(int(L) + page_size - 1) // page_size for L in seq_lens]
+    max_blocks = max(max(npages), 1) if max_blocks is None else int(max_blocks)
+    num_blocks = sum(npages) + spare_pages
+    q = torch.randn(B, 1, H, d, generator=g, dtype=torch.float32)
+    perm = torch.randperm(num_blocks, generator=g)
+    k_cache = torch.randn(num_blocks, page_size, H, d, generator=g, dtype=torch.float32)
+    v_cache = torch.randn(num_blocks, page_size, H, d, generator=g, dtype=torch.float32)
+    block_table = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    nxt = 0
+    for b, n in enumerate(npages):
+        block_table[b, :n] = perm[nxt:nxt + n].to(torch.int32)
+        nxt += n
+    dt = DTYPES[dtype]
+    return (q.to(dt), k_cache.to(dt), v_cache.to(dt), block_table,
+            torch.tensor([int(L) for L in seq_lens], dtype=torch.int32))
 
 
 def workload_inputs(name):

@@ -132,6 +132,44 @@ ATTN_API int attn_fwd_decode_noalloc(const void* q, const void* k, const void* v
                                      int dtype, int splits, attn_stream_t stream);
 
 /*
+ * attn_fwd_decode_paged -- attn_fwd_decode over a paged key/value cache.
+ *
+ * One query row per request; request b's keys and values are its first
+ * seq_lens[b] cache rows, stored page by page: keys [i*page_size,
+ * (i+1)*page_size) of request b are rows [0, page_size) of cache page
+ * block_table[b*max_blocks + i].  This is the decode metadata of the vLLM
+ * MiniMax-M3 indexer page ("PR #45743 完整报告", section "关键源码片段":
+ * per-request int32 seq_lens and a block table); the page size is the caller's.
+ * The result equals attn_fwd_decode on each request's keys gathered densely.
+ *
+ *   q            [B, 1, H, d]                          dtype   (read)
+ *   k_cache      [num_blocks, page_size, H, d]         dtype   (read)
+ *   v_cache      [num_blocks, page_size, H, d]         dtype   (read)
+ *   block_table  [B, max_blocks]                       int32   (read, DEVICE memory)
+ *   seq_lens     [B]                                   int32   (read, DEVICE memory)
+ *   out          [B, 1, H, d]                          dtype   (written)
+ *   lse          [B, H] float32 (written) or NULL
+ *   page_size: 8, 16, 32, 64 or a multiple of 128;  max_blocks * page_size and
+ *   num_blocks * page_size below 2^31;  splits: 0 = automatic, else the number
+ *   of key ranges per (b, h) (sized for max_blocks * page_size keys).
+ *
+ * seq_lens[b] is clamped to [0, max_blocks * page_size]; a request with no key
+ * gets O = 0 and lse = -inf.  Table entries of pages holding keys below
+ * seq_lens[b] must lie in [0, num_blocks) (others are clamped into it, so reads
+ * stay inside the cache); entries past the sequence are not read.  Alignment
+ * as attn_fwd, plus 4 bytes for block_table and seq_lens.  The workspace of
+ * B*H*splits*(d+2)*4 bytes is taken stream-ordered as for attn_fwd_decode.
+ *
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (d, dtype, page
+ * size or device) or ATTN_ERR_CUDA; asynchronous like attn_fwd.
+ */
+ATTN_API int attn_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                                   const int* block_table, const int* seq_lens, void* out,
+                                   float* lse, int B, int H, int d, int num_blocks, int page_size,
+                                   int max_blocks, float scale, int dtype, int splits,
+                                   attn_stream_t stream);
+
+/*
  * attn_get_status -- synchronises `stream`, then returns and clears the
  * current device's status word: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel
  * since the last call gave up on a pipeline wait (its outputs are then

@@ -102,6 +102,34 @@ def test_decode_entry_validation(lib):
     assert lib.attn_fwd_decode(Q, K, V, O, L, 1, 2, 128, 80, 0.1, 0, 0, NULL) == attn.ATTN_ERR_UNSUPPORTED
 
 
+BT, SL = ctypes.c_void_p(0x700000000), ctypes.c_void_p(0x800000000)  # block table, seq lens
+
+
+def paged(lib, q=Q, kc=K, vc=V, bt=BT, sl=SL, o=O, lse=L, B=2, H=4, d=128, num_blocks=64,
+          page_size=16, max_blocks=32, scale=0.1, dtype=0, splits=0):
+    return lib.attn_fwd_decode_paged(q, kc, vc, bt, sl, o, lse, B, H, d, num_blocks, page_size,
+                                     max_blocks, scale, dtype, splits, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bt=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(sl=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(kc=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(num_blocks=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(max_blocks=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(splits=-1), attn.ATTN_ERR_INVALID_ARG),
+    (dict(page_size=24), attn.ATTN_ERR_UNSUPPORTED),    # 128 is no multiple of 24
+    (dict(page_size=4), attn.ATTN_ERR_UNSUPPORTED),     # below 8 rows
+    (dict(page_size=192), attn.ATTN_ERR_UNSUPPORTED),   # above 128: multiples of 128 only
+    (dict(d=80), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(max_blocks=1 << 28, page_size=16), attn.ATTN_ERR_INVALID_ARG),  # table length >= 2^31 keys
+    (dict(bt=ctypes.c_void_p(0x700000002)), attn.ATTN_ERR_INVALID_ARG),   # misaligned table
+    (dict(o=ctypes.c_void_p(0x200000000 + 4096)), attn.ATTN_ERR_INVALID_ARG),  # out inside k_cache
+])
+def test_paged_decode_entry_validation(lib, kw, code):
+    assert paged(lib, **kw) == code
+
+
 def test_prefill_entry_validation(lib):
     assert lib.attn_fwd_prefill(Q, K, V, NULL, L, 1, 2, 64, 64, 64, 0, 0.1, 0, NULL) == attn.ATTN_ERR_INVALID_ARG
     assert lib.attn_fwd_prefill(Q, K, V, O, L, 1, 2, 64, 64, 32, 0, 0.1, 1, NULL) == attn.ATTN_ERR_UNSUPPORTED
