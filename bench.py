@@ -193,11 +193,18 @@ def workload_config(name, w):
 # ---------------------------------------------------------------------------
 def time_gpu_steps(step, K, stream, flush=None):
     """Per-step device times (ms) from CUDA events on `stream`; an L2 flush, when
-    given, runs between steps outside the timed intervals."""
+    given, runs between steps outside the timed intervals.
+
+    The stream first runs a device-side spin long enough for the host to enqueue all K
+    steps, so the timed steps run back to back on the GPU instead of waiting for a host
+    thread (Python launch overhead, the clock sampler's share of the interpreter) between
+    short launches; the spin itself is outside every timed interval."""
     import torch
+    spin_cycles = max(10_000_000, K * 1_000_000)  # >= 5 ms at 2 GHz, 0.5 ms of host time per step
     if flush is None:  # back-to-back steps: one event between consecutive steps
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
         with torch.cuda.stream(stream):
+            torch.cuda._sleep(spin_cycles)
             evs[0].record(stream)
             for i in range(K):
                 step()
@@ -207,6 +214,7 @@ def time_gpu_steps(step, K, stream, flush=None):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     with torch.cuda.stream(stream):
+        torch.cuda._sleep(spin_cycles)
         for i in range(K):
             flush()
             starts[i].record(stream)
