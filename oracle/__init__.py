@@ -45,6 +45,9 @@ def load(path=None):
     lib.oracle_attn_fwd_blocked_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i, i]
     lib.oracle_attn_fwd_blocked_f64.restype = i
     lib.oracle_attn_probs_f64.argtypes = [dp, dp, dp, i, i, i, i, i, i, d]
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.oracle_attn_fwd_relpos_f64.restype = i
+    lib.oracle_attn_fwd_relpos_f64.argtypes = [dp, dp, dp, dp, ip, dp, dp, i, i, i, i, i, i, i, d]
     lib.oracle_attn_probs_f64.restype = i
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = i
@@ -114,6 +117,27 @@ def attn_probs(q, k, causal=False, scale=None, lib=None):
     if rc != 0:
         raise RuntimeError(f"oracle_attn_probs_f64 failed ({rc})")
     return p
+
+
+def attn_fwd_relpos(q, k, v, emb, dist, causal=False, scale=None, lib=None):
+    """Attention whose scores carry the relative-position term scale * q_i . emb[dist[i, j]]
+    (emb [n_emb, d], dist int [Nq, Nk], shared by every batch and head)."""
+    q, k, v, emb = _f64(q), _f64(k), _f64(v), _f64(emb)
+    B, H, Nq, Nk, d = _shapes(q, k, v)
+    if hasattr(dist, "detach"):
+        dist = dist.detach().cpu().numpy()
+    dist = np.ascontiguousarray(dist, dtype=np.int32)
+    if dist.shape != (Nq, Nk) or emb.ndim != 2 or emb.shape[1] != d:
+        raise ValueError("dist must be [Nq, Nk] and emb [n_emb, d]")
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    o = np.zeros((B, Nq, H, d), dtype=np.float64)
+    lse = np.zeros((B, H, Nq), dtype=np.float64)
+    rc = (lib or load()).oracle_attn_fwd_relpos_f64(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(emb), dist.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+        _ptr(o), _ptr(lse), B, H, Nq, Nk, d, emb.shape[0], int(bool(causal)), scale)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_relpos_f64 failed ({rc})")
+    return o, lse
 
 
 def num_threads():

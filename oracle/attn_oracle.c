@@ -230,6 +230,80 @@ int oracle_attn_fwd_blocked_f64(const double* q, const double* k, const double* 
     return err;
 }
 
+/*
+ * Attention with a relative-position score term (the Granite-Speech conformer
+ * attention of the vLLM page "PR #42933", section "关键源码片段": the term
+ * einsum("bnhid,ijd->bnhij", q, rel_pos_emb) * scale is added to the scores that
+ * masking and SDPA then use).  rel_pos_emb[i, j, :] is the embedding row
+ * emb[dist[i, j]] of a relative-distance index, as the page builds it from
+ * `dist`; dist is an input here (int32 [Nq, Nk], values in [0, n_emb)), emb is
+ * [n_emb, d], both shared by every batch and head:
+ *
+ *   s_ij = scale * (sum_t q[b,i,h,t] * k[b,j,h,t] + sum_t q[b,i,h,t] * emb[dist[i,j], t])
+ *
+ * over allowed j, then the same softmax, output and lse as oracle_attn_fwd_f64.
+ */
+int oracle_attn_fwd_relpos_f64(const double* q, const double* k, const double* v,
+                               const double* emb, const int* dist, double* o, double* lse,
+                               int B, int H, int Nq, int Nk, int d, int n_emb, int causal,
+                               double scale)
+{
+    if (check_args(B, H, Nq, Nk, d) || n_emb <= 0) return -1;
+    for (long ij = 0; ij < (long)Nq * Nk; ++ij)
+        if (dist[ij] < 0 || dist[ij] >= n_emb) return -3;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        double* S = (double*)malloc(sizeof(double) * (size_t)Nq * (size_t)Nk);
+        if (!S) {
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        for (long i = 0; i < Nq; ++i) {
+            const double* qi = q + IDX4(b, i, h, 0, Nq, H, d);
+            for (long j = 0; j < Nk; ++j) {
+                if (!is_allowed(i, j, Nq, Nk, causal)) {
+                    S[i * Nk + j] = -INFINITY;
+                    continue;
+                }
+                const double* e = emb + (long)dist[i * Nk + j] * d;
+                double rel = 0.0;
+                for (int t = 0; t < d; ++t) rel += qi[t] * e[t];
+                S[i * Nk + j] = scale * (dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + rel);
+            }
+        }
+        /* softmax over each row, output and lse, as in oracle_attn_fwd_f64 */
+        for (long i = 0; i < Nq; ++i) {
+            double* row = S + i * Nk;
+            double mx = -INFINITY;
+            for (long j = 0; j < Nk; ++j) mx = row[j] > mx ? row[j] : mx;
+            double* out_i = o + IDX4(b, i, h, 0, Nq, H, d);
+            double* lse_i = lse + ((long)b * H + h) * Nq + i;
+            if (mx == -INFINITY) {
+                for (int t = 0; t < d; ++t) out_i[t] = 0.0;
+                *lse_i = -INFINITY;
+                continue;
+            }
+            double denom = 0.0;
+            for (long j = 0; j < Nk; ++j) {
+                row[j] = (row[j] == -INFINITY) ? 0.0 : exp(row[j] - mx);
+                denom += row[j];
+            }
+            for (int t = 0; t < d; ++t) {
+                double num = 0.0;
+                for (long j = 0; j < Nk; ++j)
+                    if (row[j] != 0.0) num += row[j] * v[IDX4(b, j, h, t, Nk, H, d)];
+                out_i[t] = num / denom;
+            }
+            *lse_i = mx + log(denom);
+        }
+        free(S);
+    }
+    return err;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -33,7 +33,19 @@ MUTANTS = {
     "blocked_l_not_rescaled": [("l[r] = alpha * l[r] + bsum;", "l[r] = l[r] + bsum;")],
     "blocked_acc_not_rescaled": [("for (int t = 0; t < d; ++t) acc[r * d + t] *= alpha;",
                                   "for (int t = 0; t < d; ++t) acc[r * d + t] *= 1.0;")],
+    # the relative-position term of oracle_attn_fwd_relpos_f64
+    "relpos_term_unscaled": [("S[i * Nk + j] = scale * (dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + rel);",
+                              "S[i * Nk + j] = scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + rel;")],
+    "relpos_dist_transposed": [("const double* e = emb + (long)dist[i * Nk + j] * d;",
+                                "const double* e = emb + (long)dist[(j % Nq) * Nk + (i % Nk)] * d;")],
+    "relpos_term_uses_key": [("for (int t = 0; t < d; ++t) rel += qi[t] * e[t];",
+                              "for (int t = 0; t < d; ++t) rel += k[IDX4(b, j, h, t, Nk, H, d)] * e[t];")],
+    "relpos_term_dropped": [("S[i * Nk + j] = scale * (dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + rel);",
+                             "S[i * Nk + j] = scale * (dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + 0.0 * rel);")],
 }
+
+PIN_FILES = [os.path.join(ROOT, "tests", "test_oracle.py"),
+             os.path.join(ROOT, "tests", "test_oracle_relpos.py")]
 
 RUNNER = textwrap.dedent("""
     import sys
@@ -43,8 +55,7 @@ RUNNER = textwrap.dedent("""
     lib = oracle.load({lib!r})
     oracle._lib, oracle._lib_path = lib, build.LIB
     import pytest
-    sys.exit(pytest.main(["-x", "-q", "-p", "no:cacheprovider",
-                          {tests!r}]))
+    sys.exit(pytest.main(["-x", "-q", "-p", "no:cacheprovider"] + {tests!r}))
 """)
 
 
@@ -57,7 +68,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     mpath = tmp_path / f"{name}.c"
     mpath.write_text(src)
     lib = obuild.build(src=str(mpath), out=str(tmp_path / f"lib{name}.so"))
-    code = RUNNER.format(root=ROOT, lib=lib, tests=os.path.join(ROOT, "tests", "test_oracle.py"))
+    code = RUNNER.format(root=ROOT, lib=lib, tests=PIN_FILES)
     res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
                          cwd=str(tmp_path), timeout=600)
     assert res.returncode != 0, f"mutant {name} survived the pin suite:\n{res.stdout[-2000:]}"
@@ -66,7 +77,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
 def test_unmutated_copy_passes(tmp_path):
     """Control: the same harness on an unmodified copy passes."""
     lib = obuild.build(src=obuild.SRC, out=str(tmp_path / "libcopy.so"))
-    code = RUNNER.format(root=ROOT, lib=lib, tests=os.path.join(ROOT, "tests", "test_oracle.py"))
+    code = RUNNER.format(root=ROOT, lib=lib, tests=PIN_FILES)
     res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
                          cwd=str(tmp_path), timeout=600)
     assert res.returncode == 0, res.stdout[-3000:] + res.stderr[-2000:]
