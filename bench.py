@@ -8,9 +8,12 @@ A step is one call of the whole forward (the tiled prefill kernel for the
 prefill workloads; the split-KV partial and combine kernels for decode) over
 one batch of seeded synthetic inputs already resident in HBM.  Timing: W
 untimed warm-up steps, then exactly K steps bracketed by a barrier and a device
-synchronise, CUDA events on the launching stream, max over ranks.  Every rank
-runs an independent replica of the workload (the forward of one (b, h) never
-talks to another, so there is no data-path collective): scaling is weak.
+synchronise, CUDA events on the launching stream, max over ranks; the stream spins
+on the device while the host enqueues the K steps, so they run back to back (the
+spin is outside the timed intervals).  Every rank runs an independent replica of
+the workload (the forward of one (b, h) never talks to another, so there is no
+data-path collective): scaling is weak.  `extra` carries the decode, causal8k and
+bf16_k3 workloads and the decode over a 16-key-page cache, each with its roofline.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the method available here) on bounded samples of the same workload.
