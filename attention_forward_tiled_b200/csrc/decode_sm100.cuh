@@ -109,61 +109,69 @@ __global__ void __launch_bounds__(DecodeCfg<D>::kThreads, 1)
 
   if (warp == C::kProducerWarp) {
     // ======================= TMA producer =======================
+    // The whole warp walks the ring; lane 0 waits, arms the stage and issues dense tiles.
+    // A paged tile comes in 128 / page_rows pieces, one lane per piece, so the pieces'
+    // block-table reads overlap instead of following one another.
     if (lane == 0) {
       tma_prefetch_map(&p.tm_k);
       tma_prefetch_map(&p.tm_v);
-      int g = 0;  // ring position across all items of this CTA
-      bool stop = false;
-      for (int item = blockIdx.x; item < p.n_items && !stop; item += gridDim.x) {
-        const int bh = item / p.splits;
-        const int sp = item - bh * p.splits;
-        const int b = bh / p.H, h = bh - b * p.H;
-        const int seq_len = decode_seq_len<kPaged>(p, b);
-        const int t0 = sp * p.tiles_per_split;
-        const int t1 = min(min(ntiles, (seq_len + 127) / 128), t0 + p.tiles_per_split);
-        for (int tile = t0; tile < t1; ++tile, ++g) {
-          const int stage = g % C::kStages;
-          const int round = g / C::kStages;
-          if (round > 0) mbar_wait(EMPTY(stage), (round - 1) & 1, wctx);
-          if (*abort_flag) {
-            stop = true;
-            break;
-          }
-          const uint32_t dst = sbase + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(FULL(stage), C::kStageBytes);
-          if constexpr (kPaged) {
-            // the tile's 128 keys come in 128 / page_rows pieces, each from its page; a piece
-            // lands at a multiple of 8 rows, where the 128-byte swizzle pattern restarts
-            for (int key = tile * 128; key < tile * 128 + 128; key += p.page_rows) {
-              const int page = key / p.page_size;
-              // table entries outside [0, num_blocks) are clamped: every read stays in the cache
-              const int phys = key < seq_len
-                                   ? min(max(__ldg(p.block_table + (long long)b * p.max_blocks + page), 0),
-                                         p.num_blocks - 1)
-                                   : 0;
-              const int row = phys * p.page_size + (key - page * p.page_size);
-              const uint32_t off = (uint32_t)(key - tile * 128) * 128;
-              for (int bx = 0; bx < C::kBoxes; ++bx) {
-                tma_load_4d(dst + bx * C::kBoxBytes + off, &p.tm_k, FULL(stage), bx * 64, h, row, 0);
-                tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes + off, &p.tm_v, FULL(stage),
-                            bx * 64, h, row, 0);
-              }
-            }
-          } else {
+    }
+    int g = 0;  // ring position across all items of this CTA
+    bool stop = false;
+    for (int item = blockIdx.x; item < p.n_items && !stop; item += gridDim.x) {
+      const int bh = item / p.splits;
+      const int sp = item - bh * p.splits;
+      const int b = bh / p.H, h = bh - b * p.H;
+      const int seq_len = decode_seq_len<kPaged>(p, b);
+      const int t0 = sp * p.tiles_per_split;
+      const int t1 = min(min(ntiles, (seq_len + 127) / 128), t0 + p.tiles_per_split);
+      for (int tile = t0; tile < t1; ++tile, ++g) {
+        const int stage = g % C::kStages;
+        const int round = g / C::kStages;
+        if (round > 0) mbar_wait(EMPTY(stage), (round - 1) & 1, wctx);
+        __syncwarp();
+        if (warp_flag(abort_flag)) {
+          stop = true;
+          break;
+        }
+        const uint32_t dst = sbase + stage * C::kStageBytes;
+        if (lane == 0) mbar_arrive_expect_tx(FULL(stage), C::kStageBytes);
+        __syncwarp();
+        if constexpr (kPaged) {
+          // piece `lane` holds keys [key, key + page_rows) of one page; it lands at a multiple
+          // of 8 rows, where the 128-byte swizzle pattern restarts
+          if (lane < 128 / p.page_rows) {
+            const int key = tile * 128 + lane * p.page_rows;
+            const int page = key / p.page_size;
+            // table entries outside [0, num_blocks) are clamped: every read stays in the cache
+            const int phys = key < seq_len
+                                 ? min(max(__ldg(p.block_table + (long long)b * p.max_blocks + page), 0),
+                                       p.num_blocks - 1)
+                                 : 0;
+            const int row = phys * p.page_size + (key - page * p.page_size);
+            const uint32_t off = (uint32_t)(lane * p.page_rows) * 128;
             for (int bx = 0; bx < C::kBoxes; ++bx) {
-              tma_load_4d(dst + bx * C::kBoxBytes, &p.tm_k, FULL(stage), bx * 64, h, tile * 128, b);
-              tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes, &p.tm_v, FULL(stage), bx * 64, h,
-                          tile * 128, b);
+              tma_load_4d(dst + bx * C::kBoxBytes + off, &p.tm_k, FULL(stage), bx * 64, h, row, 0);
+              tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes + off, &p.tm_v, FULL(stage),
+                          bx * 64, h, row, 0);
             }
+          }
+        } else if (lane == 0) {
+          for (int bx = 0; bx < C::kBoxes; ++bx) {
+            tma_load_4d(dst + bx * C::kBoxBytes, &p.tm_k, FULL(stage), bx * 64, h, tile * 128, b);
+            tma_load_4d(dst + C::kTileBytes + bx * C::kBoxBytes, &p.tm_v, FULL(stage), bx * 64, h,
+                        tile * 128, b);
           }
         }
-      }
-      if (*abort_flag) {
-        const int first = g > C::kStages ? g - C::kStages : 0;
-        for (int i = first; i < g; ++i)
-          mbar_wait_drain(FULL(i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+        __syncwarp();
       }
     }
+    if (lane == 0 && *abort_flag) {
+      const int first = g > C::kStages ? g - C::kStages : 0;
+      for (int i = first; i < g; ++i)
+        mbar_wait_drain(FULL(i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+    }
+    __syncwarp();
   } else {
     // ======================= consumer warps 0-3 =======================
     constexpr int E = C::kElemsPerLane;

@@ -52,14 +52,20 @@ def load_peaks():
     return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def kernel_source_sha():
-    """Hash of the CUDA sources' code (comments and blank space removed): ties a committed
-    ncu traffic figure to the kernel it measured, so editing a comment does not orphan it."""
+# Sources each kind of kernel is built from (its launcher lives in attn_api.cu).
+KERNEL_SOURCES = {
+    "prefill": ("prefill_sm100.cuh", "sm100_ptx.cuh", "exp2_poly.cuh", "attn_api.cu"),
+    "decode": ("decode_sm100.cuh", "sm100_ptx.cuh", "attn_api.cu"),
+}
+
+
+def kernel_source_sha(kind="prefill"):
+    """Hash of the code (comments and blank space removed) of the sources one kind of
+    kernel is built from: ties a committed ncu traffic figure to the kernel it measured,
+    so editing a comment, or the other kernel, does not orphan it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_forward_tiled_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if not name.endswith((".cu", ".cuh", ".h")):
-            continue
+    for name in KERNEL_SOURCES[kind]:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -71,7 +77,8 @@ def kernel_source_sha():
 
 def committed_traffic(workload):
     """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel."""
-    sha = kernel_source_sha()
+    kind = "decode" if workload.startswith("decode") else "prefill"
+    sha = kernel_source_sha(kind)
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
