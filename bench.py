@@ -303,6 +303,7 @@ def measure_workload(name, K, W, world, device, peaks, want_e2e=True):
                                         "sustained %.1f" % (peaks["source"], peaks["bf16_tflops_sustained"])}
         res["gpu_launches"] = K
     res["min_ms"] = min(t_steps)
+    res["median_ms"] = statistics.median(t_steps)
 
     if want_e2e:
         runner = attn.HostRunner(w["B"], w["H"], w["Nq"], w["Nk"], w["d"], q.dtype, device=device,
@@ -455,6 +456,8 @@ def run_ours(args):
         "steps": K,
         "warmup": W,
         "ms_per_step": main["ms_per_step"],
+        "ms_per_step_median": main["median_ms"],  # this rank's steps
+        "ms_per_step_min": main["min_ms"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
