@@ -45,6 +45,8 @@ def load(path=None):
     lib.oracle_attn_fwd_blocked_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i, i]
     lib.oracle_attn_fwd_blocked_f64.restype = i
     lib.oracle_attn_probs_f64.argtypes = [dp, dp, dp, i, i, i, i, i, i, d]
+    lib.oracle_attn_bwd_f64.restype = i
+    lib.oracle_attn_bwd_f64.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, d]
     ip = ctypes.POINTER(ctypes.c_int)
     lib.oracle_attn_fwd_relpos_f64.restype = i
     lib.oracle_attn_fwd_relpos_f64.argtypes = [dp, dp, dp, dp, ip, dp, dp, i, i, i, i, i, i, i, d]
@@ -138,6 +140,22 @@ def attn_fwd_relpos(q, k, v, emb, dist, causal=False, scale=None, lib=None):
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd_relpos_f64 failed ({rc})")
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, causal=False, scale=None, lib=None):
+    """Gradients (dq, dk, dv) of attn_fwd's O for an upstream gradient dout [B, Nq, H, d]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, Nq, Nk, d = _shapes(q, k, v)
+    if dout.shape != q.shape:
+        raise ValueError("dout must have q's shape")
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    rc = (lib or load()).oracle_attn_bwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq),
+                                             _ptr(dk), _ptr(dv), B, H, Nq, Nk, d,
+                                             int(bool(causal)), scale)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd_f64 failed ({rc})")
+    return dq, dk, dv
 
 
 def num_threads():

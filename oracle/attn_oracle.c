@@ -304,6 +304,100 @@ int oracle_attn_fwd_relpos_f64(const double* q, const double* k, const double* v
     return err;
 }
 
+/*
+ * Gradients of the forward above (the step after it on the pages: the ai6s.net
+ * article notes that eager attention keeps the N x N matrix for the backward
+ * pass, section "传统注意力的显存陷阱"), from the definition by the chain rule,
+ * for an upstream gradient dO of O:
+ *
+ *   P = softmax(S) row-wise (S = scale * Q K^T, masked),  O = P V
+ *   dV = P^T dO
+ *   dP = dO V^T
+ *   dS_ij = P_ij * (dP_ij - sum_t dO_it O_it)      (softmax Jacobian; sum_t dO.O = sum_j P_ij dP_ij)
+ *   dQ = scale * dS K,   dK = scale * dS^T Q
+ *
+ * Masked entries have P = 0, hence dS = 0; a row with no allowed key has O = 0 and
+ * contributes nothing.  Layouts as the forward; dq [B,Nq,H,d], dk and dv [B,Nk,H,d].
+ */
+int oracle_attn_bwd_f64(const double* q, const double* k, const double* v, const double* dout,
+                        double* dq, double* dk, double* dv,
+                        int B, int H, int Nq, int Nk, int d, int causal, double scale)
+{
+    if (check_args(B, H, Nq, Nk, d)) return -1;
+    memset(dq, 0, sizeof(double) * (size_t)B * Nq * H * d);
+    memset(dk, 0, sizeof(double) * (size_t)B * Nk * H * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * Nk * H * d);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        double* P = (double*)malloc(sizeof(double) * (size_t)Nq * (size_t)Nk);
+        double* dP = (double*)malloc(sizeof(double) * (size_t)Nq * (size_t)Nk);
+        if (!P || !dP) {
+            free(P);
+            free(dP);
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        /* P row by row */
+        for (long i = 0; i < Nq; ++i) {
+            double* Pi = P + i * Nk;
+            double top = -INFINITY;
+            for (long j = 0; j < Nk; ++j) {
+                Pi[j] = is_allowed(i, j, Nq, Nk, causal) ? scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d)
+                                                          : -INFINITY;
+                if (Pi[j] > top) top = Pi[j];
+            }
+            if (top == -INFINITY) {
+                for (long j = 0; j < Nk; ++j) Pi[j] = 0.0;
+                continue;
+            }
+            double z = 0.0;
+            for (long j = 0; j < Nk; ++j) {
+                Pi[j] = (Pi[j] == -INFINITY) ? 0.0 : exp(Pi[j] - top);
+                z += Pi[j];
+            }
+            for (long j = 0; j < Nk; ++j) Pi[j] /= z;
+        }
+        /* dV = P^T dO and dP = dO V^T */
+        for (long i = 0; i < Nq; ++i) {
+            const double* doi = dout + IDX4(b, i, h, 0, Nq, H, d);
+            for (long j = 0; j < Nk; ++j) {
+                const double pij = P[i * Nk + j];
+                const double* vj = v + IDX4(b, j, h, 0, Nk, H, d);
+                double* dvj = dv + IDX4(b, j, h, 0, Nk, H, d);
+                double g = 0.0;
+                for (int t = 0; t < d; ++t) {
+                    dvj[t] += pij * doi[t];
+                    g += doi[t] * vj[t];
+                }
+                dP[i * Nk + j] = g;
+            }
+        }
+        /* dS, then dQ and dK */
+        for (long i = 0; i < Nq; ++i) {
+            double delta = 0.0;  /* sum_j P_ij dP_ij */
+            for (long j = 0; j < Nk; ++j) delta += P[i * Nk + j] * dP[i * Nk + j];
+            const double* qi = q + IDX4(b, i, h, 0, Nq, H, d);
+            double* dqi = dq + IDX4(b, i, h, 0, Nq, H, d);
+            for (long j = 0; j < Nk; ++j) {
+                const double ds = P[i * Nk + j] * (dP[i * Nk + j] - delta);
+                if (ds == 0.0) continue;
+                const double* krow = k + IDX4(b, j, h, 0, Nk, H, d);
+                double* dkj = dk + IDX4(b, j, h, 0, Nk, H, d);
+                for (int t = 0; t < d; ++t) {
+                    dqi[t] += scale * ds * krow[t];
+                    dkj[t] += scale * ds * qi[t];
+                }
+            }
+        }
+        free(P);
+        free(dP);
+    }
+    return err;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

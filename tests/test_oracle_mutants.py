@@ -42,10 +42,17 @@ MUTANTS = {
                               "for (int t = 0; t < d; ++t) rel += k[IDX4(b, j, h, t, Nk, H, d)] * e[t];")],
     "relpos_term_dropped": [("S[i * Nk + j] = scale * (dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + rel);",
                              "S[i * Nk + j] = scale * (dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) + 0.0 * rel);")],
+    # the backward oracle
+    "bwd_no_delta": [("const double ds = P[i * Nk + j] * (dP[i * Nk + j] - delta);",
+                      "const double ds = P[i * Nk + j] * dP[i * Nk + j];")],
+    "bwd_dq_unscaled": [("dqi[t] += scale * ds * krow[t];", "dqi[t] += ds * krow[t];")],
+    "bwd_dk_uses_key": [("dkj[t] += scale * ds * qi[t];", "dkj[t] += scale * ds * krow[t];")],
+    "bwd_dv_transposed": [("dvj[t] += pij * doi[t];", "dvj[t] += pij * vj[t];")],
 }
 
 PIN_FILES = [os.path.join(ROOT, "tests", "test_oracle.py"),
-             os.path.join(ROOT, "tests", "test_oracle_relpos.py")]
+             os.path.join(ROOT, "tests", "test_oracle_relpos.py"),
+             os.path.join(ROOT, "tests", "test_oracle_bwd.py")]
 
 RUNNER = textwrap.dedent("""
     import sys
