@@ -14,6 +14,10 @@ Functions
 attn_fwd(q, k, v, causal, scale)            -> (o, lse)   definition order
 attn_fwd_blocked(q, k, v, causal, scale, block_m=128, block_n=64) -> (o, lse)
 attn_probs(q, k, causal, scale)             -> p [B, H, Nq, Nk]
+attn_fwd_relpos(q, k, v, emb, dist, causal, scale) -> (o, lse)   relative-position term
+attn_bwd(q, k, v, dout, causal, scale)      -> (dq, dk, dv)
+indexer_score(q, kp, w, mask)               -> score [B, T, P]   lightning indexer
+topk(score, k)                              -> idx [..., k]
 num_threads() / set_num_threads(n)
 
 Layouts: q, o [B, Nq, H, d]; k, v [B, Nk, H, d]; lse [B, H, Nq].
@@ -51,6 +55,10 @@ def load(path=None):
     lib.oracle_attn_fwd_relpos_f64.restype = i
     lib.oracle_attn_fwd_relpos_f64.argtypes = [dp, dp, dp, dp, ip, dp, dp, i, i, i, i, i, i, i, d]
     lib.oracle_attn_probs_f64.restype = i
+    lib.oracle_indexer_score_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i]
+    lib.oracle_indexer_score_f64.restype = i
+    lib.oracle_topk_f64.argtypes = [dp, i, i, i, ip]
+    lib.oracle_topk_f64.restype = i
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = i
     lib.oracle_set_num_threads.argtypes = [i]
@@ -158,6 +166,44 @@ def attn_bwd(q, k, v, dout, causal=False, scale=None, lib=None):
     return dq, dk, dv
 
 
+def indexer_score(q, kp, w, mask=None, lib=None):
+    """Lightning-indexer score [B, T, P] = sum_h w[b,t,h] * relu(q[b,t,h] . kp[b,p]) + mask
+    (q [B, T, H, d], kp [B, P, d], w [B, T, H], mask [B, T, P] or None)."""
+    q, kp, w = _f64(q), _f64(kp), _f64(w)
+    if q.ndim != 4 or kp.ndim != 3 or w.ndim != 3:
+        raise ValueError("q must be [B, T, H, d], kp [B, P, d] and w [B, T, H]")
+    B, T, H, d = q.shape
+    P = kp.shape[1]
+    if kp.shape != (B, P, d) or w.shape != (B, T, H):
+        raise ValueError("kp must be [B, P, d] and w [B, T, H] with q's B, T, H, d")
+    mptr = None
+    if mask is not None:
+        mask = _f64(mask)
+        if mask.shape != (B, T, P):
+            raise ValueError("mask must be [B, T, P]")
+        mptr = _ptr(mask)
+    score = np.zeros((B, T, P), dtype=np.float64)
+    rc = (lib or load()).oracle_indexer_score_f64(_ptr(q), _ptr(kp), _ptr(w), mptr, _ptr(score),
+                                                  B, T, H, P, d)
+    if rc != 0:
+        raise RuntimeError(f"oracle_indexer_score_f64 failed ({rc})")
+    return score
+
+
+def topk(score, k, lib=None):
+    """Positions of the k largest finite entries of each row of score [..., P], largest
+    first, ties lowest position first; -1 where a row has fewer than k finite entries."""
+    score = _f64(score)
+    lead, P = score.shape[:-1], score.shape[-1]
+    R = int(np.prod(lead)) if lead else 1
+    idx = np.zeros((R, int(k)), dtype=np.int32)
+    rc = (lib or load()).oracle_topk_f64(_ptr(score), R, P, int(k),
+                                         idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int)))
+    if rc != 0:
+        raise RuntimeError(f"oracle_topk_f64 failed ({rc})")
+    return idx.reshape(*lead, int(k))
+
+
 def num_threads():
     return load().oracle_num_threads()
 
@@ -166,4 +212,5 @@ def set_num_threads(n):
     load().oracle_set_num_threads(int(n))
 
 
-__all__ = ["attn_fwd", "attn_fwd_blocked", "attn_probs", "num_threads", "set_num_threads", "load"]
+__all__ = ["attn_fwd", "attn_fwd_blocked", "attn_probs", "attn_fwd_relpos", "attn_bwd",
+           "indexer_score", "topk", "num_threads", "set_num_threads", "load"]

@@ -398,6 +398,83 @@ int oracle_attn_bwd_f64(const double* q, const double* k, const double* v, const
     return err;
 }
 
+/*
+ * Lightning-indexer score (the aispot.cmou.io report "llama.cpp 最佳化 lightning
+ * indexer 視訊記憶體與多後端支援", release b11372, entry "compute the indexer score
+ * with the lightning indexer"): every query token scores every pooled key by the
+ * rectified dot product of each of its indexer heads with that key, weighted per
+ * head and summed over heads; the keys have no head axis (one key row serves all
+ * heads).  An additive pool mask (0 or -inf) follows the sum:
+ *
+ *   score[b,t,p] = sum_h w[b,t,h] * max(0, sum_c q[b,t,h,c] * kp[b,p,c]) + mask[b,t,p]
+ *
+ * The report's unweighted variant is w = 1/sqrt(d) for every head.  Readings: the
+ * weights may differ per token as well as per head (the per-head case has equal
+ * rows); the mask is per (token, pool entry) and may be NULL (no mask).
+ * Layouts: q [B, T, H, d], kp [B, P, d], w [B, T, H], mask and score [B, T, P].
+ */
+int oracle_indexer_score_f64(const double* q, const double* kp, const double* w,
+                             const double* mask, double* score,
+                             int B, int T, int H, int P, int d)
+{
+    if (B <= 0 || T <= 0 || H <= 0 || P <= 0 || d <= 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < (long)B * T; ++bt) {
+        const long b = bt / T, t = bt % T;
+        for (long p = 0; p < P; ++p) {
+            const double* key = kp + (b * P + p) * d;
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h) {
+                const double* qh = q + ((b * T + t) * H + h) * d;
+                double dotp = 0.0;
+                for (int c = 0; c < d; ++c) dotp += qh[c] * key[c];
+                const double relu = dotp > 0.0 ? dotp : 0.0;
+                acc += w[(b * T + t) * H + h] * relu;
+            }
+            if (mask) acc += mask[(b * T + t) * P + p];
+            score[(b * T + t) * P + p] = acc;
+        }
+    }
+    return 0;
+}
+
+/*
+ * Top-k selection over each score row (the prhub.com.cn report "PR #45743 完整报告",
+ * section "实现拆解": the decode-side indexer keeps only the order of the scores,
+ * which is why its kernel drops the softmax scale).  For each of R rows of P
+ * scores, idx receives the positions of the kk largest finite scores, largest
+ * first; equal scores go lowest position first (reading: the report fixes no
+ * order among ties); -inf and NaN entries are never chosen, and slots left over
+ * when a row has fewer than kk finite scores hold -1.  Layouts: score [R, P],
+ * idx [R, kk].
+ */
+int oracle_topk_f64(const double* score, int R, int P, int kk, int* idx)
+{
+    if (R <= 0 || P <= 0 || kk <= 0) return -1;
+    int err = 0;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < R; ++r) {
+        const double* srow = score + r * P;
+        char* taken = (char*)calloc((size_t)P, 1);
+        if (!taken) {
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        for (int s = 0; s < kk; ++s) {
+            long best = -1;
+            for (long j = 0; j < P; ++j) {
+                if (taken[j] || !(srow[j] > -INFINITY)) continue;  /* skips -inf and NaN */
+                if (best < 0 || srow[j] > srow[best]) best = j;
+            }
+            idx[r * kk + s] = (int)best;
+            if (best >= 0) taken[best] = 1;
+        }
+        free(taken);
+    }
+    return err;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -48,11 +48,25 @@ MUTANTS = {
     "bwd_dq_unscaled": [("dqi[t] += scale * ds * krow[t];", "dqi[t] += ds * krow[t];")],
     "bwd_dk_uses_key": [("dkj[t] += scale * ds * qi[t];", "dkj[t] += scale * ds * krow[t];")],
     "bwd_dv_transposed": [("dvj[t] += pij * doi[t];", "dvj[t] += pij * vj[t];")],
+    # the lightning-indexer score and top-k
+    "indexer_relu_dropped": [("const double relu = dotp > 0.0 ? dotp : 0.0;", "const double relu = dotp;")],
+    "indexer_relu_after_sum": [("const double relu = dotp > 0.0 ? dotp : 0.0;", "const double relu = dotp;"),
+                               ("if (mask) acc += mask[(b * T + t) * P + p];",
+                                "if (acc < 0.0) acc = 0.0;\n            if (mask) acc += mask[(b * T + t) * P + p];")],
+    "indexer_weight_transposed": [("acc += w[(b * T + t) * H + h] * relu;",
+                                   "acc += w[(b * H + h) * T + t] * relu;")],
+    "indexer_mask_dropped": [("if (mask) acc += mask[(b * T + t) * P + p];", "if (!mask) acc += 0.0;")],
+    "indexer_key_batch": [("const double* key = kp + (b * P + p) * d;", "const double* key = kp + p * d;")],
+    "topk_ties_last": [("if (best < 0 || srow[j] > srow[best]) best = j;",
+                        "if (best < 0 || srow[j] >= srow[best]) best = j;")],
+    "topk_keeps_neg_inf": [("if (taken[j] || !(srow[j] > -INFINITY)) continue;  /* skips -inf and NaN */",
+                            "if (taken[j]) continue;")],
 }
 
 PIN_FILES = [os.path.join(ROOT, "tests", "test_oracle.py"),
              os.path.join(ROOT, "tests", "test_oracle_relpos.py"),
-             os.path.join(ROOT, "tests", "test_oracle_bwd.py")]
+             os.path.join(ROOT, "tests", "test_oracle_bwd.py"),
+             os.path.join(ROOT, "tests", "test_oracle_indexer.py")]
 
 RUNNER = textwrap.dedent("""
     import sys
