@@ -16,6 +16,7 @@ attn_fwd_blocked(q, k, v, causal, scale, block_m=128, block_n=64) -> (o, lse)
 attn_probs(q, k, causal, scale)             -> p [B, H, Nq, Nk]
 attn_fwd_relpos(q, k, v, emb, dist, causal, scale) -> (o, lse)   relative-position term
 attn_bwd(q, k, v, dout, causal, scale)      -> (dq, dk, dv)
+attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, causal, scale) -> (o, lse)
 indexer_score(q, kp, w, mask)               -> score [B, T, P]   lightning indexer
 topk(score, k)                              -> idx [..., k]
 num_threads() / set_num_threads(n)
@@ -55,6 +56,8 @@ def load(path=None):
     lib.oracle_attn_fwd_relpos_f64.restype = i
     lib.oracle_attn_fwd_relpos_f64.argtypes = [dp, dp, dp, dp, ip, dp, dp, i, i, i, i, i, i, i, d]
     lib.oracle_attn_probs_f64.restype = i
+    lib.oracle_attn_fwd_paged_f64.argtypes = [dp, dp, dp, ip, ip, dp, dp, i, i, i, i, i, i, i, i, d]
+    lib.oracle_attn_fwd_paged_f64.restype = i
     lib.oracle_indexer_score_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i]
     lib.oracle_indexer_score_f64.restype = i
     lib.oracle_topk_f64.argtypes = [dp, i, i, i, ip]
@@ -166,6 +169,38 @@ def attn_bwd(q, k, v, dout, causal=False, scale=None, lib=None):
     return dq, dk, dv
 
 
+def _i32(x):
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, causal=False, scale=None, lib=None):
+    """Attention of q [B, Lq, H, d] over a paged cache (k_cache, v_cache [num_blocks, page_size,
+    H, d], block_table int [B, max_blocks], seq_lens int [B]); the Lq queries of a request are
+    the last Lq positions of its sequence.  Returns (o [B, Lq, H, d], lse [B, H, Lq])."""
+    q, k_cache, v_cache = _f64(q), _f64(k_cache), _f64(v_cache)
+    block_table, seq_lens = _i32(block_table), _i32(seq_lens)
+    if q.ndim != 4 or k_cache.ndim != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [B, Lq, H, d] and k_cache, v_cache [num_blocks, page_size, H, d]")
+    B, Lq, H, d = q.shape
+    num_blocks, page_size = k_cache.shape[:2]
+    if k_cache.shape[2:] != (H, d) or block_table.ndim != 2 or block_table.shape[0] != B \
+            or seq_lens.shape != (B,):
+        raise ValueError("k_cache [num_blocks, page_size, H, d], block_table [B, max_blocks], seq_lens [B]")
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    o = np.zeros((B, Lq, H, d), dtype=np.float64)
+    lse = np.zeros((B, H, Lq), dtype=np.float64)
+    ip = ctypes.POINTER(ctypes.c_int)
+    rc = (lib or load()).oracle_attn_fwd_paged_f64(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), block_table.ctypes.data_as(ip),
+        seq_lens.ctypes.data_as(ip), _ptr(o), _ptr(lse), B, Lq, H, d, num_blocks, page_size,
+        block_table.shape[1], int(bool(causal)), scale)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_paged_f64 failed ({rc})")
+    return o, lse
+
+
 def indexer_score(q, kp, w, mask=None, lib=None):
     """Lightning-indexer score [B, T, P] = sum_h w[b,t,h] * relu(q[b,t,h] . kp[b,p]) + mask
     (q [B, T, H, d], kp [B, P, d], w [B, T, H], mask [B, T, P] or None)."""
@@ -213,4 +248,4 @@ def set_num_threads(n):
 
 
 __all__ = ["attn_fwd", "attn_fwd_blocked", "attn_probs", "attn_fwd_relpos", "attn_bwd",
-           "indexer_score", "topk", "num_threads", "set_num_threads", "load"]
+           "attn_fwd_paged", "indexer_score", "topk", "num_threads", "set_num_threads", "load"]

@@ -399,6 +399,94 @@ int oracle_attn_bwd_f64(const double* q, const double* k, const double* v, const
 }
 
 /*
+ * Attention over a paged key/value cache, for one or more query tokens per
+ * request (the vLLM page "PR #45743 完整报告": decode metadata of per-request
+ * seq_lens and a block table, section "关键源码片段", and several query tokens of
+ * one request scored together, section "功能与动机").  Request b owns the first
+ * L = seq_lens[b] rows of its logical sequence; logical row j sits in row
+ * j mod page_size of cache page block_table[b][j / page_size].  Its Lq query
+ * tokens are the last Lq positions of the sequence, so under the causal flag
+ * query i sees logical rows j <= i + L - Lq (the bottom-right alignment of the
+ * dense definition); without it every query sees all L rows.  Scores, softmax,
+ * output and lse are then those of oracle_attn_fwd_f64 on the gathered rows.
+ * Layouts: q, o [B, Lq, H, d]; k_cache, v_cache [num_blocks, page_size, H, d];
+ * block_table [B, max_blocks] int; seq_lens [B] int; lse [B, H, Lq].
+ * Returns -3 when a seq_len exceeds max_blocks * page_size or a table entry a
+ * row below it needs lies outside [0, num_blocks).
+ */
+int oracle_attn_fwd_paged_f64(const double* q, const double* k_cache, const double* v_cache,
+                              const int* block_table, const int* seq_lens, double* o,
+                              double* lse, int B, int Lq, int H, int d, int num_blocks,
+                              int page_size, int max_blocks, int causal, double scale)
+{
+    if (B <= 0 || Lq <= 0 || H <= 0 || d <= 0 || num_blocks <= 0 || page_size <= 0 ||
+        max_blocks <= 0)
+        return -1;
+    for (int b = 0; b < B; ++b) {
+        const long L = seq_lens[b];
+        if (L < 0 || L > (long)max_blocks * page_size) return -3;
+        for (long pg = 0; pg * page_size < L; ++pg) {
+            const int e = block_table[(long)b * max_blocks + pg];
+            if (e < 0 || e >= num_blocks) return -3;
+        }
+    }
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        const long L = seq_lens[b];
+        double* w = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        if (!w) {
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        for (long i = 0; i < Lq; ++i) {
+            const double* qrow = q + (((long)b * Lq + i) * H + h) * d;
+            double* orow = o + (((long)b * Lq + i) * H + h) * d;
+            double top = -INFINITY;
+            for (long j = 0; j < L; ++j) {
+                if (causal && j > i + (L - Lq)) {
+                    w[j] = -INFINITY;
+                    continue;
+                }
+                const long page = block_table[(long)b * max_blocks + j / page_size];
+                const long slot = page * page_size + j % page_size;
+                const double* krow = k_cache + (slot * H + h) * d;
+                double dotp = 0.0;
+                for (int t = 0; t < d; ++t) dotp += qrow[t] * krow[t];
+                w[j] = scale * dotp;
+                top = w[j] > top ? w[j] : top;
+            }
+            double* lse_bhi = lse + ((long)b * H + h) * Lq + i;
+            if (top == -INFINITY) {
+                for (int t = 0; t < d; ++t) orow[t] = 0.0;
+                *lse_bhi = -INFINITY;
+                continue;
+            }
+            double total = 0.0;
+            for (long j = 0; j < L; ++j) {
+                w[j] = (w[j] == -INFINITY) ? 0.0 : exp(w[j] - top);
+                total += w[j];
+            }
+            for (int t = 0; t < d; ++t) {
+                double sum_wv = 0.0;
+                for (long j = 0; j < L; ++j) {
+                    if (w[j] == 0.0) continue;
+                    const long page = block_table[(long)b * max_blocks + j / page_size];
+                    const long slot = page * page_size + j % page_size;
+                    sum_wv += w[j] * v_cache[(slot * H + h) * d + t];
+                }
+                orow[t] = sum_wv / total;
+            }
+            *lse_bhi = top + log(total);
+        }
+        free(w);
+    }
+    return err;
+}
+
+/*
  * Lightning-indexer score (the aispot.cmou.io report "llama.cpp 最佳化 lightning
  * indexer 視訊記憶體與多後端支援", release b11372, entry "compute the indexer score
  * with the lightning indexer"): every query token scores every pooled key by the

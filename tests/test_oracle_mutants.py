@@ -5,6 +5,7 @@ wrong sign, corner or index, a missing normalisation), compiled into a
 throw-away library.  The pin suite (test_oracle.py) is then run against it in a
 subprocess and must fail.  The committed oracle itself is never modified.
 """
+import concurrent.futures
 import os
 import subprocess
 import sys
@@ -48,6 +49,15 @@ MUTANTS = {
     "bwd_dq_unscaled": [("dqi[t] += scale * ds * krow[t];", "dqi[t] += ds * krow[t];")],
     "bwd_dk_uses_key": [("dkj[t] += scale * ds * qi[t];", "dkj[t] += scale * ds * krow[t];")],
     "bwd_dv_transposed": [("dvj[t] += pij * doi[t];", "dvj[t] += pij * vj[t];")],
+    # the paged-cache, multi-query oracle
+    "paged_top_left": [("if (causal && j > i + (L - Lq)) {", "if (causal && j > i) {")],
+    "paged_row_in_page_dropped": [("const long slot = page * page_size + j % page_size;\n                const double* krow",
+                                   "const long slot = page * page_size;\n                const double* krow")],
+    "paged_head_offset_dropped": [("const double* krow = k_cache + (slot * H + h) * d;",
+                                   "const double* krow = k_cache + (slot * H) * d;")],
+    "paged_values_from_keys": [("sum_wv += w[j] * v_cache[(slot * H + h) * d + t];",
+                                "sum_wv += w[j] * k_cache[(slot * H + h) * d + t];")],
+    "paged_lse_without_max": [("*lse_bhi = top + log(total);", "*lse_bhi = log(total);")],
     # the lightning-indexer score and top-k
     "indexer_relu_dropped": [("const double relu = dotp > 0.0 ? dotp : 0.0;", "const double relu = dotp;")],
     "indexer_relu_after_sum": [("const double relu = dotp > 0.0 ? dotp : 0.0;", "const double relu = dotp;"),
@@ -66,7 +76,12 @@ MUTANTS = {
 PIN_FILES = [os.path.join(ROOT, "tests", "test_oracle.py"),
              os.path.join(ROOT, "tests", "test_oracle_relpos.py"),
              os.path.join(ROOT, "tests", "test_oracle_bwd.py"),
-             os.path.join(ROOT, "tests", "test_oracle_indexer.py")]
+             os.path.join(ROOT, "tests", "test_oracle_indexer.py"),
+             os.path.join(ROOT, "tests", "test_oracle_paged.py")]
+
+PIN_FIRST = {"relpos": "test_oracle_relpos.py", "bwd": "test_oracle_bwd.py",
+             "indexer": "test_oracle_indexer.py", "topk": "test_oracle_indexer.py",
+             "paged": "test_oracle_paged.py"}
 
 RUNNER = textwrap.dedent("""
     import sys
@@ -80,25 +95,49 @@ RUNNER = textwrap.dedent("""
 """)
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
+def _run_pins(lib, tests, cwd):
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    code = RUNNER.format(root=ROOT, lib=lib, tests=tests)
+    return subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                          cwd=str(cwd), timeout=600, env=env)
+
+
+def _run_mutant(name, workdir):
+    """Build mutant `name` and run every pin file against it; returns (error, result)."""
     src = open(obuild.SRC).read()
     for old, new in MUTANTS[name]:
-        assert src.count(old) == 1, f"mutation anchor for {name} not unique/present"
+        if src.count(old) != 1:
+            return f"mutation anchor for {name} not unique/present", None
         src = src.replace(old, new)
-    mpath = tmp_path / f"{name}.c"
+    mpath = workdir / f"{name}.c"
     mpath.write_text(src)
-    lib = obuild.build(src=str(mpath), out=str(tmp_path / f"lib{name}.so"))
-    code = RUNNER.format(root=ROOT, lib=lib, tests=PIN_FILES)
-    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
-                         cwd=str(tmp_path), timeout=600)
+    lib = obuild.build(src=str(mpath), out=str(workdir / f"lib{name}.so"))
+    # the pin file written for the mutated function goes first, so that the run (which
+    # stops at the first failure) ends early
+    first = [f for f in PIN_FILES if os.path.basename(f) == PIN_FIRST.get(name.split("_")[0])]
+    return None, _run_pins(lib, first + [f for f in PIN_FILES if f not in first], workdir)
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """All mutants, built and run against the pins a few at a time (each run is a fresh
+    interpreter, so most of its time is start-up)."""
+    workdir = tmp_path_factory.mktemp("mutants")
+    workers = max(1, min(6, os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+        futures = {name: pool.submit(_run_mutant, name, workdir) for name in MUTANTS}
+        return {name: f.result() for name, f in futures.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_results):
+    err, res = mutant_results[name]
+    assert err is None, err
     assert res.returncode != 0, f"mutant {name} survived the pin suite:\n{res.stdout[-2000:]}"
 
 
 def test_unmutated_copy_passes(tmp_path):
     """Control: the same harness on an unmodified copy passes."""
     lib = obuild.build(src=obuild.SRC, out=str(tmp_path / "libcopy.so"))
-    code = RUNNER.format(root=ROOT, lib=lib, tests=PIN_FILES)
-    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
-                         cwd=str(tmp_path), timeout=600)
+    res = _run_pins(lib, PIN_FILES, tmp_path)
     assert res.returncode == 0, res.stdout[-3000:] + res.stderr[-2000:]
