@@ -100,6 +100,17 @@ def _check(q, k, v):
     return B, H, Nq, k.shape[1], d
 
 
+def _check_buffer(name, t, shape, dtype, device):
+    """A caller-supplied result buffer must be exactly what the library writes: it fills
+    the whole of it, so a smaller or strided tensor, or one on another device, would be
+    written out of bounds."""
+    import torch
+    if not isinstance(t, torch.Tensor) or t.device != device:
+        raise ValueError(f"{name} must be a tensor on {device}")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
 def _stream_ptr(stream, device):
     import torch
     if stream is None:
@@ -123,11 +134,9 @@ def attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_lse=T
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
-        raise ValueError("out must be a contiguous tensor like q")
-    if lse is not None and (lse.shape != (B, H, Nq) or lse.dtype != torch.float32
-                            or not lse.is_contiguous()):
-        raise ValueError("lse must be a contiguous float32 [B, H, Nq] tensor")
+    _check_buffer("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_buffer("lse", lse, (B, H, Nq), torch.float32, q.device)
     dt = _dtype_code(q.dtype)
     lse_ptr = ctypes.c_void_p(lse.data_ptr() if lse is not None else 0)
     with torch.cuda.device(q.device):
@@ -158,13 +167,15 @@ def attn_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None
     """
     import torch
     lib = load_library()
-    B, one, H, d = q.shape
-    if one != 1:
-        raise ValueError("q must be [batch, 1, heads, head_dim]")
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
                     ("block_table", block_table), ("seq_lens", seq_lens)):
         if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
             raise TypeError(f"{name} must be a contiguous CUDA tensor")
+        if t.device != q.device:
+            raise ValueError(f"{name} must be on q's device {q.device}")
+    if q.dim() != 4 or q.shape[1] != 1:
+        raise ValueError("q must be [batch, 1, heads, head_dim]")
+    B, _, H, d = q.shape
     if not (q.dtype == k_cache.dtype == v_cache.dtype):
         raise TypeError("q, k_cache, v_cache must share one dtype")
     if k_cache.shape != v_cache.shape or k_cache.dim() != 4 or k_cache.shape[2:] != (H, d):
@@ -179,6 +190,9 @@ def attn_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_buffer("lse", lse, (B, H), torch.float32, q.device)
     with torch.cuda.device(q.device):
         rc = lib.attn_fwd_decode_paged(
             ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k_cache.data_ptr()),

@@ -152,3 +152,32 @@ def test_package_import_is_lazy_and_loud_without_library(tmp_path):
             _binding.load_library(str(tmp_path / "missing.so"))
     finally:
         _binding._lib = saved
+
+
+def test_result_buffers_are_checked_before_the_call():
+    """A caller's out/lse buffer must match exactly: the library writes all of it."""
+    import torch
+    from attention_forward_tiled_b200._binding import _check_buffer
+    cpu = torch.device("cpu")
+    ok = torch.empty(2, 3, 4, dtype=torch.float16)
+    _check_buffer("out", ok, (2, 3, 4), torch.float16, cpu)
+    bad = [
+        torch.empty(2, 3, 3, dtype=torch.float16),                 # too small
+        torch.empty(2, 3, 4, dtype=torch.float32),                 # wrong dtype
+        torch.empty(2, 4, 3, dtype=torch.float16).transpose(1, 2),  # strided
+        torch.empty(2, 3, 4, dtype=torch.float16, device="meta"),  # another device
+        ok.numpy(),                                                # not a tensor
+    ]
+    for t in bad:
+        with pytest.raises(ValueError):
+            _check_buffer("out", t, (2, 3, 4), torch.float16, cpu)
+
+
+def test_paged_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 2, 64, dtype=torch.float16)
+    kc = torch.zeros(4, 16, 2, 64, dtype=torch.float16)
+    bt = torch.zeros(1, 4, dtype=torch.int32)
+    sl = torch.ones(1, dtype=torch.int32)
+    with pytest.raises(TypeError):
+        attn.attn_fwd_decode_paged(q, kc, kc, bt, sl)
