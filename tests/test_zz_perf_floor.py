@@ -1,0 +1,78 @@
+"""Throughput floors on the GPU: no large performance regression.
+
+Each timed workload must reach at least half of the throughput recorded for it
+on a B200 (CUDA events over 20 back-to-back calls after 3 warm-up calls, inputs
+resident on the device).  The floor is loose on purpose: it does not replace
+the benchmark, whose numbers are the measured ones, but a kernel that lost its
+pipelining, its overlap or its load balance falls far below it.  These are not
+parity tests; the parity files cover the results.
+"""
+import pytest
+import torch
+
+import attention_forward_tiled_b200 as attn
+from attention_forward_tiled_b200.inputs import (PAGED_WORKLOADS, WORKLOADS, flops, kv_bytes,
+                                                 make_inputs, make_paged_inputs)
+
+pytestmark = pytest.mark.gpu
+
+# throughput recorded on a B200 at 1965 MHz (the benchmark's workloads and metric)
+RECORDED = {
+    "causal4k": (1050.0, "TFLOP/s"),
+    "causal8k": (1128.0, "TFLOP/s"),
+    "bf16_k3": (447.0, "TFLOP/s"),
+    "decode": (6405.0, "GB/s"),
+    "decode_paged16": (5669.0, "GB/s"),
+}
+FLOOR = 0.5
+
+
+def seconds_per_call(fn, iters=20, warmup=3):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(iters):
+        fn()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) * 1e-3 / iters
+
+
+def check_floor(name, value):
+    recorded, unit = RECORDED[name]
+    assert value >= FLOOR * recorded, (
+        f"{name}: {value:.1f} {unit} is below {FLOOR:.0%} of the recorded {recorded:.0f} {unit}")
+
+
+@pytest.mark.parametrize("name", ["causal4k", "causal8k", "bf16_k3", "decode"])
+def test_dense_workload_floor(name):
+    w = WORKLOADS[name]
+    q, k, v = (t.cuda() for t in make_inputs(**w))
+    out = torch.empty_like(q)
+    lse = torch.empty((w["B"], w["H"], w["Nq"]), dtype=torch.float32, device=q.device)
+    sec = seconds_per_call(lambda: attn.attn_fwd(q, k, v, causal=w["causal"], scale=w["scale"],
+                                                 out=out, lse=lse))
+    assert attn.get_status() == 0
+    if RECORDED[name][1] == "TFLOP/s":
+        value = flops(**w) / sec / 1e12
+    else:
+        value = kv_bytes(**w) / sec / 1e9
+    check_floor(name, value)
+
+
+def test_paged_decode_floor():
+    name = "decode_paged16"
+    w = PAGED_WORKLOADS[name]
+    q, kc, vc, bt, sl = (t.cuda() for t in make_paged_inputs(
+        w["B"], w["H"], w["d"], w["seq_lens"], w["page_size"], dtype=w["dtype"], seed=w["seed"]))
+    out = torch.empty_like(q)
+    lse = torch.empty((w["B"], w["H"]), dtype=torch.float32, device=q.device)
+    sec = seconds_per_call(lambda: attn.attn_fwd_decode_paged(q, kc, vc, bt, sl, scale=w["scale"],
+                                                              out=out, lse=lse))
+    assert attn.get_status() == 0
+    value = kv_bytes(B=w["B"], H=w["H"], Nk=sum(w["seq_lens"]) // w["B"], d=w["d"],
+                     dtype=w["dtype"]) / sec / 1e9
+    check_floor(name, value)
