@@ -13,6 +13,7 @@ Functions
 ---------
 attn_fwd(q, k, v, causal, scale)            -> (o, lse)   definition order
 attn_fwd_blocked(q, k, v, causal, scale, block_m=128, block_n=64) -> (o, lse)
+attn_fwd_splitkv(q, k, v, splits, causal, scale) -> (o, lse)   split-KV + combine order
 attn_probs(q, k, causal, scale)             -> p [B, H, Nq, Nk]
 attn_fwd_relpos(q, k, v, emb, dist, causal, scale) -> (o, lse)   relative-position term
 attn_bwd(q, k, v, dout, causal, scale)      -> (dq, dk, dv)
@@ -56,6 +57,8 @@ def load(path=None):
     lib.oracle_attn_fwd_relpos_f64.restype = i
     lib.oracle_attn_fwd_relpos_f64.argtypes = [dp, dp, dp, dp, ip, dp, dp, i, i, i, i, i, i, i, d]
     lib.oracle_attn_probs_f64.restype = i
+    lib.oracle_attn_fwd_splitkv_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i]
+    lib.oracle_attn_fwd_splitkv_f64.restype = i
     lib.oracle_attn_fwd_paged_f64.argtypes = [dp, dp, dp, ip, ip, dp, dp, i, i, i, i, i, i, i, i, d]
     lib.oracle_attn_fwd_paged_f64.restype = i
     lib.oracle_indexer_score_f64.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i]
@@ -117,6 +120,22 @@ def attn_fwd_blocked(q, k, v, causal=False, scale=None, block_m=128, block_n=64,
                                                      int(block_m), int(block_n))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd_blocked_f64 failed ({rc})")
+    return o, lse
+
+
+def attn_fwd_splitkv(q, k, v, splits, causal=False, scale=None, lib=None):
+    """The decode path's ordering: keys cut into `splits` ranges, per-range (m, l, o)
+    states, then the combine step.  Same result as attn_fwd up to rounding."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, Nk, d = _shapes(q, k, v)
+    scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+    o = np.zeros((B, Nq, H, d), dtype=np.float64)
+    lse = np.zeros((B, H, Nq), dtype=np.float64)
+    rc = (lib or load()).oracle_attn_fwd_splitkv_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                                     B, H, Nq, Nk, d, int(bool(causal)), scale,
+                                                     int(splits))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_splitkv_f64 failed ({rc})")
     return o, lse
 
 
@@ -247,5 +266,5 @@ def set_num_threads(n):
     load().oracle_set_num_threads(int(n))
 
 
-__all__ = ["attn_fwd", "attn_fwd_blocked", "attn_probs", "attn_fwd_relpos", "attn_bwd",
-           "attn_fwd_paged", "indexer_score", "topk", "num_threads", "set_num_threads", "load"]
+__all__ = ["attn_fwd", "attn_fwd_blocked", "attn_fwd_splitkv", "attn_probs", "attn_fwd_relpos",
+           "attn_bwd", "attn_fwd_paged", "indexer_score", "topk", "num_threads", "set_num_threads", "load"]

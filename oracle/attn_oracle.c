@@ -231,6 +231,87 @@ int oracle_attn_fwd_blocked_f64(const double* q, const double* k, const double* 
 }
 
 /*
+ * The split-KV ordering of the decode path: the keys of each query row are cut
+ * into `splits` contiguous ranges of ceil(Nk / splits) keys (the last range holds
+ * the rest), each range keeps its own state
+ *   m_s = max_j s_ij,   l_s = sum_j exp(s_ij - m_s),   o_s = sum_j exp(s_ij - m_s) v_j
+ * and a combine step merges them:
+ *   M = max_s m_s,   L = sum_s l_s exp(m_s - M),   O = sum_s o_s exp(m_s - M) / L,
+ *   lse = M + ln L.
+ * This is the same recurrence as the blocked ordering (the ai6s.net article's
+ * online softmax, section "FlashAttention的核心逻辑"), applied to ranges that are
+ * processed side by side instead of one after another.  A range with no allowed key
+ * (m_s = -inf) drops out.  Must agree with oracle_attn_fwd_f64 to rounding.
+ */
+int oracle_attn_fwd_splitkv_f64(const double* q, const double* k, const double* v,
+                                double* o, double* lse,
+                                int B, int H, int Nq, int Nk, int d, int causal, double scale,
+                                int splits)
+{
+    if (check_args(B, H, Nq, Nk, d) || splits <= 0) return -1;
+    const long span = ((long)Nk + splits - 1) / splits;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        double* part_m = (double*)malloc(sizeof(double) * (size_t)splits);
+        double* part_l = (double*)malloc(sizeof(double) * (size_t)splits);
+        double* part_o = (double*)malloc(sizeof(double) * (size_t)splits * (size_t)d);
+        if (!part_m || !part_l || !part_o) {
+#pragma omp atomic write
+            err = -2;
+            free(part_m); free(part_l); free(part_o);
+            continue;
+        }
+        for (long i = 0; i < Nq; ++i) {
+            for (int sp = 0; sp < splits; ++sp) {
+                const long j_lo = (long)sp * span;
+                const long j_hi = (j_lo + span < Nk) ? j_lo + span : Nk;
+                double ms = -INFINITY;
+                for (long j = j_lo; j < j_hi; ++j) {
+                    if (!is_allowed(i, j, Nq, Nk, causal)) continue;
+                    const double sc = scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d);
+                    ms = sc > ms ? sc : ms;
+                }
+                part_m[sp] = ms;
+                part_l[sp] = 0.0;
+                for (int t = 0; t < d; ++t) part_o[(long)sp * d + t] = 0.0;
+                if (ms == -INFINITY) continue;
+                for (long j = j_lo; j < j_hi; ++j) {
+                    if (!is_allowed(i, j, Nq, Nk, causal)) continue;
+                    const double e = exp(scale * dot_qk(q, k, b, h, i, j, H, Nq, Nk, d) - ms);
+                    part_l[sp] += e;
+                    const double* vrow = v + IDX4(b, j, h, 0, Nk, H, d);
+                    for (int t = 0; t < d; ++t) part_o[(long)sp * d + t] += e * vrow[t];
+                }
+            }
+            /* combine */
+            double big_m = -INFINITY;
+            for (int sp = 0; sp < splits; ++sp) big_m = part_m[sp] > big_m ? part_m[sp] : big_m;
+            double* orow = o + IDX4(b, i, h, 0, Nq, H, d);
+            double* lse_row = lse + ((long)b * H + h) * Nq + i;
+            if (big_m == -INFINITY) {
+                for (int t = 0; t < d; ++t) orow[t] = 0.0;
+                *lse_row = -INFINITY;
+                continue;
+            }
+            double big_l = 0.0;
+            for (int sp = 0; sp < splits; ++sp)
+                if (part_m[sp] != -INFINITY) big_l += part_l[sp] * exp(part_m[sp] - big_m);
+            for (int t = 0; t < d; ++t) {
+                double num = 0.0;
+                for (int sp = 0; sp < splits; ++sp)
+                    if (part_m[sp] != -INFINITY) num += part_o[(long)sp * d + t] * exp(part_m[sp] - big_m);
+                orow[t] = num / big_l;
+            }
+            *lse_row = big_m + log(big_l);
+        }
+        free(part_m); free(part_l); free(part_o);
+    }
+    return err;
+}
+
+/*
  * Attention with a relative-position score term (the Granite-Speech conformer
  * attention of the vLLM page "PR #42933", section "关键源码片段": the term
  * einsum("bnhid,ijd->bnhij", q, rel_pos_emb) * scale is added to the scores that

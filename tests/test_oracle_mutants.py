@@ -49,6 +49,14 @@ MUTANTS = {
     "bwd_dq_unscaled": [("dqi[t] += scale * ds * krow[t];", "dqi[t] += ds * krow[t];")],
     "bwd_dk_uses_key": [("dkj[t] += scale * ds * qi[t];", "dkj[t] += scale * ds * krow[t];")],
     "bwd_dv_transposed": [("dvj[t] += pij * doi[t];", "dvj[t] += pij * vj[t];")],
+    # the split-KV (decode) ordering
+    "splitkv_l_not_rescaled": [("if (part_m[sp] != -INFINITY) big_l += part_l[sp] * exp(part_m[sp] - big_m);",
+                                "if (part_m[sp] != -INFINITY) big_l += part_l[sp];")],
+    "splitkv_o_not_rescaled": [("num += part_o[(long)sp * d + t] * exp(part_m[sp] - big_m);",
+                                "num += part_o[(long)sp * d + t];")],
+    "splitkv_lse_without_max": [("*lse_row = big_m + log(big_l);", "*lse_row = log(big_l);")],
+    "splitkv_range_end_short": [("const long j_hi = (j_lo + span < Nk) ? j_lo + span : Nk;",
+                                 "const long j_hi = (j_lo + span < Nk) ? j_lo + span - 1 : Nk;")],
     # the paged-cache, multi-query oracle
     "paged_top_left": [("if (causal && j > i + (L - Lq)) {", "if (causal && j > i) {")],
     "paged_row_in_page_dropped": [("const long slot = page * page_size + j % page_size;\n                const double* krow",
@@ -77,11 +85,12 @@ PIN_FILES = [os.path.join(ROOT, "tests", "test_oracle.py"),
              os.path.join(ROOT, "tests", "test_oracle_relpos.py"),
              os.path.join(ROOT, "tests", "test_oracle_bwd.py"),
              os.path.join(ROOT, "tests", "test_oracle_indexer.py"),
-             os.path.join(ROOT, "tests", "test_oracle_paged.py")]
+             os.path.join(ROOT, "tests", "test_oracle_paged.py"),
+             os.path.join(ROOT, "tests", "test_oracle_splitkv.py")]
 
 PIN_FIRST = {"relpos": "test_oracle_relpos.py", "bwd": "test_oracle_bwd.py",
              "indexer": "test_oracle_indexer.py", "topk": "test_oracle_indexer.py",
-             "paged": "test_oracle_paged.py"}
+             "paged": "test_oracle_paged.py", "splitkv": "test_oracle_splitkv.py"}
 
 RUNNER = textwrap.dedent("""
     import sys
