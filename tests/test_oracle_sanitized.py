@@ -17,7 +17,8 @@ from oracle import build as obuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["test_oracle.py", "test_oracle_relpos.py", "test_oracle_bwd.py",
-             "test_oracle_indexer.py", "test_oracle_paged.py", "test_oracle_splitkv.py"]
+             "test_oracle_indexer.py", "test_oracle_paged.py", "test_oracle_splitkv.py",
+             "test_oracle_properties.py"]
 
 # -s: the inner pytest leaves stderr alone, so a sanitizer report reaches the caller
 RUNNER = textwrap.dedent("""
