@@ -22,7 +22,6 @@ import argparse
 import hashlib
 import re
 import json
-import math
 import os
 import statistics
 import sys

@@ -25,7 +25,6 @@ num_threads() / set_num_threads(n)
 Layouts: q, o [B, Nq, H, d]; k, v [B, Nk, H, d]; lse [B, H, Nq].
 """
 import ctypes
-import os
 
 import numpy as np
 

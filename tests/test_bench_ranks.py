@@ -7,7 +7,6 @@ ranks of the elapsed time; the reference arm runs on rank 0 only.
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 

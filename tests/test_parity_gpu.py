@@ -7,7 +7,6 @@ pin) plus properties checked on every output element.
 """
 import math
 
-import numpy as np
 import pytest
 import torch
 
