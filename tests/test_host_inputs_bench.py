@@ -82,3 +82,39 @@ def test_committed_traffic_needs_a_matching_hash(tmp_path, monkeypatch):
     assert bench.committed_traffic("causal4k") == 123.0
     assert bench.committed_traffic("bf16_k3") is None
     assert bench.committed_traffic("decode") is None
+
+
+def test_clock_sampler_against_a_fake_nvml(monkeypatch):
+    """The bench's clock record (median SM clock under load and every clock-event reason
+    seen), read from a fake NVML: the sampler only reads, it sets nothing."""
+    import sys
+    import types
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlClocksEventReasonSwPowerCap=0x4, nvmlClocksEventReasonHwSlowdown=0x8,
+        nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonGpuIdle=0x1)
+    clocks = iter([1965, 1800, 1965, 1950, 1965])
+    reasons = iter([0x0, 0x4, 0x4, 0x0, 0x4 | 0x8])
+    calls = []
+    fake.nvmlInit = lambda: calls.append("init")
+    fake.nvmlDeviceGetHandleByIndex = lambda i: ("handle", i)
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    fake.nvmlDeviceGetClockInfo = lambda h, kind: next(clocks)
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: next(reasons)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0)
+    for _ in range(5):
+        s.sample_once()
+    summ = s.summary()
+    assert summ["sm_mhz"] == 1965 and summ["sm_max_mhz"] == 1965 and summ["samples"] == 5
+    assert summ["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert calls == ["init"]
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    import sys
+    monkeypatch.setitem(sys.modules, "pynvml", None)   # import fails
+    s = bench.ClockSampler(0)
+    s.start()
+    s.stop()
+    summ = s.summary()
+    assert summ["sm_mhz"] is None and summ["samples"] == 0 and "error" in summ
