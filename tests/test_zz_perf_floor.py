@@ -2,8 +2,9 @@
 
 Each timed workload must reach at least half of the throughput recorded for it
 on a B200 (CUDA events over 20 back-to-back calls after 3 warm-up calls, inputs
-resident on the device).  The floor is loose on purpose: it does not replace
-the benchmark, whose numbers are the measured ones, but a kernel that lost its
+resident on the device, the calls enqueued behind a device-side spin as the
+benchmark does).  The floor is loose on purpose: it does not replace the
+benchmark, whose numbers are the measured ones, but a kernel that lost its
 pipelining, its overlap or its load balance falls far below it.  These are not
 parity tests; the parity files cover the results.
 """
@@ -33,6 +34,9 @@ def seconds_per_call(fn, iters=20, warmup=3):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    # a device-side spin ahead of the timed calls lets the host enqueue all of them, so short
+    # kernels are not paced by the Python launch path; the spin is outside the timed interval
+    torch.cuda._sleep(20_000_000)
     start.record()
     for _ in range(iters):
         fn()
