@@ -2,8 +2,9 @@
 
 Each mutant is the oracle's C source with one textual slip (a dropped term, a
 wrong sign, corner or index, a missing normalisation), compiled into a
-throw-away library.  The pin suite (test_oracle.py) is then run against it in a
-subprocess and must fail.  The committed oracle itself is never modified.
+throw-away library.  Every pin file of the oracle (PIN_FILES: the forward, the
+split-KV order, and the next-row oracles) is then run against it in a fresh
+interpreter and must fail.  The committed oracle itself is never modified.
 """
 import concurrent.futures
 import os
