@@ -31,13 +31,20 @@
  * Layouts: q, o are [B, Nq, H, d]; k, v are [B, Nk, H, d]; lse is [B, H, Nq];
  * p (probabilities, tiny cases only) is [B, H, Nq, Nk].  Everything is double.
  *
- * Two orderings are provided.  oracle_attn_fwd_f64 follows the definition
- * literally and materialises each (b, h) score matrix.  The blocked variant
- * follows the article's "FlashAttention的核心逻辑" section: an outer loop over
- * query blocks, an inner loop over key/value blocks, a running row maximum and
- * row sum updated block by block (the online softmax update, written out in
- * its standard form because the article only names it), and one
- * normalisation after the inner loop.  Both must agree to rounding.
+ * Three orderings of the forward are provided.  oracle_attn_fwd_f64 follows the
+ * definition literally and materialises each (b, h) score matrix.  The blocked
+ * variant follows the article's "FlashAttention的核心逻辑" section: an outer loop
+ * over query blocks, an inner loop over key/value blocks, a running row maximum
+ * and row sum updated block by block (the online softmax update, written out in
+ * its standard form because the article only names it), and one normalisation
+ * after the inner loop.  The split-KV variant keeps one state per key range and
+ * merges them at the end, the order of the decode path.  All must agree to
+ * rounding.
+ *
+ * Further down, for the steps next to this one on the pages: the score term of
+ * a relative-position embedding, the backward pass, attention over a paged
+ * key/value cache with several query tokens per request, and the lightning
+ * indexer's rectified head-weighted score with its top-k selection.
  */
 #include <math.h>
 #include <stdlib.h>
