@@ -412,9 +412,11 @@ int oracle_attn_bwd_f64(const double* q, const double* k, const double* v, const
                         int B, int H, int Nq, int Nk, int d, int causal, double scale)
 {
     if (check_args(B, H, Nq, Nk, d)) return -1;
-    memset(dq, 0, sizeof(double) * (size_t)B * Nq * H * d);
-    memset(dk, 0, sizeof(double) * (size_t)B * Nk * H * d);
-    memset(dv, 0, sizeof(double) * (size_t)B * Nk * H * d);
+    const size_t n_q = (size_t)B * (size_t)Nq * (size_t)H * (size_t)d;
+    const size_t n_kv = (size_t)B * (size_t)Nk * (size_t)H * (size_t)d;
+    memset(dq, 0, sizeof(double) * n_q);
+    memset(dk, 0, sizeof(double) * n_kv);
+    memset(dv, 0, sizeof(double) * n_kv);
     int err = 0;
 #pragma omp parallel for schedule(dynamic, 1)
     for (long bh = 0; bh < (long)B * H; ++bh) {
