@@ -6,7 +6,7 @@
 The library is loaded on first use; a missing build raises instead of falling
 back to anything else.  ``inputs`` holds the seeded synthetic workloads.
 """
-from ._binding import (ATTN_BF16, ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_TIMEOUT,
+from ._binding import (ATTN_BF16, ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_RANGE, ATTN_ERR_TIMEOUT,
                        ATTN_ERR_UNSUPPORTED, ATTN_F16, ATTN_OK, LIB_PATH, SIGNATURES, AttnError,
                        HostRunner, attn_fwd, attn_fwd_decode_paged, debug_set, error_string,
                        get_status, load_library, version)
@@ -14,5 +14,5 @@ from ._binding import (ATTN_BF16, ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_
 __all__ = [
     "attn_fwd", "attn_fwd_decode_paged", "get_status", "error_string", "version", "debug_set", "load_library",
     "HostRunner", "AttnError", "LIB_PATH", "SIGNATURES", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
-    "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_F16", "ATTN_BF16",
+    "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_RANGE", "ATTN_F16", "ATTN_BF16",
 ]

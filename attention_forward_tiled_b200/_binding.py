@@ -18,6 +18,7 @@ ATTN_ERR_INVALID_ARG = -1
 ATTN_ERR_UNSUPPORTED = -2
 ATTN_ERR_CUDA = -3
 ATTN_ERR_TIMEOUT = -4
+ATTN_ERR_RANGE = -5
 
 # every entry point declared in include/attn.h: name -> (restype, argtypes)
 _vp, _i, _f, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong

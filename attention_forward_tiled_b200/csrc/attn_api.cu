@@ -21,7 +21,7 @@
 
 using namespace attn_b200;
 
-// Device status word: kernels record ATTN_ERR_TIMEOUT here instead of trapping.
+// Device status word: kernels record ATTN_ERR_TIMEOUT / ATTN_ERR_RANGE here instead of trapping.
 __device__ int g_attn_status = 0;
 
 // Fixed scratch of attn_fwd_decode_noalloc: the split partials live here instead of in
@@ -38,10 +38,8 @@ constexpr int kMaxDevices = 64;
 // Prefill scheduling group: units of 16 heads are handed out together (heaviest causal
 // units first), so the K/V being read stay in L2 (16 heads x 4096 keys x d 128 x 2 x 2 B
 // = 32 MB) while the group is long enough to even out the causal unit sizes over SMs.
-#ifndef ATTN_HEADS_PER_GROUP
-#define ATTN_HEADS_PER_GROUP 16
-#endif
-constexpr int kHeadsPerGroup = ATTN_HEADS_PER_GROUP;
+// (12 or 24 heads per group measured slower or equal on the causal workloads.)
+constexpr int kHeadsPerGroup = 16;
 
 std::atomic<int> g_inject{0};
 std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
@@ -225,11 +223,12 @@ int launch_prefill(DeviceState* ds, const void* q, const void* k, const void* v,
 }
 
 // Split count for the decode kernel: minimise the largest per-CTA tile count
-// (items are dealt round-robin to one persistent CTA per SM), preferring fewer splits.
-int choose_splits(long long BH, int ntiles, int grid) {
+// (items are dealt round-robin to one persistent CTA per SM), preferring fewer splits;
+// at most max_splits.
+int choose_splits(long long BH, int ntiles, int grid, long long max_splits = 1LL << 30) {
   int best = 1;
   long long best_load = -1;
-  for (int s = 1; s <= ntiles; ++s) {
+  for (int s = 1; s <= ntiles && s <= max_splits; ++s) {
     const int tps = (ntiles + s - 1) / s;
     const int s_eff = (ntiles + tps - 1) / tps;
     if (s_eff != s) continue;
@@ -397,7 +396,10 @@ int launch_decode_noalloc(DeviceState* ds, const void* q, const void* k, const v
   const int slot = 4 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
   const int ntiles = (Nk + 127) / 128;
   const long long BH = (long long)B * H;
-  int splits = splits_req > 0 ? splits_req : choose_splits(BH, ntiles, ds->sm_count);
+  // automatic choice: only split counts whose partials fit the fixed array
+  const long long fit = (long long)(kNoAllocScratchFloats / ((size_t)BH * (D + 2)));
+  if (splits_req == 0 && fit < 1) return ATTN_ERR_INVALID_ARG;
+  int splits = splits_req > 0 ? splits_req : choose_splits(BH, ntiles, ds->sm_count, fit);
   if (splits < 1 || splits > ntiles) return ATTN_ERR_INVALID_ARG;
   const int tps = (ntiles + splits - 1) / splits;
   splits = (ntiles + tps - 1) / tps;
@@ -554,23 +556,15 @@ const char* attn_error_string(int status) {
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA runtime or driver call failed";
     case ATTN_ERR_TIMEOUT:
       return "ATTN_ERR_TIMEOUT: a bounded device-side pipeline wait expired; outputs undefined";
+    case ATTN_ERR_RANGE:
+      return "ATTN_ERR_RANGE: a bf16 V value of magnitude >= 65536 (or inf/NaN) has no fp16 value; "
+             "outputs undefined";
     default: return "unknown attn status code";
   }
 }
 
 int attn_version(void) { return kVersion; }
 
-#ifdef ATTN_TRACE
-// Timeline read-back of the instrumented build (not part of the regular library).
-ATTN_API int attn_trace_read(void* dst, unsigned long long bytes) {
-  if (bytes > sizeof(g_prefill_trace)) bytes = sizeof(g_prefill_trace);
-  return cudaMemcpyFromSymbol(dst, g_prefill_trace, bytes) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-ATTN_API int attn_trace_spans(void* dst, unsigned long long bytes) {
-  if (bytes > sizeof(g_cta_span)) bytes = sizeof(g_cta_span);
-  return cudaMemcpyFromSymbol(dst, g_cta_span, bytes) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-#endif
 
 int attn_debug_set(int inject, unsigned long long wait_timeout_ns) {
   g_inject.store(inject);

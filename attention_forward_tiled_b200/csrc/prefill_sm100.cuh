@@ -80,11 +80,9 @@ struct PrefillCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row Q, K, V or O tile
   static constexpr int kStages = (D == 128) ? 4 : 8;    // K/V ring depth
-#ifdef ATTN_CLAIM_LEAD
-  static constexpr int kClaimLead = ATTN_CLAIM_LEAD;
-#else
-  static constexpr int kClaimLead = 2 * kStages;  // ring items before a unit's last load
-#endif
+  // The next unit is claimed this many ring items before the current unit's last load
+  // (measured: a lead of 4 or 16 items at d = 128 was slower or equal).
+  static constexpr int kClaimLead = 2 * kStages;
   static constexpr int kNumOStage = kDecoupled ? 2 : 1;  // O staging buffers
   static constexpr int kOffQ = 0;                                    // Q_0, Q_1
   static constexpr int kOffKV = 2 * kTileBytes;                      // K/V ring
@@ -193,28 +191,18 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
   return u;
 }
 
-// Every ATTN_EXP_EMU_PERIOD-th pair of softmax exponentials (d = 128;
-// ATTN_EXP_EMU_PERIOD_D64 at d = 64) is evaluated with the FMA-pipe polynomial instead
-// of the MUFU unit (0 = all on MUFU).  MUFU delivers 4 exp2 per clock per SM
-// sub-partition; the polynomial costs more issue slots per result, so the best share is
-// measured: every 8th pair at d = 128 (1 in 4 and 1 in 3 were slower), every 4th at d = 64.
-#ifndef ATTN_EXP_EMU_PERIOD
-#define ATTN_EXP_EMU_PERIOD 8
-#endif
-#ifndef ATTN_EXP_EMU_PERIOD_D64
-#define ATTN_EXP_EMU_PERIOD_D64 4
-#endif
+// Every kExpEmuPeriod-th pair of softmax exponentials (d = 128; kExpEmuPeriodD64 at
+// d = 64) is evaluated with the FMA-pipe polynomial instead of the MUFU unit.  MUFU
+// delivers 4 exp2 per clock per SM sub-partition; the polynomial costs more issue slots
+// per result, so the best share is measured: every 8th pair at d = 128 (1 in 4 and 1 in 3
+// were slower), every 4th at d = 64.
+constexpr int kExpEmuPeriod = 8;
+constexpr int kExpEmuPeriodD64 = 4;
 template <int kPeriod>
 __device__ __forceinline__ constexpr bool emu_pair(int pair) {
-  return kPeriod > 0 && (pair % (kPeriod > 0 ? kPeriod : 1)) == (kPeriod > 0 ? kPeriod - 1 : 0);
+  static_assert(kPeriod > 0, "emulation period");
+  return (pair % kPeriod) == kPeriod - 1;
 }
-
-// d = 128: unmasked tiles after the first are exponentiated against the running max in
-// the same pass that finds the tile max (P kept in registers, redone in the rare case a
-// score exceeds the running max by more than 8).
-#ifndef ATTN_SPECULATIVE
-#define ATTN_SPECULATIVE 1
-#endif
 
 // Max over one 64-column half of an S row (columns 64*kHalf + c), sign-flipped for a
 // negative scale, restricted to columns < lim when kMask; four 3-input max chains.
@@ -240,16 +228,21 @@ __device__ __forceinline__ float half_max(const uint32_t (&h)[2][32], int lim) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
+// Sum of the eight partial row sums of the softmax (four pairs of accumulators).
+__device__ __forceinline__ float sum8(const float (&acc)[4][2]) {
+  return ((acc[0][0] + acc[0][1]) + (acc[1][0] + acc[1][1])) +
+         ((acc[2][0] + acc[2][1]) + (acc[3][0] + acc[3][1]));
+}
+
 // p = 2^(cs * s - m_use) for one 64-column half (0 at columns >= lim when kMask),
 // packed into 32 fp16 pairs (pk[c / 2], low half = even column c of the half).
-// Returns the half's row sum.  Unmasked halves run on the packed fp32x2 pipe.
+// Returns the half's row sum, taken over the fp16-rounded p.  Unmasked halves run on
+// the packed fp32x2 pipe.
 template <bool kMask, int kHalf>
 __device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float cs, float m_use,
                                                int lim, uint32_t (&pk)[32]) {
+  float acc[4][2] = {};
   if constexpr (!kMask) {
-    uint64_t acc[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
     const uint64_t cs2 = f2_make(cs, cs), negm2 = f2_make(-m_use, -m_use);
 #pragma unroll
     for (int c = 0; c < 64; c += 2) {
@@ -257,42 +250,35 @@ __device__ __forceinline__ float half_exp_pack(const uint32_t (&h)[2][32], float
                                          __uint_as_float(h[(c + 1) >> 5][(c + 1) & 31])),
                                  cs2, negm2);
       float2 pp;
-      if (emu_pair<ATTN_EXP_EMU_PERIOD>(c >> 1)) {
+      if (emu_pair<kExpEmuPeriod>(c >> 1)) {
         pp = exp2_poly2(x2);
       } else {
         const float2 x = f2_split(x2);
         pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       }
-      acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_make(pp.x, pp.y));
       pk[c >> 1] = pack2<false>(pp.x, pp.y);
+      add_f16x2_f32(acc[(c >> 1) & 3][0], acc[(c >> 1) & 3][1], pk[c >> 1]);
     }
-    const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
-    return a.x + a.y;
   } else {
-    float acc[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int c = 0; c < 64; c += 2) {
       const float x0 = fmaf(__uint_as_float(h[c >> 5][c & 31]), cs, -m_use);
       const float x1 = fmaf(__uint_as_float(h[(c + 1) >> 5][(c + 1) & 31]), cs, -m_use);
       const float p0 = (64 * kHalf + c) < lim ? ex2_approx(x0) : 0.f;
       const float p1 = (64 * kHalf + c + 1) < lim ? ex2_approx(x1) : 0.f;
-      acc[(c >> 1) & 3] += p0 + p1;
       pk[c >> 1] = pack2<false>(p0, p1);
+      add_f16x2_f32(acc[(c >> 1) & 3][0], acc[(c >> 1) & 3][1], pk[c >> 1]);
     }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
+  return sum8(acc);
 }
 
 // Unmasked half row (64 columns, registers h) against the running max m_use: packs
-// p = 2^(cs * s - m_use) into 32 fp16 pairs and returns the half's row sum; xmax gets the
-// largest exponent cs * s - m_use seen (the caller redoes the tile if it exceeds 8).
+// p = 2^(cs * s - m_use) into 32 fp16 pairs and returns the half's row sum (of the rounded p); xmax
+// gets the largest exponent cs * s - m_use seen (the caller redoes the tile if it exceeds 8).
 __device__ __forceinline__ float half_exp_pack_spec(const uint32_t (&h)[2][32], float cs, float m_use,
                                                     uint32_t (&pk)[32], float& xmax) {
-  uint64_t acc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
+  float acc[4][2] = {};
   float mx[2] = {xmax, -INFINITY};
   const uint64_t cs2 = f2_make(cs, cs), negm2 = f2_make(-m_use, -m_use);
 #pragma unroll
@@ -303,17 +289,16 @@ __device__ __forceinline__ float half_exp_pack_spec(const uint32_t (&h)[2][32], 
     const float2 x = f2_split(x2);
     mx[(c >> 1) & 1] = fmax3(mx[(c >> 1) & 1], x.x, x.y);
     float2 pp;
-    if (emu_pair<ATTN_EXP_EMU_PERIOD>(c >> 1)) {
+    if (emu_pair<kExpEmuPeriod>(c >> 1)) {
       pp = exp2_poly2(x2);
     } else {
       pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
     }
-    acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_make(pp.x, pp.y));
     pk[c >> 1] = pack2<false>(pp.x, pp.y);
+    add_f16x2_f32(acc[(c >> 1) & 3][0], acc[(c >> 1) & 3][1], pk[c >> 1]);
   }
   xmax = fmaxf(mx[0], mx[1]);
-  const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
-  return a.x + a.y;
+  return sum8(acc);
 }
 
 // Max over the 128 scores of an S row (sign-flipped for a negative scale),
@@ -341,7 +326,7 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32], int lim) {
 }
 
 // p for the column pair (c, c+1): 2^(cs * s - m_use); the FMA-pipe polynomial for every
-// ATTN_EXP_EMU_PERIOD_D64-th pair, MUFU ex2 otherwise; 0 at columns >= lim when kMask.
+// kExpEmuPeriodD64-th pair, MUFU ex2 otherwise; 0 at columns >= lim when kMask.
 template <bool kMask>
 __device__ __forceinline__ float2 pair_exp(const uint32_t (&sr)[4][32], int c, uint64_t cs2,
                                            uint64_t negm2, int lim) {
@@ -349,7 +334,7 @@ __device__ __forceinline__ float2 pair_exp(const uint32_t (&sr)[4][32], int c, u
                                      __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31])),
                              cs2, negm2);
   float2 pp;
-  if (!kMask && emu_pair<ATTN_EXP_EMU_PERIOD_D64>(c >> 1)) {
+  if (!kMask && emu_pair<kExpEmuPeriodD64>(c >> 1)) {
     pp = exp2_poly2(x2);
   } else {
     const float2 x = f2_split(x2);
@@ -363,14 +348,12 @@ __device__ __forceinline__ float2 pair_exp(const uint32_t (&sr)[4][32], int c, u
 }
 
 // The 128 p values of the row, packed to fp16 pairs, stored into 64 TMEM columns at
-// tP (lane = row) in four 16-column pieces.  Returns the row sum.
+// tP (lane = row) in four 16-column pieces.  Returns the row sum of the fp16-rounded p.
 template <bool kMask>
 __device__ __forceinline__ float row_exp_to_tmem(const uint32_t (&sr)[4][32], float cs, float m_use,
                                                  int lim, uint32_t tP) {
   const uint64_t cs2 = f2_make(cs, cs), negm2 = f2_make(-m_use, -m_use);
-  uint64_t acc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = f2_make(0.f, 0.f);
+  float acc[4][2] = {};
 #pragma unroll
   for (int q32 = 0; q32 < 4; ++q32) {
     uint32_t w[16];
@@ -378,40 +361,13 @@ __device__ __forceinline__ float row_exp_to_tmem(const uint32_t (&sr)[4][32], fl
     for (int i = 0; i < 16; ++i) {
       const int c = q32 * 32 + 2 * i;
       const float2 pp = pair_exp<kMask>(sr, c, cs2, negm2, lim);
-      acc[i & 3] = f2_add(acc[i & 3], f2_make(pp.x, pp.y));
       w[i] = pack2<false>(pp.x, pp.y);
+      add_f16x2_f32(acc[i & 3][0], acc[i & 3][1], w[i]);
     }
     tmem_st16(tP + q32 * 16, w);
   }
-  const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
-  return a.x + a.y;
+  return sum8(acc);
 }
-
-// Optional timeline instrumentation (build with -DATTN_TRACE): the first
-// kTraceCtas CTAs record clock64() at fixed points of every role of their first
-// unit into g_prefill_trace, read back with attn_trace_read().  Compiled out otherwise.
-#ifdef ATTN_TRACE
-constexpr int kTraceCtas = 4;
-constexpr int kTraceSlots = 2048;
-__device__ long long g_prefill_trace[kTraceCtas][kTraceSlots];
-#define ATTN_TRACE_POINT(slot)                                                        \
-  do {                                                                                \
-    if (blockIdx.x < kTraceCtas && (slot) < kTraceSlots)                              \
-      g_prefill_trace[blockIdx.x][(slot)] = clock64();                                \
-  } while (0)
-// per-CTA wall-clock span (globaltimer at start and end) and units done, first 4096 CTAs
-__device__ unsigned long long g_cta_span[4096][3];
-#else
-#define ATTN_TRACE_POINT(slot) \
-  do {                         \
-  } while (0)
-#endif
-// trace slot layout (first unit only): 0 start; 1 + 64*t + j: MMA saw P_t(j) ready;
-// 129 + 64*t + j: MMA issued S_t(j+1); 257 + 64*t + j: softmax t saw S_t(j);
-// 385 + ...: S loaded; 513 + ...: max done; 641 + ...: P computed; 769 + ...: P ready
-// arrived; 897 + i: producer issued ring item i.  Per unit k < 64 (all units):
-// 1024 + k: MMA read unit k; 1088 + k: MMA issued its first S; 1152 + 64*t + k: softmax t
-// read unit k; 1280 + 64*t + k: softmax t saw O_t final; 1408 + 64*t + k: softmax t epilogue done.
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
@@ -469,10 +425,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) ATTN_TRACE_POINT(0);
-#ifdef ATTN_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][0] = global_timer_ns();
-#endif
 
   // Every role walks the same unit sequence, decoded and published by the producer.
   // Returns the k-th unit (nmax < 0: no more) after this warp has read it and released
@@ -558,7 +510,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tma_load_4d_w(sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
                           BAR(C::kBarQFull + t), bx * 64, u.h, u.row0[t], u.b);
           q_pending[t] = true;
-          if (lane == 0 && k < 64) ATTN_TRACE_POINT(1600 + 64 * t + k);
         }
         ++nq[t];
       }
@@ -574,8 +525,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_4d_w(sbase + C::kOffKV + stage * C::kTileBytes + bx * C::kBoxBytes, map,
                         BAR(C::kBarKVFull + stage), bx * 64, u.h, (i >> 1) * 128, u.b);
-        if (lane == 0 && k == 0) ATTN_TRACE_POINT(897 + i);
-        if (lane == 0 && i == 0 && k < 64) ATTN_TRACE_POINT(1728 + k);
       }
       claim_next();  // units without K/V tiles
       int next = -1;
@@ -633,20 +582,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     for (int k = 0;; ++k) {
       const PrefillUnit u = next_unit(k);
       if (u.nmax < 0) break;
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1024 + k);
-#ifdef ATTN_TRACE
-      if (lane == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][2] = k + 1;
-#endif
-#ifdef ATTN_TRACE
-      if (lane == 0 && k < 64 && blockIdx.x < kTraceCtas) g_prefill_trace[blockIdx.x][1536 + k] = u.id;
-#endif
       if (u.nmax == 0) continue;
       for (int t = 0; t < 2; ++t)
         if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1792 + k);
       // prologue: S_t(0) for both tiles from K_0
       mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1856 + k);
       __syncwarp();
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
@@ -658,7 +598,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
           }
         tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
       }
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1088 + k);
       for (int j = 0; j < u.nmax; ++j) {
         // next score tiles: S_t(j+1) as soon as the softmax has read S_t(j) out of TMEM
         const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
@@ -679,7 +618,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             issue_s(t, stage_addr(ik));
             tc_commit_w(BAR(C::kBarSFull + t));
             if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
-            if (lane == 0 && k == 0) ATTN_TRACE_POINT(129 + 64 * t + j);
           }
         }
         if (k_ready && !warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
@@ -693,7 +631,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
           mbar_wait(BAR(C::kBarPFull + t), npf[t] & 1, wctx);
           ++npf[t];
           __syncwarp();
-          if (lane == 0 && k == 0) ATTN_TRACE_POINT(1 + 64 * t + j);
           tc_fence_after_sync();
           if (warp_flag(abort_flag)) continue;
           issue_pv(t, stage_addr(iv), j > 0);
@@ -740,20 +677,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     for (int k = 0;; ++k) {
       const PrefillUnit u = next_unit(k);
       if (u.nmax < 0) break;
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1024 + k);
-#ifdef ATTN_TRACE
-      if (lane == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][2] = k + 1;
-#endif
-#ifdef ATTN_TRACE
-      if (lane == 0 && k < 64 && blockIdx.x < kTraceCtas) g_prefill_trace[blockIdx.x][1536 + k] = u.id;
-#endif
       if (u.nmax == 0) continue;
       for (int t = 0; t < 2; ++t)
         if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1792 + k);
       // prologue: S_t(0) for both tiles from K_0
       mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
-      if (lane == 0 && k < 64) ATTN_TRACE_POINT(1856 + k);
       __syncwarp();
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
@@ -763,7 +691,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tc_commit_w(BAR(C::kBarSFull + t));
             if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
           }
-        if (lane == 0 && k < 64) ATTN_TRACE_POINT(1088 + k);
         tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
       }
       for (int j = 0; j < u.nmax; ++j) {
@@ -772,20 +699,17 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
                   wctx);
         __syncwarp();
         const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
-        if (lane == 0 && k == 0 && j < 32) ATTN_TRACE_POINT(1920 + j);
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= u.nkv[t]) continue;
           // keys 64..127 as soon as that half of P_t(j) is written, then keys 0..63
           mbar_wait(BAR(C::kBarPHalf + t), np[t] & 1, wctx);
           __syncwarp();
-          if (lane == 0 && k == 0 && j < 32) ATTN_TRACE_POINT(1952 + 32 * t + j);
           tc_fence_after_sync();
           if (!warp_flag(abort_flag)) issue_pv4(t, stage_addr(iv), 4, j > 0);
           mbar_wait(BAR(C::kBarPFull + t), np[t] & 1, wctx);
           ++np[t];
           __syncwarp();
-          if (lane == 0 && k == 0) ATTN_TRACE_POINT(1 + 64 * t + j);
           tc_fence_after_sync();
           if (warp_flag(abort_flag)) continue;
           issue_pv4(t, stage_addr(iv), 0, true);
@@ -799,7 +723,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             issue_s(t, stage_addr(ik));
             tc_commit_w(BAR(C::kBarSFull + t));
             if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
-            if (lane == 0 && k == 0) ATTN_TRACE_POINT(129 + 64 * t + j);
           } else {
             tc_commit_w(BAR(C::kBarPVDone + t));
           }
@@ -824,7 +747,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     // tile, then arrives on its v_conv barrier (the MMA issuer waits on that for V
     // tiles) and on its empty barrier (the producer refills a stage only after both the
     // tensor core and the converters are done with it).
+    // A V element of magnitude 65536 or more (or inf / NaN) has no fp16 value: the
+    // largest magnitude bit pattern met is tracked per thread and, if any such element
+    // was converted, the call's status word records kStatusRange.
     const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
+    uint32_t vmag = 0;  // per-halfword max of |bf16 bits| over every V element converted
     int g = 0;
     for (int k = 0;; ++k) {
       const PrefillUnit u = next_unit(k);
@@ -840,6 +767,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
 #pragma unroll 4
             for (int c = ct; c < C::kTileBytes / 16; c += 64) {
               uint4 w = tile[c];
+              vmag = __vmaxu2(vmag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                             __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
               w.x = bf16x2_to_f16x2_sat(w.x);
               w.y = bf16x2_to_f16x2_sat(w.y);
               w.z = bf16x2_to_f16x2_sat(w.z);
@@ -857,6 +786,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       }
       g += 2 * u.nmax;
     }
+    if (max(vmag & 0xFFFFu, vmag >> 16) >= kBf16NoF16) atomicCAS(p.status, 0, kStatusRange);
   } else {
     if constexpr (C::kDecoupled) {
     // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ======
@@ -878,7 +808,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     for (int k = 0;; ++k) {
       const PrefillUnit u = next_unit(k);
       if (u.nmax < 0) break;
-      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1152 + 64 * t + k);
       const int row0 = u.row0[t];
       const int nkv = u.nkv[t];
       const int grow = row0 + r;  // global query row
@@ -900,7 +829,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         mbar_wait(BAR(C::kBarSFull + t), ns & 1, wctx);
         ++ns;
         __syncwarp();  // lanes may leave the bounded wait on different polls
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(257 + 64 * t + j);
         tc_fence_after_sync();
         uint32_t sr[4][32];
 #pragma unroll
@@ -912,7 +840,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kBarSFree + t));
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(385 + 64 * t + j);
 
         // mask needed on the key tail and on tiles crossing the causal diagonal
         const long long key0 = (long long)j * 128;
@@ -927,7 +854,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         }
         const float mx = need_mask ? (neg ? row_max<true, true>(sr, lim) : row_max<true, false>(sr, lim))
                                    : (neg ? row_max<false, true>(sr, lim) : row_max<false, false>(sr, lim));
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(513 + 64 * t + j);
         const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cs_abs;
         const float m_new = fmaxf(m_run, m_tile);
         const bool rescale = m_new > m_run + 8.0f;
@@ -959,19 +885,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
 
         l_run += need_mask ? row_exp_to_tmem<true>(sr, cs, m_use, lim, tP)
                            : row_exp_to_tmem<false>(sr, cs, m_use, lim, tP);
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
       }
 
       // ---- epilogue: O / l -> 16-bit -> swizzled staging (this tile's buffer) -> TMA store
       mbar_wait(BAR(C::kBarPVDone + t), (npv + nkv - 1) & 1, wctx);
       npv += nkv;
       __syncwarp();
-      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1280 + 64 * t + k);
       tc_fence_after_sync();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       uint32_t o[D / 32][32];  // the whole O row: one TMEM round trip
@@ -1018,7 +941,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
                                       : -INFINITY;
         p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
       }
-      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1408 + 64 * t + k);
     }
     if (r == 0) bulk_wait_group_read0();  // the last O store has read the staging buffer
     } else {
@@ -1055,7 +977,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         store_pending = false;
       }
       if (u.nmax < 0) break;
-      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1152 + 64 * t + k);
       const int row0 = u.row0[t];
       const int nkv = u.nkv[t];
       const int grow = row0 + r;  // global query row
@@ -1079,7 +1000,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         mbar_wait(BAR(C::kBarSFull + t), ns & 1, wctx);
         ++ns;
         __syncwarp();  // lanes may leave the bounded wait on different polls
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(257 + 64 * t + j);
         tc_fence_after_sync();
         // mask needed on the key tail and on tiles crossing the causal diagonal
         const long long key0 = (long long)j * 128;
@@ -1097,7 +1017,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         // the tile max is found; P stays in registers and is written only if no exponent
         // exceeds 8 in any row of the warp (S is untouched until then), else the two-pass
         // path below redoes the tile.
-        if (ATTN_SPECULATIVE && j > 0 && !need_mask && __all_sync(0xffffffffu, m_run != -INFINITY)) {
+        if (j > 0 && !need_mask && __all_sync(0xffffffffu, m_run != -INFINITY)) {
           uint32_t pk[2][32];
           float xmax = -INFINITY;
           float rs;
@@ -1108,19 +1028,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tmem_ld_wait();
             reg_order_after_wait(sv[0]);
             reg_order_after_wait(sv[1]);
-            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(385 + 64 * t + j);
             rs = half_exp_pack_spec(sv, cs, m_run, pk[1], xmax);
             tmem_ld32(tS + 0, sv[0]);
             tmem_ld32(tS + 32, sv[1]);
             tmem_ld_wait();
             reg_order_after_wait(sv[0]);
             reg_order_after_wait(sv[1]);
-            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(513 + 64 * t + j);
             rs += half_exp_pack_spec(sv, cs, m_run, pk[0], xmax);
           }
           if (!__any_sync(0xffffffffu, xmax > 8.0f)) {
             l_run += rs;
-            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
             tmem_st32(tS + 96, pk[1]);  // keys 64..127
             tmem_st_wait();
             tc_fence_before_sync();
@@ -1131,8 +1048,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
-            if (lane == 0 && k == 0 && j >= 8 && j < 12) ATTN_TRACE_POINT(2016 + (j - 8) * 8 + t * 4 + quarter);
-            if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
             continue;
           }
         }
@@ -1144,7 +1059,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         tmem_ld_wait();
         reg_order_after_wait(hv[0]);
         reg_order_after_wait(hv[1]);
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(385 + 64 * t + j);
         float mx = need_mask ? (neg ? half_max<true, true, 0>(hv, lim) : half_max<true, false, 0>(hv, lim))
                              : (neg ? half_max<false, true, 0>(hv, lim) : half_max<false, false, 0>(hv, lim));
         tmem_ld32(tS + 64, hv[0]);
@@ -1154,7 +1068,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         reg_order_after_wait(hv[1]);
         mx = fmaxf(mx, need_mask ? (neg ? half_max<true, true, 1>(hv, lim) : half_max<true, false, 1>(hv, lim))
                                  : (neg ? half_max<false, true, 1>(hv, lim) : half_max<false, false, 1>(hv, lim)));
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(513 + 64 * t + j);
         const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cs_abs;
         const float m_new = fmaxf(m_run, m_tile);
         const bool rescale = m_new > m_run + 8.0f;
@@ -1201,21 +1114,18 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         rs += need_mask ? half_exp_pack<true, 0>(hv, cs, m_use, lim, pk)
                         : half_exp_pack<false, 0>(hv, cs, m_use, lim, pk);
         l_run += rs;
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(641 + 64 * t + j);
         __syncwarp();
         tmem_st32(tS + 64, pk);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kBarPFull + t));
-        if (threadIdx.x == 128 * t && k == 0) ATTN_TRACE_POINT(769 + 64 * t + j);
       }
 
       // ---- epilogue: O / l -> 16-bit -> swizzled staging buffer -> TMA store
       mbar_wait(BAR(C::kBarPVDone + t), no & 1, wctx);
       ++no;
       __syncwarp();
-      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1280 + 64 * t + k);
       tc_fence_after_sync();
       ostage_acquire(k);  // the previous store from the staging buffer has read it
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
@@ -1258,7 +1168,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
                                       : -INFINITY;
         p.lse[((long long)u.b * p.H + u.h) * p.Nq + grow] = lse;
       }
-      if (threadIdx.x == 128 * t && k < 64) ATTN_TRACE_POINT(1408 + 64 * t + k);
     }
     }
   }
@@ -1266,9 +1175,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   // ---- teardown: every role is done with TMEM
   tc_fence_before_sync();
   __syncthreads();
-#ifdef ATTN_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 4096) g_cta_span[blockIdx.x][1] = global_timer_ns();
-#endif
   if (warp == C::kMmaWarp) {
     __syncwarp();
     tc_fence_after_sync();

@@ -15,7 +15,12 @@
 namespace attn_b200 {
 
 // Status codes shared with include/attn.h (device-side subset).
-constexpr int kStatusTimeout = -4;
+constexpr int kStatusTimeout = -4;  // ATTN_ERR_TIMEOUT
+constexpr int kStatusRange = -5;    // ATTN_ERR_RANGE
+
+// Smallest bf16 magnitude bit pattern with no fp16 value: 0x4780 = 65536 (the bf16 value
+// below it, 65280, is within the fp16 range of +-65504); inf and NaN lie above it.
+constexpr uint32_t kBf16NoF16 = 0x4780u;
 
 // ---------------------------------------------------------------------------
 // generic helpers
@@ -127,7 +132,21 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
   }
 }
 
-// bf16 pair -> fp16 pair (round to nearest even, saturating to +-65504).
+// a += low fp16 half of w, b += high fp16 half of w: each half is widened exactly and
+// added in fp32 with one rounding (the sm_100 mixed-precision add).  The softmax sums the
+// fp16-rounded P that the tensor core multiplies, so O = (P V) / l is normalised by the
+// sum of the very weights it was built from.
+__device__ __forceinline__ void add_f16x2_f32(float& a, float& b, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\t"
+      "add.rn.f32.f16 %1, hi, %1;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "r"(w));
+}
+
+// bf16 pair -> fp16 pair (round to nearest even, saturating to +-65504; the prefill's
+// converter warps report magnitudes that saturate, see kBf16NoF16).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
   const float lo = __uint_as_float(w << 16);
   const float hi = __uint_as_float(w & 0xFFFF0000u);
@@ -157,23 +176,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// Optional upper bound (ns) on how long one try_wait may suspend the thread; 0 = the
-// hardware's default.
-#ifndef ATTN_WAIT_HINT_NS
-#define ATTN_WAIT_HINT_NS 0
-#endif
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-#if ATTN_WAIT_HINT_NS > 0
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "n"(ATTN_WAIT_HINT_NS)
-      : "memory");
-#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -181,7 +185,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
-#endif
   return ok != 0;
 }
 

@@ -50,7 +50,8 @@ typedef enum {
                                   buffers, non-finite scale, size beyond a stated limit */
     ATTN_ERR_UNSUPPORTED = -2, /* head_dim not in {64, 128}, unknown dtype, device not sm_100 */
     ATTN_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed (launch, allocation...) */
-    ATTN_ERR_TIMEOUT = -4      /* device side: a bounded pipeline wait gave up (see attn_get_status) */
+    ATTN_ERR_TIMEOUT = -4,     /* device side: a bounded pipeline wait gave up (see attn_get_status) */
+    ATTN_ERR_RANGE = -5        /* device side: a bf16 V element has no fp16 value (see attn_fwd) */
 } attn_status_t;
 
 /*
@@ -72,10 +73,19 @@ typedef enum {
  * default memory pool and returned on the same stream); every other shape runs
  * the tiled prefill kernel.  Both give the same result up to fp32 rounding.
  *
+ * Value range (bf16 only): the tiled prefill multiplies P by V with both in
+ * fp16 (fp16's 11-bit significand keeps the rounding of P small), converting
+ * each bf16 V tile to fp16 on chip.  A V element of magnitude 65536 or more,
+ * or an infinite or NaN one, has no fp16 value: the call then records
+ * ATTN_ERR_RANGE in the status word read by attn_get_status(), and its O is
+ * undefined.  Elements below 2^-14 in magnitude keep an absolute error under
+ * 2^-25.  The decode path (Nq == 1) computes in fp32 and has no such limit.
+ *
  * Asynchronous: the call validates its arguments on the host, enqueues the
  * kernels on `stream` and returns.  Argument errors return before anything is
- * enqueued.  A device-side failure (a bounded wait that expired) does not
- * trap: it is recorded in a per-device status word read by attn_get_status().
+ * enqueued.  A device-side failure (a bounded wait that expired, a V value out
+ * of range) does not trap: it is recorded in a per-device status word read by
+ * attn_get_status().
  * Since the call only enqueues work (and stream-ordered allocations) on
  * `stream`, it can be captured into a CUDA graph once a first call on the
  * device has run (that call sets the kernels' shared-memory attributes).
@@ -119,13 +129,18 @@ ATTN_API int attn_fwd_decode(const void* q, const void* k, const void* v, void* 
  * ATTN_ERR_INVALID_ARG and launches nothing.  Every GPU that loads the
  * library holds the 4 MiB array until the process exits.
  *
+ * With splits = 0 the automatic choice only considers split counts whose
+ * partials fit the array, so a shape that fits with fewer splits runs.
+ *
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's
- * contents; nothing in it has to start at zero, because every slot the
- * combining kernel reads is written earlier in the same call.  Calls whose
- * kernels overlap on the GPU (other streams, other host threads) race on the
- * array and corrupt each other's results: serialise them.
+ * device current) and caches it for the life of the process; make that first
+ * call before any stream capture, and do not keep using the library across a
+ * reset of the device (cudaDeviceReset), which invalidates the cached address.
+ * All calls share the one array and it keeps the last call's contents; nothing
+ * in it has to start at zero, because every slot the combining kernel reads is
+ * written earlier in the same call.  Calls whose kernels overlap on the GPU
+ * (other streams, other host threads) race on the array and corrupt each
+ * other's results: serialise them.
  */
 ATTN_API int attn_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* out,
                                      float* lse, int B, int H, int Nk, int d, float scale,
@@ -171,9 +186,11 @@ ATTN_API int attn_fwd_decode_paged(const void* q, const void* k_cache, const voi
 
 /*
  * attn_get_status -- synchronises `stream`, then returns and clears the
- * current device's status word: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel
- * since the last call gave up on a pipeline wait (its outputs are then
- * undefined), or ATTN_ERR_CUDA if the synchronisation itself failed.
+ * current device's status word: ATTN_OK; ATTN_ERR_TIMEOUT if any kernel since
+ * the last call gave up on a pipeline wait, or ATTN_ERR_RANGE if a bf16 prefill
+ * met a V value with no fp16 value (the first such event is kept; the outputs
+ * of the call it came from are undefined); or ATTN_ERR_CUDA if the
+ * synchronisation itself failed.
  */
 ATTN_API int attn_get_status(attn_stream_t stream);
 
