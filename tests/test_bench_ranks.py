@@ -106,3 +106,46 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert len(lines) == 1
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_launch_plan(monkeypatch):
+    """--gpus N means N ranks: run as is, relaunch a single process as N ranks, or refuse."""
+    import bench
+    monkeypatch.delenv("RANK", raising=False)
+    assert bench.launch_plan(1, 1) == "run"
+    assert bench.launch_plan(4, 1) == "spawn"
+    assert bench.launch_plan(0, 1) == "refuse"
+    monkeypatch.setenv("RANK", "0")
+    assert bench.launch_plan(2, 2) == "run"
+    assert bench.launch_plan(3, 2) == "refuse"
+    assert bench.launch_plan(2, 1) == "refuse"  # a launcher started one rank
+
+
+def test_gpus_two_without_a_launcher_runs_two_ranks():
+    """`bench.py --gpus 2` started as one process relaunches itself as two ranks (gloo-free
+    reference arm on CPU): one JSON line, from rank 0, with n_gpus 2."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    res = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                          "--gpus", "2", "--steps", "1", "--warmup", "3"], cwd=root, env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_gpus_mismatch_with_the_launcher_is_refused():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                          "--gpus", "3", "--steps", "1"], cwd=root, env=env, capture_output=True,
+                         text=True, timeout=120)
+    assert res.returncode == 2
+    assert "--gpus 3" in res.stderr and not res.stdout.strip()

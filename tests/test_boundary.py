@@ -53,7 +53,7 @@ def test_only_the_c_abi_is_exported():
 
 def test_version_and_error_strings(lib):
     assert lib.attn_version() == 10000
-    for code in (0, -1, -2, -3, -4):
+    for code in (0, -1, -2, -3, -4, -5):
         assert len(lib.attn_error_string(code)) > 10
     assert b"unknown" in lib.attn_error_string(-99)
 
