@@ -12,8 +12,11 @@ synchronise, CUDA events on the launching stream, max over ranks; the stream spi
 on the device while the host enqueues the K steps, so they run back to back (the
 spin is outside the timed intervals).  Every rank runs an independent replica of
 the workload (the forward of one (b, h) never talks to another, so there is no
-data-path collective): scaling is weak.  `extra` carries the decode, causal8k and
-bf16_k3 workloads and the decode over a 16-key-page cache, each with its roofline.
+data-path collective): scaling is weak.  `--gpus N` means N ranks: started as one
+process, the script relaunches itself under torchrun with N ranks; started by a
+launcher with a different number of ranks, it exits with status 2.  `extra`
+carries the decode, causal8k, causal8000 and bf16_k3 workloads and the decode over a
+16-key-page cache, each with its roofline.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the method available here) on bounded samples of the same workload.
@@ -167,6 +170,34 @@ def dist_setup(args):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def launch_plan(gpus, world):
+    """What `--gpus N` means for a process that sees WORLD_SIZE `world`:
+    "run" (already N ranks), "spawn" (a single process asked for N > 1 ranks: it
+    relaunches itself under torchrun with N ranks) or "refuse" (a launcher started a
+    different number of ranks than --gpus says)."""
+    if gpus < 1:
+        return "refuse"
+    if world == gpus:
+        return "run"
+    if world == 1 and "RANK" not in os.environ:
+        return "spawn"
+    return "refuse"
+
+
+def spawn_ranks(gpus, argv):
+    """Relaunch this script as `gpus` ranks (one per GPU) under torchrun on 127.0.0.1;
+    returns torchrun's exit code."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(gpus), "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def max_over_ranks(x, world, device="cuda"):
@@ -410,7 +441,7 @@ def measure_paged(name, K, W, world, device, peaks):
     return {"value": world * K * nbytes / (elapsed_ms * 1e-3) / 1e9, "unit": "GB/s",
             "ms_per_step": elapsed_ms / K,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(name),
                          "algorithmic_bytes_per_launch": nbytes,
                          "note": "launch time includes the combine kernel"},
             "clocks": sampler.summary(),
@@ -435,11 +466,27 @@ def run_ours(args):
     peaks = load_peaks()
     K, W = args.steps, max(3, args.warmup)
 
-    from attention_forward_tiled_b200.inputs import WORKLOADS
+    from attention_forward_tiled_b200.inputs import PAGED_WORKLOADS, WORKLOADS
+    if args.workload in PAGED_WORKLOADS:
+        # the paged decode on its own (profiling runs): its line has no end-to-end figure
+        r = measure_paged(args.workload, K, W, world, device, peaks)
+        line = {"metric": METRIC, "value": r["value"], "unit": r["unit"], "n_gpus": world, "steps": K,
+                "warmup": W, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": PAGED_WORKLOADS[args.workload]["dtype"],
+                "data": "synthetic (seeded randn, pages placed at random)", "config": r["config"],
+                "roofline": r["roofline"], "e2e": None, "gpu_launches": 2 * K, "clocks": r["clocks"],
+                "impl": "ours"}
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     main = measure_workload(args.workload, K, W, world, device, peaks, want_e2e=True)
     extra = {}
     if not args.no_extra:
-        for name in ("decode", "causal8k", "bf16_k3"):
+        for name in ("decode", "causal8k", "causal8000", "bf16_k3"):
             if name == args.workload:
                 continue
             r = measure_workload(name, K, W, world, device, peaks, want_e2e=False)
@@ -545,6 +592,13 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the decode/causal8k/bf16 lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    plan = launch_plan(args.gpus, world)
+    if plan == "spawn":
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
+    if plan == "refuse":
+        sys.stderr.write("bench.py: --gpus %d but the launcher started %d rank(s)\n" % (args.gpus, world))
+        sys.exit(2)
     if args.impl == "reference":
         run_reference(args)
     else:
