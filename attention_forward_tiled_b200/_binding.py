@@ -29,6 +29,8 @@ SIGNATURES = {
     "attn_fwd_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "attn_fwd_decode_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
                                    _i, _vp]),
+    "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                            _i, _i, _vp]),
     "attn_get_status": (_i, [_vp]),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_version": (_i, []),
@@ -204,6 +206,57 @@ def attn_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None
             _stream_ptr(stream, q.device))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_decode_paged")
+    return out, lse
+
+
+def attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, causal=False, scale=None, out=None,
+                   lse=None, return_lse=True, stream=None, splits=0):
+    """Lq <= 16 query tokens per request over a paged key/value cache (tensor cores).
+
+    q [B, Lq, H, d]; k_cache, v_cache [num_blocks, page_size, H, d] (q's dtype);
+    block_table [B, max_blocks] and seq_lens [B], int32 CUDA tensors.  Request b's
+    tokens are the last Lq positions of its seq_lens[b] keys; with causal, token i
+    sees keys up to its own position.  Returns (out [B, Lq, H, d], lse [B, H, Lq]
+    float32 or None).
+    """
+    import torch
+    lib = load_library()
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("block_table", block_table), ("seq_lens", seq_lens)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA tensor")
+        if t.device != q.device:
+            raise ValueError(f"{name} must be on q's device {q.device}")
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, tokens, heads, head_dim]")
+    B, Lq, H, d = q.shape
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q, k_cache, v_cache must share one dtype")
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4 or k_cache.shape[2:] != (H, d):
+        raise ValueError("k_cache and v_cache must be [num_blocks, page_size, heads, head_dim]")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be an int32 [batch, max_blocks] tensor")
+    if seq_lens.dtype != torch.int32 or seq_lens.shape != (B,):
+        raise ValueError("seq_lens must be an int32 [batch] tensor")
+    num_blocks, page_size = k_cache.shape[0], k_cache.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_buffer("lse", lse, (B, H, Lq), torch.float32, q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.attn_fwd_paged(
+            ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k_cache.data_ptr()),
+            ctypes.c_void_p(v_cache.data_ptr()), ctypes.c_void_p(block_table.data_ptr()),
+            ctypes.c_void_p(seq_lens.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+            ctypes.c_void_p(lse.data_ptr() if lse is not None else 0), B, H, Lq, d, num_blocks,
+            page_size, block_table.shape[1], int(bool(causal)), scale, _dtype_code(q.dtype),
+            int(splits), _stream_ptr(stream, q.device))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_paged")
     return out, lse
 
 

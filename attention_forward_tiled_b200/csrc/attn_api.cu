@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "decode_mq_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
 
@@ -49,7 +50,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int* status_ptr = nullptr;
-  bool attr_set[12] = {};  // per kernel instantiation: max dynamic shared memory raised
+  bool attr_set[16] = {};  // per kernel instantiation: max dynamic shared memory raised
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -353,10 +354,12 @@ int launch_decode_paged(DeviceState* ds, const void* q, const void* k_cache, con
 // Argument checks of attn_fwd_decode_paged (nothing is enqueued on failure).
 int validate_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
                    const int* seq_lens, const void* out, const float* lse, int B, int H, int d,
-                   int num_blocks, int page_size, int max_blocks, float scale, int dtype, int splits) {
+                   int num_blocks, int page_size, int max_blocks, float scale, int dtype, int splits,
+                   int Lq = 1) {
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return ATTN_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || d <= 0 || num_blocks <= 0 || page_size <= 0 || max_blocks <= 0 || splits < 0)
     return ATTN_ERR_INVALID_ARG;
+  if (Lq < 1 || Lq > kMqMaxQ) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
@@ -372,18 +375,80 @@ int validate_paged(const void* q, const void* k_cache, const void* v_cache, cons
   if (misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) || misaligned(out, 16) ||
       misaligned(block_table, 4) || misaligned(seq_lens, 4) || (lse && misaligned(lse, 4)))
     return ATTN_ERR_INVALID_ARG;
-  const size_t q_bytes = (size_t)B * row_bytes;
+  const size_t q_bytes = (size_t)B * Lq * row_bytes;
   const size_t cache_bytes = (size_t)num_blocks * page_size * row_bytes;
   if (overlaps(out, q_bytes, q, q_bytes) || overlaps(out, q_bytes, k_cache, cache_bytes) ||
       overlaps(out, q_bytes, v_cache, cache_bytes))
     return ATTN_ERR_INVALID_ARG;
   if (lse) {
-    const size_t lse_bytes = (size_t)B * H * sizeof(float);
+    const size_t lse_bytes = (size_t)B * H * Lq * sizeof(float);
     if (overlaps(lse, lse_bytes, out, q_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
         overlaps(lse, lse_bytes, k_cache, cache_bytes) || overlaps(lse, lse_bytes, v_cache, cache_bytes))
       return ATTN_ERR_INVALID_ARG;
   }
   return ATTN_OK;
+}
+
+// Several query tokens per request over a paged cache: the tensor-core partial kernel,
+// then the combine kernel over the key splits.
+template <int D, bool BF16>
+int launch_mq(DeviceState* ds, const void* q, const void* k_cache, const void* v_cache,
+              const int* block_table, const int* seq_lens, void* out, float* lse, int B, int H,
+              int Lq, int num_blocks, int page_size, int max_blocks, int causal, float scale,
+              int splits_req, cudaStream_t stream) {
+  using C = MqCfg<D>;
+  auto kernel = attn_mq_partial_kernel<D, BF16>;
+  const int slot = 12 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  const int Nk = max_blocks * page_size;  // validated < 2^31
+  const int ntiles = (Nk + 127) / 128;
+  const long long BH = (long long)B * H;
+  int splits = splits_req > 0 ? splits_req : choose_splits(BH, ntiles, ds->sm_count);
+  if (splits < 1 || splits > ntiles) return ATTN_ERR_INVALID_ARG;
+  const int tps = (ntiles + splits - 1) / splits;
+  splits = (ntiles + tps - 1) / tps;
+  const long long items = BH * splits;
+  if (items >= (1LL << 31) || items * Lq >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+
+  MqParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  const int page_rows = page_size < 128 ? page_size : 128;
+  if (int rc = encode_bnhd(&p.tm_q, q, B, Lq, H, D, dtype, kMqMaxQ)) return rc;
+  if (int rc = encode_bnhd(&p.tm_k, k_cache, 1, num_blocks * page_size, H, D, dtype, page_rows)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v_cache, 1, num_blocks * page_size, H, D, dtype, page_rows)) return rc;
+  float* part = nullptr;
+  const size_t ws_bytes = (size_t)items * Lq * (D + 2) * sizeof(float);
+  if (cudaMallocAsync(reinterpret_cast<void**>(&part), ws_bytes, stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  p.part = part;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Lq = Lq;
+  p.Nk = Nk;
+  p.causal = causal;
+  p.splits = splits;
+  p.tiles_per_split = tps;
+  p.n_items = (int)items;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.max_blocks = max_blocks;
+  p.page_size = page_size;
+  p.page_rows = page_rows;
+  p.num_blocks = num_blocks;
+  const int grid = (int)std::min<long long>(items, ds->sm_count);
+  kernel<<<dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  int rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  if (rc == ATTN_OK) {
+    const long long rows = BH * Lq;
+    attn_mq_combine_kernel<D, BF16><<<dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream>>>(
+        part, out, lse, B, H, Lq, splits);
+    rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (cudaFreeAsync(part, stream) != cudaSuccess) rc = ATTN_ERR_CUDA;
+  return rc;
 }
 
 // Same kernels as launch_decode, with the partials in g_noalloc_scratch: no allocation.
@@ -529,6 +594,27 @@ int attn_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cach
   return bf16 ? launch_decode_paged<64, true>(ATTN_PAGED_ARGS)
               : launch_decode_paged<64, false>(ATTN_PAGED_ARGS);
 #undef ATTN_PAGED_ARGS
+}
+
+int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                   const int* seq_lens, void* out, float* lse, int B, int H, int Lq, int d,
+                   int num_blocks, int page_size, int max_blocks, int causal, float scale, int dtype,
+                   int splits, attn_stream_t stream) {
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (int rc = validate_paged(q, k_cache, v_cache, block_table, seq_lens, out, lse, B, H, d,
+                              num_blocks, page_size, max_blocks, scale, dtype, splits, Lq))
+    return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_BF16;
+#define ATTN_MQ_ARGS                                                                            \
+  ds, q, k_cache, v_cache, block_table, seq_lens, out, lse, B, H, Lq, num_blocks, page_size,   \
+      max_blocks, causal, scale, splits, st
+  if (d == 128)
+    return bf16 ? launch_mq<128, true>(ATTN_MQ_ARGS) : launch_mq<128, false>(ATTN_MQ_ARGS);
+  return bf16 ? launch_mq<64, true>(ATTN_MQ_ARGS) : launch_mq<64, false>(ATTN_MQ_ARGS);
+#undef ATTN_MQ_ARGS
 }
 
 int attn_get_status(attn_stream_t stream) {

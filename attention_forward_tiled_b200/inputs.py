@@ -34,10 +34,13 @@ WORKLOADS = {
 }
 
 # The decode workload over a paged cache: the same 16 requests x 4096 keys, stored in
-# randomly placed 16-key pages (a common serving page size).
+# randomly placed 16-key pages (a common serving page size).  The speculative-decoding
+# variant scores 8 query tokens per request together (causal within the request).
 PAGED_WORKLOADS = {
     "decode_paged16": dict(B=16, H=32, d=128, seq_lens=[4096] * 16, page_size=16, dtype="f16",
-                           scale=1.0 / math.sqrt(128), seed=6),
+                           scale=1.0 / math.sqrt(128), seed=6, Lq=1, causal=False),
+    "spec8_paged16": dict(B=16, H=32, d=128, seq_lens=[4096] * 16, page_size=16, dtype="f16",
+                          scale=1.0 / math.sqrt(128), seed=7, Lq=8, causal=True),
 }
 
 
@@ -54,8 +57,8 @@ def make_inputs(B, H, Nq, Nk, d, dtype="f16", seed=0, k_mult=1.0, **_):
 
 
 def make_paged_inputs(B, H, d, seq_lens, page_size, dtype="f16", seed=0, max_blocks=None,
-                      spare_pages=3):
-    """Seeded paged decode inputs (CPU tensors): q [B, 1, H, d]; k_cache, v_cache
+                      spare_pages=3, Lq=1):
+    """Seeded paged decode inputs (CPU tensors): q [B, Lq, H, d]; k_cache, v_cache
     [num_blocks, page_size, H, d]; block_table [B, max_blocks] int32 (-1 past each
     sequence); seq_lens [B] int32.  The pages of all requests (plus `spare_pages`
     unused ones) are a random permutation of the cache, so no request's pages are
@@ -64,7 +67,7 @@ def make_paged_inputs(B, H, d, seq_lens, page_size, dtype="f16", seed=0, max_blo
     npages = [(int(L) + page_size - 1) // page_size for L in seq_lens]
     max_blocks = max(max(npages), 1) if max_blocks is None else int(max_blocks)
     num_blocks = sum(npages) + spare_pages
-    q = torch.randn(B, 1, H, d, generator=g, dtype=torch.float32)
+    q = torch.randn(B, Lq, H, d, generator=g, dtype=torch.float32)
     perm = torch.randperm(num_blocks, generator=g)
     k_cache = torch.randn(num_blocks, page_size, H, d, generator=g, dtype=torch.float32)
     v_cache = torch.randn(num_blocks, page_size, H, d, generator=g, dtype=torch.float32)

@@ -15,8 +15,9 @@ the workload (the forward of one (b, h) never talks to another, so there is no
 data-path collective): scaling is weak.  `--gpus N` means N ranks: started as one
 process, the script relaunches itself under torchrun with N ranks; started by a
 launcher with a different number of ranks, it exits with status 2.  `extra`
-carries the decode, causal8k, causal8000 and bf16_k3 workloads and the decode over a
-16-key-page cache, each with its roofline.
+carries the decode, causal8k, causal8000 and bf16_k3 workloads, the decode over a
+16-key-page cache and the 8-token (speculative) decode over the same cache on the
+tensor cores, each with its roofline.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the method available here) on bounded samples of the same workload.
@@ -407,16 +408,23 @@ def measure_paged(name, K, W, world, device, peaks):
     from attention_forward_tiled_b200.inputs import PAGED_WORKLOADS, make_paged_inputs
 
     w = PAGED_WORKLOADS[name]
-    B, H, d = w["B"], w["H"], w["d"]
+    B, H, d, Lq = w["B"], w["H"], w["d"], w["Lq"]
     q, kc, vc, bt, sl = (t.to(device) for t in make_paged_inputs(
-        B, H, d, w["seq_lens"], w["page_size"], dtype=w["dtype"], seed=w["seed"]))
+        B, H, d, w["seq_lens"], w["page_size"], dtype=w["dtype"], seed=w["seed"], Lq=Lq))
     out = torch.empty_like(q)
-    lse = torch.empty((B, H), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
+    if Lq == 1 and not w["causal"]:  # one token: the CUDA-core split-KV decode
+        lse = torch.empty((B, H), dtype=torch.float32, device=device)
 
-    def step():
-        attn.attn_fwd_decode_paged(q, kc, vc, bt, sl, scale=w["scale"], out=out, lse=lse,
-                                   stream=stream)
+        def step():
+            attn.attn_fwd_decode_paged(q, kc, vc, bt, sl, scale=w["scale"], out=out, lse=lse,
+                                       stream=stream)
+    else:  # several tokens per request: the tensor-core kernel
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=device)
+
+        def step():
+            attn.attn_fwd_paged(q, kc, vc, bt, sl, causal=w["causal"], scale=w["scale"], out=out,
+                                lse=lse, stream=stream)
 
     for _ in range(W):
         step()
@@ -446,6 +454,7 @@ def measure_paged(name, K, W, world, device, peaks):
                          "note": "launch time includes the combine kernel"},
             "clocks": sampler.summary(),
             "config": {"workload": name, "B": B, "H": H, "d": d, "seq_lens": "4096 each",
+                       "query_tokens": Lq, "causal": w["causal"],
                        "page_size": w["page_size"], "pages": "randomly placed", "dtype": w["dtype"],
                        "l2": "K+V of 1074 MB per step vs 126 MB L2: no flush"}}
 
@@ -494,6 +503,7 @@ def run_ours(args):
                            "roofline": r["roofline"], "clocks": r["clocks"],
                            "config": workload_config(name, WORKLOADS[name])}
         extra["decode_paged16"] = measure_paged("decode_paged16", K, W, world, device, peaks)
+        extra["spec8_paged16"] = measure_paged("spec8_paged16", K, W, world, device, peaks)
     line = {
         "metric": METRIC,
         "value": main["value"],

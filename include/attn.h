@@ -18,8 +18,12 @@
  *   - a query row with no allowed key yields O = 0 and lse = -inf;
  *   - lse is the natural-log row log-sum-exp of the scaled, masked scores.
  *
- * Nothing here allocates host memory or keeps a pointer after a call returns.
- * All pointers except `stream` are DEVICE pointers on the current CUDA device.
+ * Nothing here allocates host memory or keeps a caller's pointer after a call
+ * returns.  All pointers except `stream` are DEVICE pointers on the current CUDA
+ * device.  Per device, the library caches what it looks up on its first call
+ * there (the device's properties, the kernels' shared-memory attributes, the
+ * addresses of its status word and of the no-alloc array) for the life of the
+ * process: do not keep using it on a device after cudaDeviceReset.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -183,6 +187,41 @@ ATTN_API int attn_fwd_decode_paged(const void* q, const void* k_cache, const voi
                                    float* lse, int B, int H, int d, int num_blocks, int page_size,
                                    int max_blocks, float scale, int dtype, int splits,
                                    attn_stream_t stream);
+
+/*
+ * attn_fwd_paged -- several query tokens per request against a paged key/value
+ * cache, on the tensor cores.
+ *
+ * The speculative-decoding step of the vLLM MiniMax-M3 indexer page ("PR #45743
+ * 完整报告", section "功能与动机": the query tokens of one request are scored
+ * together; section "关键源码片段": per-request int32 seq_lens and a block
+ * table).  Request b's Lq query tokens are the last Lq positions of its
+ * sequence of L = seq_lens[b] keys, stored page by page as for
+ * attn_fwd_decode_paged.  With causal = 1, query i (0-based) sees keys
+ * j <= L - Lq + i (the bottom-right alignment of attn_fwd); with causal = 0
+ * every query sees all L keys.  A query with no key gets O = 0, lse = -inf.
+ *
+ *   q            [B, Lq, H, d]                         dtype   (read)
+ *   k_cache      [num_blocks, page_size, H, d]         dtype   (read)
+ *   v_cache      [num_blocks, page_size, H, d]         dtype   (read)
+ *   block_table  [B, max_blocks]                       int32   (read, DEVICE memory)
+ *   seq_lens     [B]                                   int32   (read, DEVICE memory)
+ *   out          [B, Lq, H, d]                         dtype   (written)
+ *   lse          [B, H, Lq] float32 (written) or NULL
+ *   1 <= Lq <= 16; page_size, max_blocks, num_blocks, splits, seq_lens and
+ *   table entries as attn_fwd_decode_paged; causal 0/1.
+ *
+ * The probabilities multiply V in the input type (fp16 or bf16) and O is
+ * normalised by the sum of those rounded probabilities.  The workspace of
+ * B*H*splits*Lq*(d+2)*4 bytes is taken stream-ordered from the default pool.
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA;
+ * asynchronous like attn_fwd.
+ */
+ATTN_API int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                            const int* block_table, const int* seq_lens, void* out, float* lse,
+                            int B, int H, int Lq, int d, int num_blocks, int page_size,
+                            int max_blocks, int causal, float scale, int dtype, int splits,
+                            attn_stream_t stream);
 
 /*
  * attn_get_status -- synchronises `stream`, then returns and clears the

@@ -18,7 +18,8 @@ import pytest
 from attention_forward_tiled_b200 import build as abuild
 
 THREADS = {"attn_prefill_kernel": 384, "attn_decode_partial_kernel": 160,
-           "attn_decode_combine_kernel": 128}
+           "attn_decode_combine_kernel": 128, "attn_mq_partial_kernel": 192,
+           "attn_mq_combine_kernel": 128}
 # bytes of spill stores / loads per prefill instantiation (head_dim, bf16) at this version
 PREFILL_SPILL_CEILING = {(64, False): (112, 168), (64, True): (152, 300),
                          (128, False): (8, 8), (128, True): (16, 16)}
@@ -66,11 +67,14 @@ def template_args(mangled):
     return int(m.group(1)), m.group(2) == "1"
 
 
+
 def test_every_kernel_is_reported(ptxas_report):
     kinds = [kernel_kind(k) for k in ptxas_report]
     assert kinds.count("attn_prefill_kernel") == 4      # d 64/128 x fp16/bf16
     assert kinds.count("attn_decode_partial_kernel") == 8  # x dense/paged
     assert kinds.count("attn_decode_combine_kernel") == 4
+    assert kinds.count("attn_mq_partial_kernel") == 4
+    assert kinds.count("attn_mq_combine_kernel") == 4
     assert all(kinds)
 
 

@@ -136,6 +136,7 @@ def test_noalloc_allocates_nothing():
     """The device's default memory pool (where the allocating decode takes its partials)
     sees no allocation during a no-alloc call; the allocating call, as a control, does."""
     rt = pytest.importorskip("cuda.bindings.runtime")
+    drv = pytest.importorskip("cuda.bindings.driver")
     lib = attn.load_library()
     stream = torch.cuda.current_stream()
     err, pool = rt.cudaDeviceGetDefaultMemPool(torch.cuda.current_device())
@@ -149,7 +150,7 @@ def test_noalloc_allocates_nothing():
         return int(val)
 
     def reset_high():
-        (e,) = rt.cudaMemPoolSetAttribute(pool, high, rt.cuuint64_t(0))
+        (e,) = rt.cudaMemPoolSetAttribute(pool, high, drv.cuuint64_t(0))
         assert e == rt.cudaError_t.cudaSuccess
 
     B, H, Nk, d = 4, 8, 2048, 128
