@@ -31,6 +31,8 @@ SIGNATURES = {
                                    _i, _vp]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                             _i, _i, _vp]),
+    "attn_indexer_score": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "attn_topk": (_i, [_vp, _i, _i, _i, _vp, _vp]),
     "attn_get_status": (_i, [_vp]),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_version": (_i, []),
@@ -258,6 +260,61 @@ def attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, causal=False, sca
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_paged")
     return out, lse
+
+
+def indexer_score(q, kp, w, mask=None, out=None, stream=None):
+    """Lightning-indexer score: q [B, T, H, d], kp [B, P, d] (fp16/bf16), w [B, T, H]
+    float32, mask [B, T, P] float16 (0 / -inf) or None.  Returns score [B, T, P] float32."""
+    import torch
+    lib = load_library()
+    for name, t in (("q", q), ("kp", kp), ("w", w)) + ((("mask", mask),) if mask is not None else ()):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA tensor")
+        if t.device != q.device:
+            raise ValueError(f"{name} must be on q's device {q.device}")
+    if q.dim() != 4 or kp.dim() != 3:
+        raise ValueError("q must be [B, T, H, d] and kp [B, P, d]")
+    B, T, H, d = q.shape
+    P = kp.shape[1]
+    if kp.shape[0] != B or kp.shape[2] != d or kp.dtype != q.dtype:
+        raise ValueError("kp must be [B, P, d] in q's dtype")
+    if w.dtype != torch.float32 or tuple(w.shape) != (B, T, H):
+        raise ValueError("w must be a float32 [B, T, H] tensor")
+    if mask is not None and (mask.dtype != torch.float16 or tuple(mask.shape) != (B, T, P)):
+        raise ValueError("mask must be a float16 [B, T, P] tensor")
+    if out is None:
+        out = torch.empty((B, T, P), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, (B, T, P), torch.float32, q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.attn_indexer_score(
+            ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(kp.data_ptr()), ctypes.c_void_p(w.data_ptr()),
+            ctypes.c_void_p(mask.data_ptr() if mask is not None else 0), ctypes.c_void_p(out.data_ptr()),
+            B, T, H, P, d, _dtype_code(q.dtype), _stream_ptr(stream, q.device))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_indexer_score")
+    return out
+
+
+def topk(score, k, out=None, stream=None):
+    """Positions [..., k] int32 of the k largest finite scores of each row of score [..., P]
+    (float32 CUDA tensor), largest first, ties to the lower position, -1 padding."""
+    import torch
+    lib = load_library()
+    if not isinstance(score, torch.Tensor) or not score.is_cuda or not score.is_contiguous() \
+            or score.dtype != torch.float32:
+        raise TypeError("score must be a contiguous float32 CUDA tensor")
+    P = score.shape[-1]
+    R = score.numel() // P
+    shape = tuple(score.shape[:-1]) + (int(k),)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.int32, device=score.device)
+    _check_buffer("out", out, shape, torch.int32, score.device)
+    with torch.cuda.device(score.device):
+        rc = lib.attn_topk(ctypes.c_void_p(score.data_ptr()), R, P, int(k), ctypes.c_void_p(out.data_ptr()),
+                           _stream_ptr(stream, score.device))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_topk")
+    return out
 
 
 def get_status(stream=None, device=None):

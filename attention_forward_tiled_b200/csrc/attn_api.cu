@@ -18,6 +18,7 @@
 #include "attn.h"
 #include "decode_mq_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "indexer_sm100.cuh"
 #include "prefill_sm100.cuh"
 
 using namespace attn_b200;
@@ -50,7 +51,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int* status_ptr = nullptr;
-  bool attr_set[16] = {};  // per kernel instantiation: max dynamic shared memory raised
+  bool attr_set[24] = {};  // per kernel instantiation: max dynamic shared memory raised
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -145,6 +146,22 @@ int encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, i
   const CUtensorMapDataType ty =
       dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUresult r = encode(map, ty, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 3-D view (d, rows, B) of a contiguous [B, rows, d] tensor; box (64, 128, 1), 128B swizzle.
+int encode_rows3d(CUtensorMap* map, const void* ptr, int B, long long rows, int d, int dtype) {
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return ATTN_ERR_CUDA;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType ty =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = encode(map, ty, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
@@ -451,6 +468,41 @@ int launch_mq(DeviceState* ds, const void* q, const void* k_cache, const void* v
   return rc;
 }
 
+template <int D, bool BF16>
+int launch_indexer(DeviceState* ds, const void* q, const void* kp, const float* w, const void* mask,
+                   float* score, int B, int T, int H, int P, cudaStream_t stream) {
+  using C = IndexerCfg<D>;
+  auto kernel = attn_indexer_score_kernel<D, BF16>;
+  const int slot = 16 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  IndexerParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  if (int rc = encode_rows3d(&p.tm_q, q, B, (long long)T * H, D, dtype)) return rc;
+  if (int rc = encode_rows3d(&p.tm_k, kp, B, P, D, dtype)) return rc;
+  int lg = 0;
+  while ((1 << lg) < H) ++lg;
+  p.w = w;
+  p.mask = static_cast<const uint16_t*>(mask);
+  p.score = score;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.P = P;
+  p.lg_h = lg;
+  p.tok_per_tile = 128 / H;
+  p.n_ttiles = (T + p.tok_per_tile - 1) / p.tok_per_tile;
+  p.n_ptiles = (P + 127) / 128;
+  const long long items = (long long)B * p.n_ptiles * p.n_ttiles;
+  if (items >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+  p.n_items = (int)items;
+  p.timeout_ns = g_timeout_ns.load();
+  const int grid = (int)std::min<long long>(items, ds->sm_count);
+  const int per_cta = (int)((items + grid - 1) / grid);
+  kernel<<<dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream>>>(p, per_cta);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // Same kernels as launch_decode, with the partials in g_noalloc_scratch: no allocation.
 template <int D, bool BF16>
 int launch_decode_noalloc(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
@@ -615,6 +667,62 @@ int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache, cons
     return bf16 ? launch_mq<128, true>(ATTN_MQ_ARGS) : launch_mq<128, false>(ATTN_MQ_ARGS);
   return bf16 ? launch_mq<64, true>(ATTN_MQ_ARGS) : launch_mq<64, false>(ATTN_MQ_ARGS);
 #undef ATTN_MQ_ARGS
+}
+
+int attn_indexer_score(const void* q, const void* kp, const float* w, const void* mask, float* score,
+                       int B, int T, int H, int P, int d, int dtype, attn_stream_t stream) {
+  if (!q || !kp || !w || !score) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0 || H <= 0 || P <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (H > 128 || (H & (H - 1)) != 0) return ATTN_ERR_UNSUPPORTED;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) != 0; };
+  if (misaligned(q, 16) || misaligned(kp, 16) || misaligned(w, 4) || misaligned(score, 4) ||
+      (mask && misaligned(mask, 2)))
+    return ATTN_ERR_INVALID_ARG;
+  const unsigned long long q_bytes = (unsigned long long)B * T * H * d * 2;
+  const unsigned long long k_bytes = (unsigned long long)B * P * d * 2;
+  const unsigned long long s_bytes = (unsigned long long)B * T * P * 4;
+  if ((unsigned long long)T * H * d * 2 >= (1ull << 40) || (unsigned long long)P * d * 2 >= (1ull << 40))
+    return ATTN_ERR_INVALID_ARG;
+  if (overlaps(score, s_bytes, q, q_bytes) || overlaps(score, s_bytes, kp, k_bytes) ||
+      overlaps(score, s_bytes, w, (size_t)B * T * H * 4) ||
+      (mask && overlaps(score, s_bytes, mask, (size_t)B * T * P * 2)))
+    return ATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_BF16;
+  if (d == 128)
+    return bf16 ? launch_indexer<128, true>(ds, q, kp, w, mask, score, B, T, H, P, st)
+                : launch_indexer<128, false>(ds, q, kp, w, mask, score, B, T, H, P, st);
+  return bf16 ? launch_indexer<64, true>(ds, q, kp, w, mask, score, B, T, H, P, st)
+              : launch_indexer<64, false>(ds, q, kp, w, mask, score, B, T, H, P, st);
+}
+
+int attn_topk(const float* score, int R, int P, int k, int* idx, attn_stream_t stream) {
+  if (!score || !idx) return ATTN_ERR_INVALID_ARG;
+  if (R <= 0 || P <= 0 || k <= 0 || k > kTopkMaxK) return ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) != 0; };
+  if (misaligned(score, 4) || misaligned(idx, 4)) return ATTN_ERR_INVALID_ARG;
+  if (overlaps(idx, (size_t)R * k * 4, score, (size_t)R * P * 4)) return ATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int kp2 = 1;
+  while (kp2 < k) kp2 <<= 1;
+  const bool cached = P <= kTopkCache;
+  const size_t smem = (size_t)(296 + 2 * kp2 + (cached ? P : 0)) * 4;
+  if (cached) {
+    if (int rc = ensure_smem_attr(ds, 20, attn_topk_kernel<true>, (int)((296 + 2 * kTopkMaxK + kTopkCache) * 4)))
+      return rc;
+    attn_topk_kernel<true><<<dim3(R), dim3(kTopkThreads), smem, st>>>(score, R, P, k, idx);
+  } else {
+    if (int rc = ensure_smem_attr(ds, 21, attn_topk_kernel<false>, (int)((296 + 2 * kTopkMaxK) * 4)))
+      return rc;
+    attn_topk_kernel<false><<<dim3(R), dim3(kTopkThreads), smem, st>>>(score, R, P, k, idx);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_get_status(attn_stream_t stream) {

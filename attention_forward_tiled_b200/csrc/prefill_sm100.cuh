@@ -194,9 +194,10 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
 // Every kExpEmuPeriod-th pair of softmax exponentials (d = 128; kExpEmuPeriodD64 at
 // d = 64) is evaluated with the FMA-pipe polynomial instead of the MUFU unit.  MUFU
 // delivers 4 exp2 per clock per SM sub-partition; the polynomial costs more issue slots
-// per result, so the best share is measured: every 8th pair at d = 128 (1 in 4 and 1 in 3
-// were slower), every 4th at d = 64.
-constexpr int kExpEmuPeriod = 8;
+// per result, so the best share is measured: every 16th pair at d = 128 (every 6th, 8th,
+// 12th and 24th were slower, none at all within 0.2 %), every 4th at d = 64 (every 3rd,
+// 6th and 8th slower).
+constexpr int kExpEmuPeriod = 16;
 constexpr int kExpEmuPeriodD64 = 4;
 template <int kPeriod>
 __device__ __forceinline__ constexpr bool emu_pair(int pair) {

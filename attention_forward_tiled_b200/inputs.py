@@ -44,6 +44,15 @@ PAGED_WORKLOADS = {
 }
 
 
+# The lightning-indexer workload: 4096 query tokens of 4 indexer heads (the head count the
+# llama.cpp report's CUDA kernel supports) against 4096 pooled keys, d 128, the unweighted
+# form (w = 1/sqrt(d)) with the bottom-right f16 pool mask; top-k keeps 512 per token.
+INDEXER_WORKLOADS = {
+    "indexer_h4": dict(B=1, T=4096, H=4, P=4096, d=128, dtype="f16", seed=8, weights="constant",
+                       masked=True, k=512),
+}
+
+
 def make_inputs(B, H, Nq, Nk, d, dtype="f16", seed=0, k_mult=1.0, **_):
     """Return CPU tensors (q, k, v) in [B, N, H, d] layout and the given dtype."""
     g = torch.Generator("cpu").manual_seed(int(seed))
@@ -95,3 +104,25 @@ def flops(B, H, Nq, Nk, d, causal, **_):
 def kv_bytes(B, H, Nk, d, dtype="f16", **_):
     """Bytes of K plus V (the decode metric's numerator)."""
     return 2 * B * Nk * H * d * torch.tensor([], dtype=DTYPES[dtype]).element_size()
+
+
+def make_indexer_inputs(B, T, H, P, d, dtype="f16", seed=0, weights="random", masked=True):
+    """Seeded lightning-indexer inputs (CPU tensors): q [B, T, H, d], kp [B, P, d] in the
+    dtype; w [B, T, H] float32 (randn, or 1/sqrt(d) everywhere for the unweighted form);
+    mask [B, T, P] float16 with 0 where pool entry p is visible to token t (p <= t + P - T,
+    the bottom-right rule) and -inf elsewhere, or None.  Draw order: q, kp, w."""
+    g = torch.Generator("cpu").manual_seed(int(seed))
+    q = torch.randn(B, T, H, d, generator=g, dtype=torch.float32)
+    kp = torch.randn(B, P, d, generator=g, dtype=torch.float32)
+    if weights == "random":
+        w = torch.randn(B, T, H, generator=g, dtype=torch.float32)
+    else:
+        w = torch.full((B, T, H), 1.0 / math.sqrt(d), dtype=torch.float32)
+    mask = None
+    if masked:
+        t = torch.arange(T).view(T, 1)
+        p = torch.arange(P).view(1, P)
+        mask = torch.where(p <= t + (P - T), 0.0, float("-inf")).to(torch.float16)
+        mask = mask.expand(B, T, P).contiguous()
+    dt = DTYPES[dtype]
+    return q.to(dt), kp.to(dt), w, mask

@@ -16,8 +16,8 @@ data-path collective): scaling is weak.  `--gpus N` means N ranks: started as on
 process, the script relaunches itself under torchrun with N ranks; started by a
 launcher with a different number of ranks, it exits with status 2.  `extra`
 carries the decode, causal8k, causal8000 and bf16_k3 workloads, the decode over a
-16-key-page cache and the 8-token (speculative) decode over the same cache on the
-tensor cores, each with its roofline.
+16-key-page cache, the 8-token (speculative) decode over the same cache on the
+tensor cores, and the lightning-indexer score and top-k, each with its roofline.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the method available here) on bounded samples of the same workload.
@@ -459,6 +459,60 @@ def measure_paged(name, K, W, world, device, peaks):
                        "l2": "K+V of 1074 MB per step vs 126 MB L2: no flush"}}
 
 
+def measure_indexer(name, K, W, world, device, peaks):
+    """Lightning-indexer score and top-k: bytes each kernel must move per call, per second."""
+    import torch
+
+    import attention_forward_tiled_b200 as attn
+    from attention_forward_tiled_b200.inputs import INDEXER_WORKLOADS, make_indexer_inputs
+
+    w = INDEXER_WORKLOADS[name]
+    B, T, H, P, d, k = w["B"], w["T"], w["H"], w["P"], w["d"], w["k"]
+    q, kp, wt, mask = (t.to(device) if t is not None else None for t in make_indexer_inputs(
+        B, T, H, P, d, dtype=w["dtype"], seed=w["seed"], weights=w["weights"], masked=w["masked"]))
+    score = torch.empty((B, T, P), dtype=torch.float32, device=device)
+    idx = torch.empty((B, T, k), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    res = {}
+    for kind in ("score", "topk"):
+        if kind == "score":
+            def step():
+                attn.indexer_score(q, kp, wt, mask, out=score, stream=stream)
+            nbytes = (q.numel() + kp.numel()) * q.element_size() + wt.numel() * 4 + score.numel() * 4 + \
+                (mask.numel() * 2 if mask is not None else 0)
+        else:
+            def step():
+                attn.topk(score, k, out=idx, stream=stream)
+            nbytes = score.numel() * 4 + idx.numel() * 4
+        for _ in range(W):
+            step()
+        torch.cuda.synchronize(device)
+        if attn.get_status(device=device) != 0:
+            raise RuntimeError("device status error during warm-up")
+        sampler = ClockSampler(device.index if device.index is not None else 0)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        sampler.start()
+        t_steps = time_gpu_steps(step, K, stream, None)
+        sampler.stop()
+        torch.cuda.synchronize(device)
+        barrier(world)
+        elapsed_ms = max_over_ranks(sum(t_steps), world)
+        achieved = nbytes / (statistics.mean(t_steps) * 1e-3) / 1e9
+        res[kind] = {"value": world * K * nbytes / (elapsed_ms * 1e-3) / 1e9, "unit": "GB/s",
+                     "ms_per_step": elapsed_ms / K,
+                     "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                                  "algorithmic_bytes_per_launch": nbytes},
+                     "clocks": sampler.summary(),
+                     "config": {"workload": name, "kernel": kind, "B": B, "T": T, "H": H, "P": P, "d": d,
+                                "k": k, "dtype": w["dtype"], "weights": w["weights"], "masked": w["masked"],
+                                "l2": "%.0f MB moved per call" % (nbytes / 1e6)}}
+    del q, kp, wt, mask, score, idx
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
 
@@ -504,6 +558,9 @@ def run_ours(args):
                            "config": workload_config(name, WORKLOADS[name])}
         extra["decode_paged16"] = measure_paged("decode_paged16", K, W, world, device, peaks)
         extra["spec8_paged16"] = measure_paged("spec8_paged16", K, W, world, device, peaks)
+        r = measure_indexer("indexer_h4", K, W, world, device, peaks)
+        extra["indexer_h4_score"] = r["score"]
+        extra["indexer_h4_topk"] = r["topk"]
     line = {
         "metric": METRIC,
         "value": main["value"],

@@ -224,6 +224,44 @@ ATTN_API int attn_fwd_paged(const void* q, const void* k_cache, const void* v_ca
                             attn_stream_t stream);
 
 /*
+ * attn_indexer_score -- lightning-indexer score on the tensor cores.
+ *
+ * The aispot.cmou.io report on llama.cpp release b11372 (entry "compute the
+ * indexer score with the lightning indexer"): each query token scores each
+ * pooled key by the rectified dot product of every indexer head with the key,
+ * weighted per head and summed over heads; keys have no head axis; an additive
+ * f16 pool mask follows:
+ *   score[b,t,p] = sum_h w[b,t,h] * max(0, q[b,t,h,:] . kp[b,p,:]) + mask[b,t,p]
+ * (the report's unweighted form is w = 1/sqrt(d) for every head).
+ *
+ *   q      [B, T, H, d]  dtype            (read)
+ *   kp     [B, P, d]     dtype            (read)
+ *   w      [B, T, H]     float32          (read)
+ *   mask   [B, T, P]     IEEE binary16 (0 or -inf), or NULL = no mask   (read)
+ *   score  [B, T, P]     float32          (written; must not overlap the inputs)
+ *   H a power of two <= 128; d in {64, 128}; alignment 16 bytes for q and kp,
+ *   4 for w and score, 2 for mask.  Products accumulate in fp32.
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA;
+ * asynchronous like attn_fwd.
+ */
+ATTN_API int attn_indexer_score(const void* q, const void* kp, const float* w, const void* mask,
+                                float* score, int B, int T, int H, int P, int d, int dtype,
+                                attn_stream_t stream);
+
+/*
+ * attn_topk -- positions of the k largest scores of each row.
+ *
+ * The selection the vLLM page "PR #45743 完整报告" (section "实现拆解") builds
+ * on: only the order of the indexer scores matters.  For each of R rows of P
+ * float32 scores, idx receives the positions of the k largest finite (or +inf)
+ * scores, largest first; equal scores go lowest position first; -inf and NaN
+ * are never chosen; slots past a row's chosen entries hold -1.
+ *   score [R, P] float32 (read), idx [R, k] int32 (written); 1 <= k <= 2048.
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG or ATTN_ERR_CUDA; asynchronous.
+ */
+ATTN_API int attn_topk(const float* score, int R, int P, int k, int* idx, attn_stream_t stream);
+
+/*
  * attn_get_status -- synchronises `stream`, then returns and clears the
  * current device's status word: ATTN_OK; ATTN_ERR_TIMEOUT if any kernel since
  * the last call gave up on a pipeline wait, or ATTN_ERR_RANGE if a bf16 prefill

@@ -1,0 +1,97 @@
+"""GPU parity of the lightning-indexer score (attn_indexer_score, tensor cores) and of
+the top-k selection (attn_topk) against the fp64 oracle.
+
+Scores: the GPU accumulates q . kp in fp32 from fp16/bf16 inputs that the oracle reads
+exactly, so each score may differ from the oracle by the fp32 rounding of the head
+products and of the weighted head sum; the bound used is 2^-14 times the sum of the
+magnitudes of the terms (sum_h |w_h| sum_c |q_hc kp_c|), about 16 times the worst-case
+fp32 accumulation error of 128 + H terms.  Masked entries must be exactly -inf.
+
+Top-k: an index result, compared bit for bit with the oracle run on the GPU's own fp32
+scores (the same precision decides the order on both sides).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_forward_tiled_b200 import get_status, indexer_score, topk
+from attention_forward_tiled_b200.inputs import make_indexer_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def score_bound(q, kp, w):
+    qa, ka, wa = q.double().abs(), kp.double().abs(), w.double().abs()
+    mag = torch.einsum("bthc,bpc->bthp", qa, ka)            # sum_c |q_hc kp_c|
+    return 2.0 ** -14 * torch.einsum("bth,bthp->btp", wa, mag).numpy() + 1e-30
+
+
+CASES = [
+    # (B, T, H, P, d, dtype, weights, masked)
+    (1, 64, 4, 1000, 128, "f16", "random", True),
+    (2, 33, 4, 257, 128, "bf16", "constant", True),
+    (1, 5, 64, 700, 128, "f16", "random", False),
+    (2, 130, 1, 384, 64, "f16", "random", True),
+    (1, 40, 16, 129, 64, "bf16", "random", True),
+    (1, 3, 128, 300, 128, "f16", "constant", False),
+]
+
+
+@pytest.mark.parametrize("B,T,H,P,d,dtype,weights,masked", CASES)
+def test_indexer_score_matches_oracle(B, T, H, P, d, dtype, weights, masked):
+    q, kp, w, mask = make_indexer_inputs(B, T, H, P, d, dtype=dtype, seed=T + P + H,
+                                         weights=weights, masked=masked)
+    out = indexer_score(q.cuda(), kp.cuda(), w.cuda(), mask.cuda() if mask is not None else None)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    ref = oracle.indexer_score(q, kp, w, mask)
+    got = out.double().cpu().numpy()
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isneginf(got), np.isneginf(ref)), "masked entries must be -inf"
+    err = np.abs(got[fin] - ref[fin])
+    bound = score_bound(q, kp, w)[fin]
+    assert (err <= bound).all(), f"score error {float((err - bound).max())} beyond the fp32 bound"
+    print(f"indexer B{B} T{T} H{H} P{P} d{d} {dtype}: max_abs={err.max():.2e} max_rel_to_bound="
+          f"{float((err / bound).max()):.3f}")
+    # the top-k of the GPU's scores, index for index
+    k = min(64, P)
+    idx = topk(out, k)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(got, k))
+
+
+def _rows_with_ties(R, P, seed):
+    g = torch.Generator("cpu").manual_seed(seed)
+    s = torch.randint(-20, 20, (R, P), generator=g).float() / 4.0   # many equal values
+    s[0, ::7] = float("-inf")
+    s[1, ::5] = float("nan")
+    s[2, 3:] = float("-inf")                                          # 3 finite entries only
+    s[3, :] = float("-inf")                                           # nothing to choose
+    s[4, 10] = float("inf")
+    s[5, :] = -0.0
+    s[5, 1::2] = 0.0                                                  # +0 and -0 tie
+    return s
+
+
+@pytest.mark.parametrize("R,P,k", [(8, 1000, 64), (8, 129, 200), (6, 60000, 2048), (6, 50000, 1),
+                                   (7, 4096, 2048), (9, 513, 513)])
+def test_topk_matches_oracle(R, P, k):
+    s = _rows_with_ties(R, P, seed=R * P + k)
+    idx = topk(s.cuda(), k)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(s.double().numpy(), k))
+
+
+def test_topk_distinct_scores_large_rows():
+    """Random distinct scores: the chosen set is the k largest, in order (rows read from
+    global memory on every pass when they exceed the shared-memory cache)."""
+    g = torch.Generator("cpu").manual_seed(11)
+    s = torch.randn(4, 70000, generator=g)
+    idx = topk(s.cuda(), 300)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(s.double().numpy(), 300))

@@ -19,7 +19,8 @@ from attention_forward_tiled_b200 import build as abuild
 
 THREADS = {"attn_prefill_kernel": 384, "attn_decode_partial_kernel": 160,
            "attn_decode_combine_kernel": 128, "attn_mq_partial_kernel": 192,
-           "attn_mq_combine_kernel": 128}
+           "attn_mq_combine_kernel": 128, "attn_indexer_score_kernel": 192,
+           "attn_topk_kernel": 512}
 # bytes of spill stores / loads per prefill instantiation (head_dim, bf16) at this version
 PREFILL_SPILL_CEILING = {(64, False): (112, 168), (64, True): (152, 300),
                          (128, False): (8, 8), (128, True): (16, 16)}
@@ -75,6 +76,8 @@ def test_every_kernel_is_reported(ptxas_report):
     assert kinds.count("attn_decode_combine_kernel") == 4
     assert kinds.count("attn_mq_partial_kernel") == 4
     assert kinds.count("attn_mq_combine_kernel") == 4
+    assert kinds.count("attn_indexer_score_kernel") == 4
+    assert kinds.count("attn_topk_kernel") == 2
     assert all(kinds)
 
 
@@ -84,7 +87,7 @@ def test_registers_fit_the_launch(ptxas_report):
         assert info["registers"] * threads <= 65536, (name, info)
 
 
-def test_decode_kernels_do_not_spill(ptxas_report):
+def test_non_prefill_kernels_do_not_spill(ptxas_report):
     for name, info in ptxas_report.items():
         if kernel_kind(name) != "attn_prefill_kernel":
             assert info["spill_stores"] == 0 and info["spill_loads"] == 0, (name, info)
