@@ -31,6 +31,7 @@ SIGNATURES = {
                                    _i, _vp]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                             _i, _i, _vp]),
+    "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_indexer_score": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "attn_topk": (_i, [_vp, _i, _i, _i, _vp, _vp]),
     "attn_get_status": (_i, [_vp]),
@@ -260,6 +261,35 @@ def attn_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, causal=False, sca
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_paged")
     return out, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal=False, scale=None, stream=None, dq=None, dk=None, dv=None):
+    """Gradients (dq, dk, dv) of attn_fwd for the upstream gradient dout, from the
+    forward's inputs, its output o and its lse (all CUDA tensors, [B, N, H, d] layout)."""
+    import torch
+    lib = load_library()
+    B, H, Nq, Nk, d = _check(q, k, v)
+    for name, t in (("o", o), ("dout", dout)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA tensor")
+    _check_buffer("o", o, q.shape, q.dtype, q.device)
+    _check_buffer("dout", dout, q.shape, q.dtype, q.device)
+    _check_buffer("lse", lse, (B, H, Nq), torch.float32, q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_buffer("dq", dq, q.shape, q.dtype, q.device)
+    _check_buffer("dk", dk, k.shape, k.dtype, q.device)
+    _check_buffer("dv", dv, v.shape, v.dtype, q.device)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    with torch.cuda.device(q.device):
+        rc = lib.attn_bwd(ptr(q), ptr(k), ptr(v), ptr(o), ptr(dout), ptr(lse), ptr(dq), ptr(dk), ptr(dv),
+                          B, H, Nq, Nk, d, int(bool(causal)), scale, _dtype_code(q.dtype),
+                          _stream_ptr(stream, q.device))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def indexer_score(q, kp, w, mask=None, out=None, stream=None):

@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "backward_sm100.cuh"
 #include "decode_mq_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "indexer_sm100.cuh"
@@ -51,7 +52,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int* status_ptr = nullptr;
-  bool attr_set[24] = {};  // per kernel instantiation: max dynamic shared memory raised
+  bool attr_set[28] = {};  // per kernel instantiation: max dynamic shared memory raised
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -503,6 +504,66 @@ int launch_indexer(DeviceState* ds, const void* q, const void* kp, const float* 
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Backward: D = rowsum(dO o O) and a zeroed fp32 dQ accumulator, the tiled gradient
+// kernel, then dQ = scale * accumulator cast to the input type.  Workspace taken
+// stream-ordered from the default pool and returned on the same stream.
+template <int D, bool BF16>
+int launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
+               const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int H,
+               int Nq, int Nk, int causal, float scale, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  auto kernel = attn_bwd_kernel<D, BF16>;
+  const int slot = 24 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  BwdParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  if (int rc = encode_bnhd(&p.tm_q, q, B, Nq, H, D, dtype, 64)) return rc;
+  if (int rc = encode_bnhd(&p.tm_do, dout, B, Nq, H, D, dtype, 64)) return rc;
+  if (int rc = encode_bnhd(&p.tm_k, k, B, Nk, H, D, dtype)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v, B, Nk, H, D, dtype)) return rc;
+  const long long rows = (long long)B * Nq * H;
+  const size_t dsum_bytes = ((size_t)rows * 4 + 255) / 256 * 256;
+  const size_t ws_bytes = dsum_bytes + (size_t)rows * D * 4;
+  uint8_t* ws = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&ws), ws_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  float* dsum = reinterpret_cast<float*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(ws + dsum_bytes);
+  p.lse = lse;
+  p.dsum = dsum;
+  p.dq_acc = dq_acc;
+  p.dk = dk;
+  p.dv = dv;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.causal = causal;
+  p.n_ktiles = (Nk + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  const long long ctas = (long long)B * H * p.n_ktiles;
+  int rc = ATTN_OK;
+  if (ctas >= (1LL << 31) || (rows + 3) / 4 >= (1LL << 31)) rc = ATTN_ERR_INVALID_ARG;
+  if (rc == ATTN_OK) {
+    attn_bwd_pre_kernel<D, BF16><<<dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream>>>(
+        o, dout, dsum, dq_acc, B, H, Nq);
+    if (cudaGetLastError() != cudaSuccess) rc = ATTN_ERR_CUDA;
+  }
+  if (rc == ATTN_OK) {
+    kernel<<<dim3((unsigned)ctas), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) rc = ATTN_ERR_CUDA;
+  }
+  if (rc == ATTN_OK) {
+    const long long n2 = rows * D / 2;
+    attn_bwd_dq_kernel<BF16><<<dim3((unsigned)((n2 + 255) / 256)), dim3(256), 0, stream>>>(dq_acc, dq, n2, scale);
+    if (cudaGetLastError() != cudaSuccess) rc = ATTN_ERR_CUDA;
+  }
+  if (cudaFreeAsync(ws, stream) != cudaSuccess) rc = ATTN_ERR_CUDA;
+  return rc;
+}
+
 // Same kernels as launch_decode, with the partials in g_noalloc_scratch: no allocation.
 template <int D, bool BF16>
 int launch_decode_noalloc(DeviceState* ds, const void* q, const void* k, const void* v, void* out,
@@ -667,6 +728,38 @@ int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache, cons
     return bf16 ? launch_mq<128, true>(ATTN_MQ_ARGS) : launch_mq<128, false>(ATTN_MQ_ARGS);
   return bf16 ? launch_mq<64, true>(ATTN_MQ_ARGS) : launch_mq<64, false>(ATTN_MQ_ARGS);
 #undef ATTN_MQ_ARGS
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
+             int causal, float scale, int dtype, attn_stream_t stream) {
+  if (!lse || !o || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  // q, k, v, o (as the forward's output) and the forward's own checks
+  if (int rc = validate(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dtype)) return rc;
+  auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) != 0; };
+  if (misaligned(dout, 16) || misaligned(dq, 16) || misaligned(dk, 16) || misaligned(dv, 16))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t row_bytes = (size_t)H * d * 2;
+  const size_t q_bytes = (size_t)B * Nq * row_bytes, kv_bytes = (size_t)B * Nk * row_bytes;
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, (size_t)B * H * Nq * 4};
+  void* outs[3] = {dq, dk, dv};
+  const size_t out_bytes[3] = {q_bytes, kv_bytes, kv_bytes};
+  for (int a = 0; a < 3; ++a) {
+    for (int c = 0; c < 6; ++c)
+      if (overlaps(outs[a], out_bytes[a], ins[c], in_bytes[c])) return ATTN_ERR_INVALID_ARG;
+    for (int c = a + 1; c < 3; ++c)
+      if (overlaps(outs[a], out_bytes[a], outs[c], out_bytes[c])) return ATTN_ERR_INVALID_ARG;
+  }
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_BF16;
+#define ATTN_BWD_ARGS ds, q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nk, causal, scale, st
+  if (d == 128)
+    return bf16 ? launch_bwd<128, true>(ATTN_BWD_ARGS) : launch_bwd<128, false>(ATTN_BWD_ARGS);
+  return bf16 ? launch_bwd<64, true>(ATTN_BWD_ARGS) : launch_bwd<64, false>(ATTN_BWD_ARGS);
+#undef ATTN_BWD_ARGS
 }
 
 int attn_indexer_score(const void* q, const void* kp, const float* w, const void* mask, float* score,

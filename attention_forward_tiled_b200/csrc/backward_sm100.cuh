@@ -1,0 +1,417 @@
+// backward_sm100.cuh -- gradients of the tiled attention forward (sm_100a).
+//
+// The step after the forward: the FlashAttention/ops-transformer article notes
+// (section "传统注意力的显存陷阱") that eager attention keeps the N x N matrix for
+// backpropagation; here, as in the forward, it is recomputed tile by tile from Q, K
+// and the row log-sum-exp the forward wrote, and never stored:
+//   P = exp(scale * Q K^T - lse)            (masked entries 0)
+//   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - D),  D_i = sum_t dO_it O_it
+//   dQ = scale * dS K,   dK = scale * dS^T Q
+//
+// One CTA per (b, h, 128-key tile): K_j and V_j stay in shared memory and the CTA
+// walks the 64-query tiles that see them.  Per query tile, on the tensor cores
+// (thread = key of the tile for the elementwise part):
+//   S^T  = K Q^T    and  dP^T = V dO^T    (shared-memory operands, TMEM accumulators)
+//   P^T, dS^T -> fp16/bf16 into the consumed TMEM columns (and dS^T into shared memory)
+//   dV  += P^T dO   and  dK  += dS^T Q    (A from TMEM, B = dO / Q read MN-major)
+//   dQ^T = K^T dS^T                       (A = K read MN-major, B = dS^T in shared memory)
+// dQ^T (lane = head-dim element, column = query) is added to an fp32 accumulator in
+// global memory with coalesced atomic adds (other key tiles add to the same rows);
+// dV and dK are written once at the end.  Roles (192 threads): warps 0-3 elementwise
+// and epilogues, warp 4 TMA producer, warp 5 MMA issuer.
+//
+// TMEM columns: S^T [0,64) (P^T packed in [0,32)), dP^T [64,128) (dS^T packed in
+// [64,96)), dQ^T [128,192), dV [256,256+D), dK [384,384+D).
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace attn_b200 {
+
+struct BwdParams {
+  CUtensorMap tm_q;   // q  [B, Nq, H, D] as 4-D (D, H, Nq, B), box (64, 1, 64, 1), 128B swizzle
+  CUtensorMap tm_do;  // dO [B, Nq, H, D], same
+  CUtensorMap tm_k;   // k  [B, Nk, H, D], box (64, 1, 128, 1)
+  CUtensorMap tm_v;   // v  [B, Nk, H, D], same
+  const float* lse;   // [B, H, Nq] natural log (the forward's)
+  const float* dsum;  // [B, H, Nq]: D_i = sum_t dO_it O_it
+  float* dq_acc;      // [B, Nq, H, D] fp32, zeroed before the launch
+  void* dk;           // [B, Nk, H, D]
+  void* dv;           // [B, Nk, H, D]
+  int* status;
+  int B, H, Nq, Nk, causal;
+  int n_ktiles;       // ceil(Nk / 128)
+  float scale;
+  float scale_log2;   // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kKBox = 128 * 128;                  // 128 rows x 64 elements x 2 bytes
+  static constexpr int kQBox = 64 * 128;                   // 64 rows x 64 elements x 2 bytes
+  static constexpr int kKTile = kBoxes * kKBox;            // K or V tile
+  static constexpr int kQTile = kBoxes * kQBox;            // Q or dO tile
+  static constexpr int kStages = 2;                        // Q + dO stages
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kKTile;
+  static constexpr int kOffQ = 2 * kKTile;                 // [stage]: Q tile then dO tile
+  static constexpr int kStageBytes = 2 * kQTile;
+  static constexpr int kOffDS = kOffQ + kStages * kStageBytes;  // dS^T [128 keys][64 queries] fp16
+  static constexpr int kDSBytes = 128 * 128;
+  static constexpr int kOffRow = kOffDS + kDSBytes;        // per-query lse2 and D, [2][2][64] fp32
+  static constexpr int kOffBar = kOffRow + 2 * 2 * 64 * 4;
+  static constexpr int kBarKV = 0;
+  static constexpr int kBarQFull = 1;                      // [2]
+  static constexpr int kBarQEmpty = 3;                     // [2]
+  static constexpr int kBarSFull = 5;                      // S^T and dP^T landed
+  static constexpr int kBarPDone = 6;                      // P^T, dS^T written (4 warps)
+  static constexpr int kBarDQFull = 7;                     // dQ^T landed
+  static constexpr int kBarDQFree = 8;                     // dQ^T read (4 warps)
+  static constexpr int kBarMmaDone = 9;
+  static constexpr int kNumBars = 10;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr int kThreads = 192;
+  static constexpr int kProducerWarp = 4;
+  static constexpr int kMmaWarp = 5;
+  static constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 128, kColDV = 256, kColDK = 384;
+  static_assert(kOffQ % 1024 == 0 && kOffDS % 1024 == 0 && kQTile % 1024 == 0, "swizzle atoms");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+// First 64-query tile that sees key tile j (keys [128 j, 128 j + 128)): under the causal
+// flag query i sees key k iff k <= i + Nk - Nq.
+__device__ __forceinline__ int bwd_first_qtile(const BwdParams& p, int j) {
+  if (!p.causal) return 0;
+  const long long q_min = (long long)j * 128 - ((long long)p.Nk - p.Nq);
+  return q_min <= 0 ? 0 : (int)(q_min / 64);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
+  // CTA -> (b, h, key tile); key tile 0 (seen by the most queries under the causal flag) first
+  const int j = blockIdx.x % p.n_ktiles;
+  const int bh = blockIdx.x / p.n_ktiles;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int qt0 = bwd_first_qtile(p, j);
+  const int nqt = max(0, (p.Nq + 63) / 64 - qt0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::kBarKV), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(C::kBarQFull + i), 1);
+      mbar_init(BAR(C::kBarQEmpty + i), 1);
+    }
+    mbar_init(BAR(C::kBarSFull), 1);
+    mbar_init(BAR(C::kBarPDone), 4);
+    mbar_init(BAR(C::kBarDQFull), 1);
+    mbar_init(BAR(C::kBarDQFree), 4);
+    mbar_init(BAR(C::kBarMmaDone), 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::kProducerWarp) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      tma_prefetch_map(&p.tm_q);
+      tma_prefetch_map(&p.tm_do);
+      tma_prefetch_map(&p.tm_k);
+      tma_prefetch_map(&p.tm_v);
+    }
+    mbar_arrive_expect_tx_w(BAR(C::kBarKV), 2 * C::kKTile);
+    for (int bx = 0; bx < C::kBoxes; ++bx) {
+      tma_load_4d_w(sbase + C::kOffK + bx * C::kKBox, &p.tm_k, BAR(C::kBarKV), bx * 64, h, j * 128, b);
+      tma_load_4d_w(sbase + C::kOffV + bx * C::kKBox, &p.tm_v, BAR(C::kBarKV), bx * 64, h, j * 128, b);
+    }
+    int i = 0;
+    for (; i < nqt; ++i) {
+      const int st = i & 1;
+      if (i >= 2) mbar_wait(BAR(C::kBarQEmpty + st), ((i >> 1) - 1) & 1, wctx);
+      __syncwarp();
+      if (warp_flag(abort_flag)) break;
+      const uint32_t dst = sbase + C::kOffQ + st * C::kStageBytes;
+      const int q0 = (qt0 + i) * 64;
+      mbar_arrive_expect_tx_w(BAR(C::kBarQFull + st), C::kStageBytes);
+      for (int bx = 0; bx < C::kBoxes; ++bx) {
+        tma_load_4d_w(dst + bx * C::kQBox, &p.tm_q, BAR(C::kBarQFull + st), bx * 64, h, q0, b);
+        tma_load_4d_w(dst + C::kQTile + bx * C::kQBox, &p.tm_do, BAR(C::kBarQFull + st), bx * 64, h, q0, b);
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // let every copy this warp started land before the CTA can exit
+      mbar_wait_drain(BAR(C::kBarKV), 0, p.timeout_ns);
+      for (int t = max(0, i - 2); t < i; ++t)
+        mbar_wait_drain(BAR(C::kBarQFull + (t & 1)), (t >> 1) & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == C::kMmaWarp) {
+    // ======================= tcgen05 MMA issuer =======================
+    // S^T = K Q^T, dP^T = V dO^T: M = 128 keys, N = 64 queries, both operands K-major.
+    constexpr uint32_t idesc_s = make_idesc_f16(128, 64, BF16, false, false);
+    // dV += P^T dO, dK += dS^T Q: A (keys x queries) from TMEM, B = dO / Q read MN-major.
+    constexpr uint32_t idesc_kv = make_idesc_f16(128, D, BF16, true, false);
+    // dQ^T = K^T dS^T: M = 128 (head dim; at D = 64 the 64 rows are read twice), N = 64
+    // queries, K = 128 keys; A = K tile read MN-major, B = dS^T in shared memory MN-major.
+    constexpr uint32_t idesc_q = make_idesc_f16(128, 64, BF16, true, true);
+    constexpr uint32_t kLboK = (D == 128) ? C::kKBox : 0;
+    const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV, sDS = sbase + C::kOffDS;
+    mbar_wait(BAR(C::kBarKV), 0, wctx);
+    for (int i = 0; i < nqt; ++i) {
+      const int st = i & 1;
+      const uint32_t sQ = sbase + C::kOffQ + st * C::kStageBytes, sDO = sQ + C::kQTile;
+      mbar_wait(BAR(C::kBarQFull + st), (i >> 1) & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      if (!warp_flag(abort_flag)) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // 16 head-dim elements per k-step
+          const uint32_t ka = (kk >> 2) * C::kKBox + (kk & 3) * 32;
+          const uint32_t kb = (kk >> 2) * C::kQBox + (kk & 3) * 32;
+          mma_f16_ss_w(tmem + C::kColS, make_sdesc_sw128(sK + ka, 16, 1024),
+                       make_sdesc_sw128(sQ + kb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          mma_f16_ss_w(tmem + C::kColDP, make_sdesc_sw128(sV + ka, 16, 1024),
+                       make_sdesc_sw128(sDO + kb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit_w(BAR(C::kBarSFull));
+      }
+      mbar_wait(BAR(C::kBarPDone), i & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      if (!warp_flag(abort_flag)) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per k-step: 8 packed TMEM columns
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          mma_f16_ts_w(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                       make_sdesc_sw128(sDO + kk * 2048, C::kQBox, 1024), idesc_kv, acc);
+          mma_f16_ts_w(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+                       make_sdesc_sw128(sQ + kk * 2048, C::kQBox, 1024), idesc_kv, acc);
+        }
+      }
+      if (i > 0) mbar_wait(BAR(C::kBarDQFree), (i - 1) & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      if (!warp_flag(abort_flag)) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 16 keys per k-step
+          mma_f16_ss_w(tmem + C::kColDQ, make_sdesc_sw128(sK + kk * 2048, kLboK, 1024),
+                       make_sdesc_sw128(sDS + kk * 2048, 16, 1024), idesc_q, kk > 0 ? 1u : 0u);
+        }
+        tc_commit_w(BAR(C::kBarDQFull));
+        tc_commit_w(BAR(C::kBarQEmpty + st));
+      }
+    }
+    // every MMA (and every commit arrive) has landed before TMEM is released
+    tc_commit_w(BAR(C::kBarMmaDone));
+    mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+    __syncwarp();
+  } else {
+    // ======================= elementwise warps 0-3 (thread = key of the tile) ==========
+    const int r = threadIdx.x;  // key of the tile (S^T, dP^T, dV, dK lanes); head-dim element of dQ^T
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int key = j * 128 + r;
+    const long long diag = (long long)p.Nk - p.Nq;
+    float* rowbuf = reinterpret_cast<float*>(smem + C::kOffRow);  // [2][2][64]: lse2, D
+    uint8_t* ds_row = smem + C::kOffDS + r * 128;                  // dS^T row of this key
+    for (int i = 0; i < nqt; ++i) {
+      const int q0 = (qt0 + i) * 64;
+      float* lse2 = rowbuf + (i & 1) * 128;
+      float* dsm = lse2 + 64;
+      if (r < 64) {
+        const int q = q0 + r;
+        const long long o = ((long long)b * p.H + h) * p.Nq + q;
+        lse2[r] = q < p.Nq ? __ldg(p.lse + o) * 1.4426950408889634f : 0.f;
+        dsm[r] = q < p.Nq ? __ldg(p.dsum + o) : 0.f;
+      }
+      named_bar_sync(1, 128);
+      mbar_wait(BAR(C::kBarSFull), i & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      uint32_t s[2][32], dp[2][32];
+      tmem_ld32(tmem + lane_base + C::kColS, s[0]);
+      tmem_ld32(tmem + lane_base + C::kColS + 32, s[1]);
+      tmem_ld32(tmem + lane_base + C::kColDP, dp[0]);
+      tmem_ld32(tmem + lane_base + C::kColDP + 32, dp[1]);
+      tmem_ld_wait();
+      reg_order_after_wait(s[0]);
+      reg_order_after_wait(s[1]);
+      reg_order_after_wait(dp[0]);
+      reg_order_after_wait(dp[1]);
+      // query q0 + c sees this key iff key < Nk, q0 + c < Nq and (causal) key <= q0 + c + Nk - Nq
+      uint32_t pk[2][16], dk2[2][16];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float pv[2], dv2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = c + e;
+          const int q = q0 + col;
+          const bool ok = key < p.Nk && q < p.Nq && (!p.causal || (long long)key <= q + diag);
+          const float x = __uint_as_float(s[col >> 5][col & 31]) * p.scale_log2 - lse2[col];
+          const float pr = ok ? ex2_approx(x) : 0.f;
+          pv[e] = pr;
+          dv2[e] = pr * (__uint_as_float(dp[col >> 5][col & 31]) - dsm[col]);
+        }
+        pk[c >> 5][(c & 31) >> 1] = pack2<BF16>(pv[0], pv[1]);
+        dk2[c >> 5][(c & 31) >> 1] = pack2<BF16>(dv2[0], dv2[1]);
+      }
+      // P^T and dS^T (packed pairs) into the consumed S^T / dP^T columns
+      tmem_st16(tmem + lane_base + C::kColS, pk[0]);
+      tmem_st16(tmem + lane_base + C::kColS + 16, pk[1]);
+      tmem_st16(tmem + lane_base + C::kColDP, dk2[0]);
+      tmem_st16(tmem + lane_base + C::kColDP + 16, dk2[1]);
+      // dS^T row (64 queries, 128 bytes) into shared memory, 128-byte swizzle (MN-major B)
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const uint4 w = make_uint4(dk2[cc >> 2][(cc & 3) * 4 + 0], dk2[cc >> 2][(cc & 3) * 4 + 1],
+                                   dk2[cc >> 2][(cc & 3) * 4 + 2], dk2[cc >> 2][(cc & 3) * 4 + 3]);
+        *reinterpret_cast<uint4*>(ds_row + ((cc ^ (r & 7)) << 4)) = w;
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::kBarPDone));
+
+      // dQ^T of this tile: lane = head-dim element, 64 query columns -> fp32 accumulator
+      mbar_wait(BAR(C::kBarDQFull), i & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      uint32_t dq[2][32];
+      tmem_ld32(tmem + lane_base + C::kColDQ, dq[0]);
+      tmem_ld32(tmem + lane_base + C::kColDQ + 32, dq[1]);
+      tmem_ld_wait();
+      reg_order_after_wait(dq[0]);
+      reg_order_after_wait(dq[1]);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::kBarDQFree));
+      if (r < D && !*abort_flag) {
+        float* dst = p.dq_acc + (((long long)b * p.Nq + q0) * p.H + h) * D + r;
+        const long long qstride = (long long)p.H * D;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (q0 + c < p.Nq) atomicAdd(dst + c * qstride, __uint_as_float(dq[c >> 5][c & 31]));
+      }
+    }
+
+    // ---- epilogue: dV and scale * dK (lane = key) -> 16-bit -> global.  The last tile's
+    // dQ^T commit covered every earlier product, so dV and dK are final here.  The TMEM
+    // loads are warp-collective: every lane takes part, and only rows of keys below Nk
+    // are stored (the last key tile may be partial).
+    const bool key_row = key < p.Nk;
+    const long long row = (((long long)b * p.Nk + (key_row ? key : 0)) * p.H + h) * D;
+    uint4* dvrow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dv) + row * 2);
+    uint4* dkrow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dk) + row * 2);
+    if (nqt == 0) {  // no query sees this key tile
+      if (key_row) {
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          dvrow[c] = make_uint4(0u, 0u, 0u, 0u);
+          dkrow[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    } else {
+      tc_fence_after_sync();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32], k2[32];
+        tmem_ld32(tmem + lane_base + C::kColDV + c * 32, a);
+        tmem_ld32(tmem + lane_base + C::kColDK + c * 32, k2);
+        tmem_ld_wait();
+        reg_order_after_wait(a);
+        reg_order_after_wait(k2);
+        if (!key_row) continue;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 wv, wk;
+          wv.x = pack2<BF16>(__uint_as_float(a[q4 * 8 + 0]), __uint_as_float(a[q4 * 8 + 1]));
+          wv.y = pack2<BF16>(__uint_as_float(a[q4 * 8 + 2]), __uint_as_float(a[q4 * 8 + 3]));
+          wv.z = pack2<BF16>(__uint_as_float(a[q4 * 8 + 4]), __uint_as_float(a[q4 * 8 + 5]));
+          wv.w = pack2<BF16>(__uint_as_float(a[q4 * 8 + 6]), __uint_as_float(a[q4 * 8 + 7]));
+          wk.x = pack2<BF16>(__uint_as_float(k2[q4 * 8 + 0]) * p.scale, __uint_as_float(k2[q4 * 8 + 1]) * p.scale);
+          wk.y = pack2<BF16>(__uint_as_float(k2[q4 * 8 + 2]) * p.scale, __uint_as_float(k2[q4 * 8 + 3]) * p.scale);
+          wk.z = pack2<BF16>(__uint_as_float(k2[q4 * 8 + 4]) * p.scale, __uint_as_float(k2[q4 * 8 + 5]) * p.scale);
+          wk.w = pack2<BF16>(__uint_as_float(k2[q4 * 8 + 6]) * p.scale, __uint_as_float(k2[q4 * 8 + 7]) * p.scale);
+          dvrow[c * 4 + q4] = wv;
+          dkrow[c * 4 + q4] = wk;
+        }
+      }
+    }
+  }
+
+  // ---- teardown: every role is done with TMEM
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D_i = sum_t dO_it O_it in fp32 (one warp per (b, i, h) row) and zeroed dQ accumulator rows.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+    attn_bwd_pre_kernel(const void* __restrict__ o, const void* __restrict__ dout,
+                        float* __restrict__ dsum, float* __restrict__ dq_acc, int B, int H, int Nq) {
+  constexpr int E = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 4 + warp;  // (b * Nq + i) * H + h
+  if (row >= (long long)B * Nq * H) return;
+  const int h = (int)(row % H);
+  const long long bi = row / H;
+  const int i = (int)(bi % Nq), b = (int)(bi / Nq);
+  const uint8_t* orow = static_cast<const uint8_t*>(o) + row * D * 2 + lane * E * 2;
+  const uint8_t* grow = static_cast<const uint8_t*>(dout) + row * D * 2 + lane * E * 2;
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) {
+    const float2 a = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(orow + e * 2));
+    const float2 g = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(grow + e * 2));
+    acc = fmaf(a.x, g.x, fmaf(a.y, g.y, acc));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) dsum[((long long)b * H + h) * Nq + i] = acc;
+  float* z = dq_acc + row * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) z[e] = 0.f;
+}
+
+// dQ = scale * accumulated dS K, cast to the input type (two elements per thread).
+template <bool BF16>
+__global__ void __launch_bounds__(256)
+    attn_bwd_dq_kernel(const float* __restrict__ dq_acc, void* __restrict__ dq, long long n2, float scale) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n2) return;
+  const float2 a = reinterpret_cast<const float2*>(dq_acc)[t];
+  reinterpret_cast<uint32_t*>(dq)[t] = pack2<BF16>(a.x * scale, a.y * scale);
+}
+
+}  // namespace attn_b200

@@ -50,11 +50,12 @@ struct IndexerCfg {
   static constexpr int kBoxBytes = 128 * 128;             // 128 rows x 64 elements x 2 bytes
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;   // 128 rows x D
-  static constexpr int kQStages = 4;
+  static constexpr int kQStages = 2;
   static constexpr int kOffK = 0;                                  // key tiles [2]
   static constexpr int kOffQ = 2 * kTileBytes;                     // query tiles [kQStages]
   static constexpr int kOffW = kOffQ + kQStages * kTileBytes;     // head weights [2][128] fp32
-  static constexpr int kOffBar = kOffW + 2 * 128 * 4;
+  static constexpr int kOffM = kOffW + 2 * 128 * 4;                // pool mask [2][128 tokens][128 keys] f16
+  static constexpr int kOffBar = kOffM + 2 * 128 * 128 * 2;
   static constexpr int kBarKFull = 0;                     // [2]
   static constexpr int kBarKEmpty = 2;                    // [2]
   static constexpr int kBarQFull = 4;                     // [kQStages]
@@ -217,27 +218,53 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
     __syncwarp();
   } else {
     // ======================= epilogue warps 0-3 (thread = pooled key) ===========
+    // The head weights and pool mask of item g + 1 are loaded into shared memory while item
+    // g's product runs (plain loads: the mask rows of arbitrary length P need not meet any
+    // copy-engine alignment), so no global load sits between the score stores.
     const int r = threadIdx.x;  // key of the tile
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int lg_h = p.lg_h, tpt = p.tok_per_tile;
-    float* wbuf = reinterpret_cast<float*>(smem + C::kOffW);  // [2][128]: the item's head weights
+    float* wbuf = reinterpret_cast<float*>(smem + C::kOffW);        // [2][128]
+    uint16_t* mbuf = reinterpret_cast<uint16_t*>(smem + C::kOffM);  // [2][128][128]
+    auto prefetch = [&](int item, int buf) {
+      const IndexerItem it = indexer_item(p, item);
+      const int t0 = it.tt * tpt;
+      const long long row_bt = (long long)it.b * p.T;
+      {  // weight of column r: w[b, t0 + r / H, r % H]
+        const int t = t0 + (r >> lg_h);
+        wbuf[buf * 128 + r] = t < p.T ? __ldg(p.w + (row_bt + t0) * (1 << lg_h) + r) : 0.f;
+      }
+      if (p.mask != nullptr) {
+        const int key = it.pt * 128 + r;
+        uint16_t* mb = mbuf + buf * 128 * 128 + r;
+        for (int c0 = 0; c0 < tpt; c0 += 32) {  // 32 independent loads in flight, then the stores
+          uint16_t v[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int t = t0 + c0 + u;
+            v[u] = (c0 + u < tpt && t < p.T && key < p.P) ? __ldg(p.mask + (row_bt + t) * p.P + key) : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            if (c0 + u < tpt) mb[(c0 + u) * 128] = v[u];
+        }
+      }
+    };
+    if (item0 < item1) prefetch(item0, 0);
+    named_bar_sync(1, 128);
     int g = 0;
     for (int item = item0; item < item1; ++item, ++g) {
       const IndexerItem it = indexer_item(p, item);
       const int ab = g & 1;
+      if (item + 1 < item1) prefetch(item + 1, ab ^ 1);
       const int t0 = it.tt * tpt;
       const long long row_bt = (long long)it.b * p.T;
-      // weights of the tile's (token, head) pairs, column order: w[b, t0 + c / H, c % H]
-      {
-        const int t = t0 + (r >> lg_h);
-        wbuf[ab * 128 + r] = t < p.T ? __ldg(p.w + (row_bt + t0) * (1 << lg_h) + r) : 0.f;
-      }
-      named_bar_sync(1, 128);
       mbar_wait(BAR(C::kBarAccFull + ab), (g >> 1) & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
       const int key = it.pt * 128 + r;
       const float* wb = wbuf + ab * 128;
+      const uint16_t* mb = mbuf + ab * 128 * 128 + r;
       float acc = 0.f;
       // 32 columns at a time: column c = t_local * H + h
 #pragma unroll 1
@@ -251,12 +278,12 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
           const int col = c0 + c;
           acc = fmaf(wb[col], fmaxf(__uint_as_float(s[c]), 0.f), acc);
           if (((col + 1) & ((1 << lg_h) - 1)) == 0) {  // last head of a token: its score is complete
-            const int t = t0 + (col >> lg_h);
+            const int tl = col >> lg_h;
+            const int t = t0 + tl;
             if (t < p.T && key < p.P) {
-              const long long o = (row_bt + t) * p.P + key;
               float v = acc;
-              if (p.mask != nullptr) v += __half2float(__ushort_as_half(__ldg(p.mask + o)));
-              p.score[o] = v;
+              if (p.mask != nullptr) v += __half2float(__ushort_as_half(mb[tl * 128]));
+              p.score[(row_bt + t) * p.P + key] = v;
             }
             acc = 0.f;
           }
@@ -265,6 +292,9 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarAccFree + ab));
+      // every thread is done with buffer ab, and buffer ab ^ 1 is complete, before the next
+      // item reads ab ^ 1 and prefetches into ab
+      named_bar_sync(1, 128);
     }
   }
 
@@ -354,19 +384,41 @@ __global__ void __launch_bounds__(kTopkThreads)
       if (hit && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, sel = -1;
-      for (int dgt = 255; dgt >= 0; --dgt) {
-        const int c = (int)hist[dgt];
-        if (cum + c >= remaining) {
-          sel = dgt;
-          break;
-        }
-        cum += c;
+    if (tid < 32) {
+      // warp 0 finds the digit where the count from the top reaches `remaining`: lane l
+      // holds digits 255 - 8 l ... 248 - 8 l, a shuffle scan gives the count above them
+      const int lane_t = tid;
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        cnt[u] = (int)hist[255 - 8 * lane_t - u];
+        tot += cnt[u];
       }
-      ctl[0] = sel;
-      ctl[1] = sel < 0 ? cum : remaining - cum;
-      ctl[2] = sel < 0 ? 0 : (int)hist[sel];
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane_t >= o) incl += y;
+      }
+      const int excl = incl - tot;
+      if (excl < remaining && remaining <= incl) {
+        int cum = excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (cum + cnt[u] >= remaining) {
+            ctl[0] = 255 - 8 * lane_t - u;
+            ctl[1] = remaining - cum;
+            ctl[2] = cnt[u];
+            break;
+          }
+          cum += cnt[u];
+        }
+      }
+      if (lane_t == 31 && incl < remaining) {  // fewer entries than remaining in total
+        ctl[0] = -1;
+        ctl[1] = incl;
+        ctl[2] = 0;
+      }
     }
     __syncthreads();
     const int sel = ctl[0];

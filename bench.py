@@ -17,7 +17,8 @@ process, the script relaunches itself under torchrun with N ranks; started by a
 launcher with a different number of ranks, it exits with status 2.  `extra`
 carries the decode, causal8k, causal8000 and bf16_k3 workloads, the decode over a
 16-key-page cache, the 8-token (speculative) decode over the same cache on the
-tensor cores, and the lightning-indexer score and top-k, each with its roofline.
+tensor cores, the lightning-indexer score and top-k, and the backward pass on the
+causal4k shapes, each with its roofline.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the method available here) on bounded samples of the same workload.
@@ -513,6 +514,75 @@ def measure_indexer(name, K, W, world, device, peaks):
     return res
 
 
+BWD_WORKLOADS = {"bwd_causal4k": "causal4k"}  # backward of a forward workload, same shapes
+
+
+def measure_bwd(name, K, W, world, device, peaks):
+    """Backward pass (attn_bwd) on a forward workload's shapes: TFLOP/s counted as 2.5 times
+    the forward's (five products of the forward's size instead of two), halved when causal."""
+    import torch
+
+    import attention_forward_tiled_b200 as attn
+    from attention_forward_tiled_b200.inputs import WORKLOADS, flops, make_inputs
+
+    w = WORKLOADS[BWD_WORKLOADS[name]]
+    q, k, v = (t.to(device) for t in make_inputs(**w))
+    g = torch.Generator("cpu").manual_seed(w["seed"] + 1000)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).to(device)
+    o, lse = attn.attn_fwd(q, k, v, causal=w["causal"], scale=w["scale"])
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        attn.attn_bwd(q, k, v, o, lse, dout, causal=w["causal"], scale=w["scale"], stream=stream,
+                      dq=dq, dk=dk, dv=dv)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(device)
+    if attn.get_status(device=device) != 0:
+        raise RuntimeError("device status error during warm-up")
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    t_steps = time_gpu_steps(step, K, stream, None)
+    sampler.stop()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    if attn.get_status(device=device) != 0:
+        raise RuntimeError("device status error during the timed region")
+    elapsed_ms = max_over_ranks(sum(t_steps), world)
+    f = 2.5 * flops(**w)
+    achieved = f / (statistics.mean(t_steps) * 1e-3) / 1e12
+    del q, k, v, dout, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+    cfg = workload_config(BWD_WORKLOADS[name], w)
+    cfg["workload"] = name
+    return {"value": world * K * f / (elapsed_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": elapsed_ms / K,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "algorithmic_flops_per_launch": f,
+                         "note": "the step is the D pre-pass, the gradient kernel and the dQ cast"},
+            "clocks": sampler.summary(), "config": cfg}
+
+
+def print_single(args, world, rank, r, dtype):
+    """One JSON line for a workload timed on its own (profiling and single-kernel runs)."""
+    line = {"metric": METRIC, "value": r["value"], "unit": r["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded randn)",
+            "config": r["config"], "roofline": r["roofline"], "e2e": None, "clocks": r["clocks"],
+            "impl": "ours"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
     import torch
 
@@ -529,7 +599,14 @@ def run_ours(args):
     peaks = load_peaks()
     K, W = args.steps, max(3, args.warmup)
 
-    from attention_forward_tiled_b200.inputs import PAGED_WORKLOADS, WORKLOADS
+    from attention_forward_tiled_b200.inputs import INDEXER_WORKLOADS, PAGED_WORKLOADS, WORKLOADS
+    if args.workload in INDEXER_WORKLOADS:
+        r = measure_indexer(args.workload, K, W, world, device, peaks)
+        r["score"]["topk"] = r["topk"]
+        return print_single(args, world, rank, r["score"], INDEXER_WORKLOADS[args.workload]["dtype"])
+    if args.workload in BWD_WORKLOADS:
+        r = measure_bwd(args.workload, K, W, world, device, peaks)
+        return print_single(args, world, rank, r, WORKLOADS[BWD_WORKLOADS[args.workload]]["dtype"])
     if args.workload in PAGED_WORKLOADS:
         # the paged decode on its own (profiling runs): its line has no end-to-end figure
         r = measure_paged(args.workload, K, W, world, device, peaks)
@@ -561,6 +638,7 @@ def run_ours(args):
         r = measure_indexer("indexer_h4", K, W, world, device, peaks)
         extra["indexer_h4_score"] = r["score"]
         extra["indexer_h4_topk"] = r["topk"]
+        extra["bwd_causal4k"] = measure_bwd("bwd_causal4k", K, W, world, device, peaks)
     line = {
         "metric": METRIC,
         "value": main["value"],

@@ -224,6 +224,34 @@ ATTN_API int attn_fwd_paged(const void* q, const void* k_cache, const void* v_ca
                             attn_stream_t stream);
 
 /*
+ * attn_bwd -- gradients of attn_fwd (the backward pass).
+ *
+ * The step after the forward: the article notes (section "传统注意力的显存陷阱")
+ * that eager attention keeps the N x N matrix for backpropagation.  Here the
+ * probabilities are recomputed tile by tile from q, k and the forward's lse and
+ * never stored; for an upstream gradient dO of O:
+ *   P = exp(scale * Q K^T - lse) (masked entries 0),  dV = P^T dO,
+ *   dS = P o (dO V^T - D) with D_i = sum_t dO_it O_it,
+ *   dQ = scale * dS K,   dK = scale * dS^T Q.
+ *
+ *   q, o, dout   [B, Nq, H, d]   dtype      (read; o and lse as attn_fwd wrote them)
+ *   k, v         [B, Nk, H, d]   dtype      (read)
+ *   lse          [B, H, Nq]      float32    (read, required)
+ *   dq           [B, Nq, H, d]   dtype      (written)
+ *   dk, dv       [B, Nk, H, d]   dtype      (written)
+ *   Sizes, causal rule, scale, dtype and alignment as attn_fwd; the outputs
+ *   must not overlap each other or any input.  P and dS multiply on the tensor
+ *   cores in the input type with fp32 accumulation; dQ is accumulated over key
+ *   tiles in fp32.  A workspace of B*Nq*H*(d+1)*4 bytes (rounded up) is taken
+ *   stream-ordered from the default pool and returned on the same stream.
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA;
+ * asynchronous like attn_fwd.
+ */
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk,
+                      int d, int causal, float scale, int dtype, attn_stream_t stream);
+
+/*
  * attn_indexer_score -- lightning-indexer score on the tensor cores.
  *
  * The aispot.cmou.io report on llama.cpp release b11372 (entry "compute the
