@@ -168,6 +168,21 @@ int encode_rows3d(CUtensorMap* map, const void* ptr, int B, long long rows, int 
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// 4-D view (d, H, N, B) of a contiguous fp32 [B, N, H, d] tensor; box (d, 1, box_rows, 1),
+// no swizzle (the backward's dQ accumulator, written by TMA reduce-adds).
+int encode_f32_bnhd(CUtensorMap* map, void* ptr, int B, int N, int H, int d, int box_rows) {
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return ATTN_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)N * H * d * 4};
+  const cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
@@ -528,6 +543,10 @@ int launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, con
   if (cudaMallocAsync(reinterpret_cast<void**>(&ws), ws_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
   float* dsum = reinterpret_cast<float*>(ws);
   float* dq_acc = reinterpret_cast<float*>(ws + dsum_bytes);
+  if (encode_f32_bnhd(&p.tm_dq, dq_acc, B, Nq, H, D, 64) != ATTN_OK) {
+    cudaFreeAsync(ws, stream);
+    return ATTN_ERR_CUDA;
+  }
   p.lse = lse;
   p.dsum = dsum;
   p.dq_acc = dq_acc;

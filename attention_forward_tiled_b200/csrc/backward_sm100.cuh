@@ -15,8 +15,9 @@
 //   P^T, dS^T -> fp16/bf16 into the consumed TMEM columns (and dS^T into shared memory)
 //   dV  += P^T dO   and  dK  += dS^T Q    (A from TMEM, B = dO / Q read MN-major)
 //   dQ^T = K^T dS^T                       (A = K read MN-major, B = dS^T in shared memory)
-// dQ^T (lane = head-dim element, column = query) is added to an fp32 accumulator in
-// global memory with coalesced atomic adds (other key tiles add to the same rows);
+// dQ^T (lane = head-dim element, column = query) is staged in shared memory and added to
+// an fp32 accumulator in global memory with one TMA reduce-add per tile (other key tiles
+// add to the same rows);
 // dV and dK are written once at the end.  Roles (192 threads): warps 0-3 elementwise
 // and epilogues, warp 4 TMA producer, warp 5 MMA issuer.
 //
@@ -33,6 +34,7 @@ struct BwdParams {
   CUtensorMap tm_do;  // dO [B, Nq, H, D], same
   CUtensorMap tm_k;   // k  [B, Nk, H, D], box (64, 1, 128, 1)
   CUtensorMap tm_v;   // v  [B, Nk, H, D], same
+  CUtensorMap tm_dq;  // dq_acc [B, Nq, H, D] fp32 as 4-D (D, H, Nq, B), box (D, 1, 64, 1), no swizzle
   const float* lse;   // [B, H, Nq] natural log (the forward's)
   const float* dsum;  // [B, H, Nq]: D_i = sum_t dO_it O_it
   float* dq_acc;      // [B, Nq, H, D] fp32, zeroed before the launch
@@ -62,7 +64,8 @@ struct BwdCfg {
   static constexpr int kOffDS = kOffQ + kStages * kStageBytes;  // dS^T [128 keys][64 queries] fp16
   static constexpr int kDSBytes = 128 * 128;
   static constexpr int kOffRow = kOffDS + kDSBytes;        // per-query lse2 and D, [2][2][64] fp32
-  static constexpr int kOffBar = kOffRow + 2 * 2 * 64 * 4;
+  static constexpr int kOffDQ = kOffRow + 2 * 2 * 64 * 4;  // dQ tile [64 queries][D] fp32 for the reduce
+  static constexpr int kOffBar = kOffDQ + 64 * D * 4;
   static constexpr int kBarKV = 0;
   static constexpr int kBarQFull = 1;                      // [2]
   static constexpr int kBarQEmpty = 3;                     // [2]
@@ -79,6 +82,7 @@ struct BwdCfg {
   static constexpr int kMmaWarp = 5;
   static constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 128, kColDV = 256, kColDK = 384;
   static_assert(kOffQ % 1024 == 0 && kOffDS % 1024 == 0 && kQTile % 1024 == 0, "swizzle atoms");
+  static_assert(kOffDQ % 128 == 0, "bulk-copy source alignment");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -143,6 +147,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       tma_prefetch_map(&p.tm_do);
       tma_prefetch_map(&p.tm_k);
       tma_prefetch_map(&p.tm_v);
+      tma_prefetch_map(&p.tm_dq);
     }
     mbar_arrive_expect_tx_w(BAR(C::kBarKV), 2 * C::kKTile);
     for (int bx = 0; bx < C::kBoxes; ++bx) {
@@ -238,17 +243,29 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     const long long diag = (long long)p.Nk - p.Nq;
     float* rowbuf = reinterpret_cast<float*>(smem + C::kOffRow);  // [2][2][64]: lse2, D
     uint8_t* ds_row = smem + C::kOffDS + r * 128;                  // dS^T row of this key
+    float* dq_stage = reinterpret_cast<float*>(smem + C::kOffDQ);  // [64][D]
+    // per-query lse (base 2) and D of query tile i into rowbuf[i & 1]: loaded a tile ahead,
+    // stored to shared memory after this tile's work, so the load latency is hidden
+    auto row_load = [&](int i, float& l2, float& dd) {
+      const int q = (qt0 + i) * 64 + r;
+      const long long o = ((long long)b * p.H + h) * p.Nq + q;
+      l2 = (r < 64 && q < p.Nq) ? __ldg(p.lse + o) * 1.4426950408889634f : 0.f;
+      dd = (r < 64 && q < p.Nq) ? __ldg(p.dsum + o) : 0.f;
+    };
+    float nl2 = 0.f, ndd = 0.f;
+    if (nqt > 0) {
+      row_load(0, nl2, ndd);
+      if (r < 64) {
+        rowbuf[r] = nl2;
+        rowbuf[64 + r] = ndd;
+      }
+    }
+    named_bar_sync(1, 128);
     for (int i = 0; i < nqt; ++i) {
       const int q0 = (qt0 + i) * 64;
       float* lse2 = rowbuf + (i & 1) * 128;
       float* dsm = lse2 + 64;
-      if (r < 64) {
-        const int q = q0 + r;
-        const long long o = ((long long)b * p.H + h) * p.Nq + q;
-        lse2[r] = q < p.Nq ? __ldg(p.lse + o) * 1.4426950408889634f : 0.f;
-        dsm[r] = q < p.Nq ? __ldg(p.dsum + o) : 0.f;
-      }
-      named_bar_sync(1, 128);
+      if (i + 1 < nqt) row_load(i + 1, nl2, ndd);
       mbar_wait(BAR(C::kBarSFull), i & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
@@ -298,7 +315,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarPDone));
 
-      // dQ^T of this tile: lane = head-dim element, 64 query columns -> fp32 accumulator
+      // dQ^T of this tile (lane = head-dim element, 64 query columns) -> shared memory as
+      // [query][D] -> one TMA reduce-add into the fp32 accumulator (rows past Nq are skipped)
       mbar_wait(BAR(C::kBarDQFull), i & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
@@ -311,14 +329,26 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarDQFree));
-      if (r < D && !*abort_flag) {
-        float* dst = p.dq_acc + (((long long)b * p.Nq + q0) * p.H + h) * D + r;
-        const long long qstride = (long long)p.H * D;
+      if (r == 0) bulk_wait_group_read0();  // the previous tile's reduce has read the stage
+      named_bar_sync(1, 128);
+      if (r < D) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (q0 + c < p.Nq) atomicAdd(dst + c * qstride, __uint_as_float(dq[c >> 5][c & 31]));
+        for (int c = 0; c < 64; ++c) dq_stage[c * D + r] = __uint_as_float(dq[c >> 5][c & 31]);
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the TMA
+      // next tile's per-query rows, loaded at the top of this iteration
+      if (i + 1 < nqt && r < 64) {
+        rowbuf[((i + 1) & 1) * 128 + r] = nl2;
+        rowbuf[((i + 1) & 1) * 128 + 64 + r] = ndd;
+      }
+      named_bar_sync(1, 128);
+      if (r == 0 && !*abort_flag) {
+        tma_reduce_add_4d(&p.tm_dq, sbase + C::kOffDQ, 0, h, q0, b);
+        bulk_commit_group();
       }
     }
+    if (r == 0) bulk_wait_group_read0();  // ... and the last one before the CTA exits
+    if (r == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 
     // ---- epilogue: dV and scale * dK (lane = key) -> 16-bit -> global.  The last tile's
     // dQ^T commit covered every earlier product, so dV and dK are final here.  The TMEM

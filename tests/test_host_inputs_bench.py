@@ -118,3 +118,14 @@ def test_clock_sampler_without_nvml(monkeypatch):
     s.stop()
     summ = s.summary()
     assert summ["sm_mhz"] is None and summ["samples"] == 0 and "error" in summ
+
+
+def test_traffic_figures_follow_their_kernel():
+    """Each benchmark workload's traffic figure is tied to the sources of the kernel it ran."""
+    import bench
+    assert bench.kernel_kind("causal4k") == "prefill" and bench.kernel_kind("bf16_k3") == "prefill"
+    assert bench.kernel_kind("decode") == "decode" and bench.kernel_kind("decode_paged16") == "decode"
+    assert bench.kernel_kind("spec8_paged16") == "mq"
+    assert bench.kernel_kind("indexer_h4") == "indexer" and bench.kernel_kind("bwd_causal4k") == "bwd"
+    shas = {k: bench.kernel_source_sha(k) for k in bench.KERNEL_SOURCES}
+    assert len(set(shas.values())) == len(shas)
