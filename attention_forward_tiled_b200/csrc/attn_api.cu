@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "attn.h"
@@ -179,6 +180,21 @@ int encode_f32_bnhd(CUtensorMap* map, void* ptr, int B, int N, int H, int d, int
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 3-D view (P, T, B) of a contiguous f16 [B, T, P] pool mask; box (128 keys, tokens, 1), no
+// swizzle.  Needs P a multiple of 8 (16-byte row pitch) and a 16-byte aligned base.
+int encode_mask3d(CUtensorMap* map, const void* ptr, int B, int T, int P, int box_tokens) {
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return ATTN_ERR_CUDA;
+  const cuuint64_t dims[3] = {(cuuint64_t)P, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)P * 2, (cuuint64_t)T * P * 2};
+  const cuuint32_t box[3] = {128, (cuuint32_t)box_tokens, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -507,6 +523,12 @@ int launch_indexer(DeviceState* ds, const void* q, const void* kp, const float* 
   p.P = P;
   p.lg_h = lg;
   p.tok_per_tile = 128 / H;
+  p.mask_tma = mask != nullptr && P % 8 == 0 && reinterpret_cast<uintptr_t>(mask) % 16 == 0;
+  if (p.mask_tma) {
+    if (int rc = encode_mask3d(&p.tm_mask, mask, B, T, P, p.tok_per_tile)) return rc;
+  } else {
+    std::memset(&p.tm_mask, 0, sizeof(p.tm_mask));
+  }
   p.n_ttiles = (T + p.tok_per_tile - 1) / p.tok_per_tile;
   p.n_ptiles = (P + 127) / 128;
   const long long items = (long long)B * p.n_ptiles * p.n_ttiles;

@@ -11,11 +11,12 @@
 // (token, head) pairs of 128 / H tokens its N = 128 columns, so the product lands
 // in TMEM with one thread per key holding every head of every token of the tile:
 // the rectifier, the head weights and the head sum stay inside a thread.  Work
-// items (b, key tile, token tile) go to persistent CTAs (192 threads):
-//   * warp 4, producer: TMA loads of the key tile (once per run of items on the same
-//     tile) and of the query tiles into shared memory;
-//   * warp 5, MMA issuer: S^T = Kp Q^T into one of two TMEM accumulators;
-//   * warps 0-3, epilogue: rectify, weight, sum over heads, add the f16 mask and
+// items (b, key tile, token tile) go to persistent CTAs (320 threads):
+//   * warp 8, producer: TMA loads of the key tile (once per run of items on the same
+//     tile), of the query tiles and of the item's mask tile, and cp.async copies of
+//     its head weights, all into shared memory;
+//   * warp 9, MMA issuer: S^T = Kp Q^T into one of two TMEM accumulators;
+//   * warps 0-7, epilogue: rectify, weight, sum over heads, add the f16 mask and
 //     store fp32 scores (one thread per key: consecutive keys, coalesced stores).
 //
 // Top-k (prhub.com.cn report "PR #45743 完整报告", section "实现拆解": the decode
@@ -31,15 +32,17 @@
 namespace attn_b200 {
 
 struct IndexerParams {
-  CUtensorMap tm_q;   // q [B, T, H, D] as 3-D (D, T*H, B), box (64, 128, 1), 128B swizzle
-  CUtensorMap tm_k;   // kp [B, P, D] as 3-D (D, P, B), box (64, 128, 1), 128B swizzle
-  const float* w;     // [B, T, H]
+  CUtensorMap tm_q;     // q [B, T, H, D] as 3-D (D, T*H, B), box (64, 128, 1), 128B swizzle
+  CUtensorMap tm_k;     // kp [B, P, D] as 3-D (D, P, B), box (64, 128, 1), 128B swizzle
+  CUtensorMap tm_mask;  // mask [B, T, P] f16 as 3-D (P, T, B), box (128, 128 / H, 1), no swizzle
+  const float* w;       // [B, T, H]
   const uint16_t* mask;  // [B, T, P] f16 (0 / -inf) or nullptr
-  float* score;       // [B, T, P]
+  float* score;         // [B, T, P]
   int* status;
   int B, T, H, P;
-  int lg_h;           // log2(H)
-  int tok_per_tile;   // 128 / H
+  int lg_h;             // log2(H)
+  int tok_per_tile;     // 128 / H
+  int mask_tma;         // 1: mask tiles come by TMA (P % 8 == 0, 16-byte aligned mask)
   int n_ttiles, n_ptiles, n_items;
   unsigned long long timeout_ns;
 };
@@ -61,14 +64,16 @@ struct IndexerCfg {
   static constexpr int kBarQFull = 4;                     // [kQStages]
   static constexpr int kBarQEmpty = 4 + kQStages;         // [kQStages]
   static constexpr int kBarAccFull = 4 + 2 * kQStages;    // [2]
-  static constexpr int kBarAccFree = 6 + 2 * kQStages;    // [2]
-  static constexpr int kBarMmaDone = 8 + 2 * kQStages;    // [1]
-  static constexpr int kNumBars = 9 + 2 * kQStages;
+  static constexpr int kBarAccFree = 6 + 2 * kQStages;    // [2] accumulator, weights and mask buffer free
+  static constexpr int kBarAuxFull = 8 + 2 * kQStages;    // [2] weights and mask of an item landed
+  static constexpr int kBarMmaDone = 10 + 2 * kQStages;   // [1]
+  static constexpr int kNumBars = 11 + 2 * kQStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // +1024: manual 1 KB alignment
-  static constexpr int kThreads = 192;
-  static constexpr int kProducerWarp = 4;
-  static constexpr int kMmaWarp = 5;
+  static constexpr int kEpiWarps = 8;                      // two per TMEM lane quarter
+  static constexpr int kThreads = 32 * (kEpiWarps + 2);
+  static constexpr int kProducerWarp = kEpiWarps;
+  static constexpr int kMmaWarp = kEpiWarps + 1;
   static constexpr uint32_t kTmemCols = 256;  // two 128-column accumulators
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -87,6 +92,136 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
   it.pt = bp % p.n_ptiles;
   it.b = bp / p.n_ptiles;
   return it;
+}
+
+// Asynchronous 4-byte global -> shared copy (the LDGSTS path); bytes past src_bytes are
+// filled with zeros without being read.
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// One arrival on the mbarrier once every earlier cp.async of this thread has landed (the
+// barrier's expected count includes it).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Epilogue of the score kernel: eight warps, thread = key (TMEM lane) of the tile; warp w
+// reads lanes 32 (w % 4) .. + 31 and accumulator columns 64 (w / 4) .. + 63.  H = 2^LGH heads,
+// so the 128 columns are 128 / H tokens of H heads each (column = token * H + head) and a
+// token's score is the weighted sum of its H rectified columns.  At H = 128 one token spans
+// all columns, and warps 0-3 take them all.  The head weights and the mask rows of the item
+// were put in shared memory by the producer warp; an aligned mask came by TMA, any other
+// is read from global memory here.
+template <int D, int LGH>
+__device__ __forceinline__ void indexer_epilogue(const IndexerParams& p, uint8_t* smem, uint32_t tmem,
+                                                 uint64_t* bars, const WaitCtx& wctx, int item0,
+                                                 int item1) {
+  using C = IndexerCfg<D>;
+  constexpr int H = 1 << LGH;
+  constexpr int TPT = 128 / H;  // tokens per tile
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = (warp & 3) * 32 + lane;  // key of the tile
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const int c_begin = LGH == 7 ? 0 : (warp >> 2) * 64;
+  const int c_end = LGH == 7 ? ((warp >> 2) == 0 ? 128 : 0) : c_begin + 64;
+  const float* wbuf = reinterpret_cast<const float*>(smem + C::kOffW);        // [2][128]
+  const uint16_t* mbuf = reinterpret_cast<const uint16_t*>(smem + C::kOffM);  // [2][128 tokens][128 keys]
+
+  int g = 0;
+  for (int item = item0; item < item1; ++item, ++g) {
+    const IndexerItem it = indexer_item(p, item);
+    const int ab = g & 1;
+    const int t0 = it.tt * TPT;
+    const int key = it.pt * 128 + r;
+    const bool key_ok = key < p.P;
+    const bool full = t0 + TPT <= p.T;  // no token of the tile lies past T
+    // this key's score for token 0 of the tile; token tl is P floats further on
+    float* const srow = p.score + ((long long)it.b * p.T + t0) * p.P + key;
+    const float* wb = wbuf + ab * 128;
+    const uint16_t* mb = mbuf + ab * 128 * 128 + r;
+    // n scores of consecutive tokens from tl0: the mask values are read before any store,
+    // so those reads are not held behind the global stores
+    auto emit = [&](int tl0, auto& v) {
+      constexpr int n = sizeof(v) / sizeof(float);
+      if (p.mask != nullptr) {
+        float mv[n];
+        if (p.mask_tma) {
+#pragma unroll
+          for (int j = 0; j < n; ++j) mv[j] = __half2float(__ushort_as_half(mb[(tl0 + j) * 128]));
+        } else {
+          const uint16_t* mrow = p.mask + ((long long)it.b * p.T + t0 + tl0) * p.P + key;
+#pragma unroll
+          for (int j = 0; j < n; ++j)
+            mv[j] = (key_ok && t0 + tl0 + j < p.T) ? __half2float(__ushort_as_half(mrow[(long long)j * p.P])) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < n; ++j) v[j] += mv[j];
+      }
+      if (!key_ok) return;
+      float* dst = srow + (long long)tl0 * p.P;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < n; ++j, dst += p.P) *dst = v[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < n; ++j, dst += p.P)
+          if (t0 + tl0 + j < p.T) *dst = v[j];
+      }
+    };
+    mbar_wait(smem_u32(&bars[C::kBarAuxFull + ab]), (g >> 1) & 1, wctx);
+    mbar_wait(smem_u32(&bars[C::kBarAccFull + ab]), (g >> 1) & 1, wctx);
+    __syncwarp();
+    tc_fence_after_sync();
+    float carry = 0.f;  // H > 32: a token spans several 32-column pieces
+#pragma unroll 1
+    for (int c0 = c_begin; c0 < c_end; c0 += 64) {
+      uint32_t s[2][32];
+      tmem_ld32(tmem + lane_base + ab * 128u + c0, s[0]);
+      tmem_ld32(tmem + lane_base + ab * 128u + c0 + 32, s[1]);
+      tmem_ld_wait();
+      reg_order_after_wait(s[0]);
+      reg_order_after_wait(s[1]);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int cb = c0 + half * 32;
+        float wv[32];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(wb + cb + c);
+          wv[c] = w4.x;
+          wv[c + 1] = w4.y;
+          wv[c + 2] = w4.z;
+          wv[c + 3] = w4.w;
+        }
+        if constexpr (H <= 32) {
+          float v[32 / H];
+#pragma unroll
+          for (int j = 0; j < 32 / H; ++j) {
+            float a = 0.f;
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+              a = fmaf(wv[j * H + h], fmaxf(__uint_as_float(s[half][j * H + h]), 0.f), a);
+            v[j] = a;
+          }
+          emit(cb >> LGH, v);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) carry = fmaf(wv[c], fmaxf(__uint_as_float(s[half][c]), 0.f), carry);
+          if (((cb + 32) & (H - 1)) == 0) {
+            float v[1] = {carry};
+            emit(cb >> LGH, v);
+            carry = 0.f;
+          }
+        }
+      }
+    }
+    // accumulator ab, and the weights and mask of buffer ab, are free for item g + 2
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars[C::kBarAccFree + ab]));
+  }
 }
 
 template <int D, bool BF16>
@@ -114,7 +249,8 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
       mbar_init(BAR(C::kBarKFull + i), 1);
       mbar_init(BAR(C::kBarKEmpty + i), 1);
       mbar_init(BAR(C::kBarAccFull + i), 1);
-      mbar_init(BAR(C::kBarAccFree + i), 4);  // one arrive per epilogue warp
+      mbar_init(BAR(C::kBarAccFree + i), C::kEpiWarps);  // one arrive per epilogue warp
+      mbar_init(BAR(C::kBarAuxFull + i), 33);  // the byte-count arrive + one cp.async arrive per producer lane
     }
     for (int s = 0; s < C::kQStages; ++s) {
       mbar_init(BAR(C::kBarQFull + s), 1);
@@ -139,15 +275,19 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
   };
 
   if (warp == C::kProducerWarp) {
-    // ======================= TMA producer =======================
+    // ======================= producer: TMA tiles, weights, mask =======================
     if (lane == 0) {
       tma_prefetch_map(&p.tm_q);
       tma_prefetch_map(&p.tm_k);
+      if (p.mask_tma) tma_prefetch_map(&p.tm_mask);
     }
+    const int tpt = p.tok_per_tile;
+    const uint32_t mask_bytes = p.mask_tma ? (uint32_t)tpt * 128u * 2u : 0u;
     int nk = 0;  // key tiles loaded
-    int g = 0;   // query tiles loaded
+    int nq = 0;  // query tiles loaded
+    int na = 0;  // weight / mask buffers loaded
     IndexerItem prev{-1, -1, -1};
-    for (int item = item0; item < item1; ++item, ++g) {
+    for (int item = item0, g = 0; item < item1; ++item, ++g) {
       const IndexerItem it = indexer_item(p, item);
       if (!same_key_tile(it, prev)) {
         const int kb = nk & 1;
@@ -169,13 +309,38 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
       for (int bx = 0; bx < C::kBoxes; ++bx)
         tma_load_3d_w(sbase + C::kOffQ + st * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
                       BAR(C::kBarQFull + st), bx * 64, it.tt * 128, it.b);
+      ++nq;
+      // weights and mask of this item into buffer g & 1, free once the epilogue is done
+      // with item g - 2
+      const int xb = g & 1;
+      if (g >= 2) mbar_wait(BAR(C::kBarAccFree + xb), ((g >> 1) - 1) & 1, wctx);
+      __syncwarp();
+      if (warp_flag(abort_flag)) break;
+      const int t0 = it.tt * tpt;
+      mbar_arrive_expect_tx_w(BAR(C::kBarAuxFull + xb), mask_bytes);
+      if (p.mask_tma)
+        tma_load_3d_w(sbase + C::kOffM + xb * (128 * 128 * 2), &p.tm_mask, BAR(C::kBarAuxFull + xb),
+                      it.pt * 128, t0, it.b);
+      const float* wrow = p.w + ((long long)it.b * p.T) * p.H;
+#pragma unroll
+      for (int c = lane; c < 128; c += 32) {  // column c: token c / H, head c % H
+        const int t = t0 + (c >> p.lg_h);
+        const bool ok = t < p.T;
+        cp_async_4(sbase + C::kOffW + (xb * 128 + c) * 4, wrow + (long long)(ok ? t : 0) * p.H + (c & (p.H - 1)),
+                   ok ? 4u : 0u);
+      }
+      cp_async_mbar_arrive(BAR(C::kBarAuxFull + xb));
+      ++na;
     }
+    cp_async_wait_all();
     if (lane == 0 && *abort_flag) {
       // let every copy this warp started land before the CTA can exit
-      for (int i = max(0, g - C::kQStages); i < g; ++i)
+      for (int i = max(0, nq - C::kQStages); i < nq; ++i)
         mbar_wait_drain(BAR(C::kBarQFull + i % C::kQStages), (i / C::kQStages) & 1, p.timeout_ns);
       for (int i = max(0, nk - 2); i < nk; ++i)
         mbar_wait_drain(BAR(C::kBarKFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
+      for (int i = max(0, na - 2); i < na; ++i)
+        mbar_wait_drain(BAR(C::kBarAuxFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
@@ -217,84 +382,16 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
     mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    // ======================= epilogue warps 0-3 (thread = pooled key) ===========
-    // The head weights and pool mask of item g + 1 are loaded into shared memory while item
-    // g's product runs (plain loads: the mask rows of arbitrary length P need not meet any
-    // copy-engine alignment), so no global load sits between the score stores.
-    const int r = threadIdx.x;  // key of the tile
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int lg_h = p.lg_h, tpt = p.tok_per_tile;
-    float* wbuf = reinterpret_cast<float*>(smem + C::kOffW);        // [2][128]
-    uint16_t* mbuf = reinterpret_cast<uint16_t*>(smem + C::kOffM);  // [2][128][128]
-    auto prefetch = [&](int item, int buf) {
-      const IndexerItem it = indexer_item(p, item);
-      const int t0 = it.tt * tpt;
-      const long long row_bt = (long long)it.b * p.T;
-      {  // weight of column r: w[b, t0 + r / H, r % H]
-        const int t = t0 + (r >> lg_h);
-        wbuf[buf * 128 + r] = t < p.T ? __ldg(p.w + (row_bt + t0) * (1 << lg_h) + r) : 0.f;
-      }
-      if (p.mask != nullptr) {
-        const int key = it.pt * 128 + r;
-        uint16_t* mb = mbuf + buf * 128 * 128 + r;
-        for (int c0 = 0; c0 < tpt; c0 += 32) {  // 32 independent loads in flight, then the stores
-          uint16_t v[32];
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int t = t0 + c0 + u;
-            v[u] = (c0 + u < tpt && t < p.T && key < p.P) ? __ldg(p.mask + (row_bt + t) * p.P + key) : 0;
-          }
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (c0 + u < tpt) mb[(c0 + u) * 128] = v[u];
-        }
-      }
-    };
-    if (item0 < item1) prefetch(item0, 0);
-    named_bar_sync(1, 128);
-    int g = 0;
-    for (int item = item0; item < item1; ++item, ++g) {
-      const IndexerItem it = indexer_item(p, item);
-      const int ab = g & 1;
-      if (item + 1 < item1) prefetch(item + 1, ab ^ 1);
-      const int t0 = it.tt * tpt;
-      const long long row_bt = (long long)it.b * p.T;
-      mbar_wait(BAR(C::kBarAccFull + ab), (g >> 1) & 1, wctx);
-      __syncwarp();
-      tc_fence_after_sync();
-      const int key = it.pt * 128 + r;
-      const float* wb = wbuf + ab * 128;
-      const uint16_t* mb = mbuf + ab * 128 * 128 + r;
-      float acc = 0.f;
-      // 32 columns at a time: column c = t_local * H + h
-#pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t s[32];
-        tmem_ld32(tmem + lane_base + ab * 128u + c0, s);
-        tmem_ld_wait();
-        reg_order_after_wait(s);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = c0 + c;
-          acc = fmaf(wb[col], fmaxf(__uint_as_float(s[c]), 0.f), acc);
-          if (((col + 1) & ((1 << lg_h) - 1)) == 0) {  // last head of a token: its score is complete
-            const int tl = col >> lg_h;
-            const int t = t0 + tl;
-            if (t < p.T && key < p.P) {
-              float v = acc;
-              if (p.mask != nullptr) v += __half2float(__ushort_as_half(mb[tl * 128]));
-              p.score[(row_bt + t) * p.P + key] = v;
-            }
-            acc = 0.f;
-          }
-        }
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::kBarAccFree + ab));
-      // every thread is done with buffer ab, and buffer ab ^ 1 is complete, before the next
-      // item reads ab ^ 1 and prefetches into ab
-      named_bar_sync(1, 128);
+    // ======================= epilogue warps 0-7 (thread = pooled key) ===========
+    switch (p.lg_h) {  // the head count fixes how columns group into tokens
+      case 0: indexer_epilogue<D, 0>(p, smem, tmem, bars, wctx, item0, item1); break;
+      case 1: indexer_epilogue<D, 1>(p, smem, tmem, bars, wctx, item0, item1); break;
+      case 2: indexer_epilogue<D, 2>(p, smem, tmem, bars, wctx, item0, item1); break;
+      case 3: indexer_epilogue<D, 3>(p, smem, tmem, bars, wctx, item0, item1); break;
+      case 4: indexer_epilogue<D, 4>(p, smem, tmem, bars, wctx, item0, item1); break;
+      case 5: indexer_epilogue<D, 5>(p, smem, tmem, bars, wctx, item0, item1); break;
+      case 6: indexer_epilogue<D, 6>(p, smem, tmem, bars, wctx, item0, item1); break;
+      default: indexer_epilogue<D, 7>(p, smem, tmem, bars, wctx, item0, item1); break;
     }
   }
 

@@ -514,7 +514,7 @@ def measure_indexer(name, K, W, world, device, peaks):
         res[kind] = {"value": world * K * nbytes / (elapsed_ms * 1e-3) / 1e9, "unit": "GB/s",
                      "ms_per_step": elapsed_ms / K,
                      "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                                  "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                                  "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic("%s.%s" % (name, kind)),
                                   "algorithmic_bytes_per_launch": nbytes},
                      "clocks": sampler.summary(),
                      "config": {"workload": name, "kernel": kind, "B": B, "T": T, "H": H, "P": P, "d": d,
@@ -573,8 +573,8 @@ def measure_bwd(name, K, W, world, device, peaks):
     return {"value": world * K * f / (elapsed_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": elapsed_ms / K,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                         "algorithmic_flops_per_launch": f,
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": committed_traffic(name), "algorithmic_flops_per_launch": f,
                          "note": "the step is the D pre-pass, the gradient kernel and the dQ cast"},
             "clocks": sampler.summary(), "config": cfg}
 

@@ -37,6 +37,13 @@ CASES = [
     (2, 130, 1, 384, 64, "f16", "random", True),
     (1, 40, 16, 129, 64, "bf16", "random", True),
     (1, 3, 128, 300, 128, "f16", "constant", False),
+    # every head count's column grouping, with both mask paths (pool length a multiple of 8
+    # or not) and a token tail in the last tile
+    (1, 70, 2, 520, 128, "f16", "random", True),
+    (1, 20, 8, 136, 64, "bf16", "random", True),
+    (2, 9, 32, 264, 128, "f16", "random", True),
+    (1, 6, 64, 1000, 128, "bf16", "random", True),
+    (1, 3, 128, 77, 64, "f16", "random", True),
 ]
 
 
