@@ -184,14 +184,14 @@ int encode_f32_bnhd(CUtensorMap* map, void* ptr, int B, int N, int H, int d, int
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// 3-D view (P, T, B) of a contiguous f16 [B, T, P] pool mask; box (128 keys, tokens, 1), no
+// 3-D view (P, T, B) of a contiguous f16 [B, T, P] pool mask; box (256 keys, tokens, 1), no
 // swizzle.  Needs P a multiple of 8 (16-byte row pitch) and a 16-byte aligned base.
 int encode_mask3d(CUtensorMap* map, const void* ptr, int B, int T, int P, int box_tokens) {
   EncodeTiledFn encode = get_encode_fn();
   if (!encode) return ATTN_ERR_CUDA;
   const cuuint64_t dims[3] = {(cuuint64_t)P, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t strides[2] = {(cuuint64_t)P * 2, (cuuint64_t)T * P * 2};
-  const cuuint32_t box[3] = {128, (cuuint32_t)box_tokens, 1};
+  const cuuint32_t box[3] = {256, (cuuint32_t)box_tokens, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -523,15 +523,16 @@ int launch_indexer(DeviceState* ds, const void* q, const void* kp, const float* 
   p.P = P;
   p.lg_h = lg;
   p.tok_per_tile = 128 / H;
-  p.mask_tma = mask != nullptr && P % 8 == 0 && reinterpret_cast<uintptr_t>(mask) % 16 == 0;
+  p.mask_tma = mask != nullptr && p.tok_per_tile <= C::kMaskTokens && P % 8 == 0 &&
+               reinterpret_cast<uintptr_t>(mask) % 16 == 0;
   if (p.mask_tma) {
     if (int rc = encode_mask3d(&p.tm_mask, mask, B, T, P, p.tok_per_tile)) return rc;
   } else {
     std::memset(&p.tm_mask, 0, sizeof(p.tm_mask));
   }
   p.n_ttiles = (T + p.tok_per_tile - 1) / p.tok_per_tile;
-  p.n_ptiles = (P + 127) / 128;
-  const long long items = (long long)B * p.n_ptiles * p.n_ttiles;
+  p.n_pairs = (P + 255) / 256;
+  const long long items = (long long)B * p.n_pairs * p.n_ttiles;
   if (items >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
   p.n_items = (int)items;
   p.timeout_ns = g_timeout_ns.load();

@@ -11,12 +11,14 @@
 // (token, head) pairs of 128 / H tokens its N = 128 columns, so the product lands
 // in TMEM with one thread per key holding every head of every token of the tile:
 // the rectifier, the head weights and the head sum stay inside a thread.  Work
-// items (b, key tile, token tile) go to persistent CTAs (320 threads):
-//   * warp 8, producer: TMA loads of the key tile (once per run of items on the same
-//     tile), of the query tiles and of the item's mask tile, and cp.async copies of
-//     its head weights, all into shared memory;
-//   * warp 9, MMA issuer: S^T = Kp Q^T into one of two TMEM accumulators;
-//   * warps 0-7, epilogue: rectify, weight, sum over heads, add the f16 mask and
+// items (b, key tile, token tile) go to persistent CTAs (608 threads):
+//   * warp 16, producer: TMA loads of a pair of key tiles (once per run of items on the
+//     same pair) and of the query tiles (a four-deep ring) into shared memory;
+//   * warp 18, auxiliary loads: the item's mask tile by TMA and its head weights by
+//     cp.async, double-buffered;
+//   * warp 17, MMA issuer: S^T = Kp Q^T for both key tiles of the pair (two TMEM
+//     accumulators per item, two items in flight), so each query tile serves 256 keys;
+//   * warps 0-15, epilogue: rectify, weight, sum over heads, add the f16 mask and
 //     store fp32 scores (one thread per key: consecutive keys, coalesced stores).
 //
 // Top-k (prhub.com.cn report "PR #45743 完整报告", section "实现拆解": the decode
@@ -34,7 +36,7 @@ namespace attn_b200 {
 struct IndexerParams {
   CUtensorMap tm_q;     // q [B, T, H, D] as 3-D (D, T*H, B), box (64, 128, 1), 128B swizzle
   CUtensorMap tm_k;     // kp [B, P, D] as 3-D (D, P, B), box (64, 128, 1), 128B swizzle
-  CUtensorMap tm_mask;  // mask [B, T, P] f16 as 3-D (P, T, B), box (128, 128 / H, 1), no swizzle
+  CUtensorMap tm_mask;  // mask [B, T, P] f16 as 3-D (P, T, B), box (256, 128 / H, 1), no swizzle
   const float* w;       // [B, T, H]
   const uint16_t* mask;  // [B, T, P] f16 (0 / -inf) or nullptr
   float* score;         // [B, T, P]
@@ -42,8 +44,8 @@ struct IndexerParams {
   int B, T, H, P;
   int lg_h;             // log2(H)
   int tok_per_tile;     // 128 / H
-  int mask_tma;         // 1: mask tiles come by TMA (P % 8 == 0, 16-byte aligned mask)
-  int n_ttiles, n_ptiles, n_items;
+  int mask_tma;         // 1: mask tiles come by TMA (H >= 4, P % 8 == 0, 16-byte aligned mask)
+  int n_ttiles, n_pairs, n_items;  // token tiles, pairs of key tiles, items
   unsigned long long timeout_ns;
 };
 
@@ -53,45 +55,58 @@ struct IndexerCfg {
   static constexpr int kBoxBytes = 128 * 128;             // 128 rows x 64 elements x 2 bytes
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;   // 128 rows x D
-  static constexpr int kQStages = 2;
-  static constexpr int kOffK = 0;                                  // key tiles [2]
+  static constexpr int kQStages = 4;      // query tiles come from L2 for every item: a deep ring
+  static constexpr int kMaskTokens = 32;  // mask rows held per buffer: tiles of H >= 4 heads
+  static constexpr int kOffK = 0;                                  // the pair of key tiles
   static constexpr int kOffQ = 2 * kTileBytes;                     // query tiles [kQStages]
   static constexpr int kOffW = kOffQ + kQStages * kTileBytes;     // head weights [2][128] fp32
-  static constexpr int kOffM = kOffW + 2 * 128 * 4;                // pool mask [2][128 tokens][128 keys] f16
-  static constexpr int kOffBar = kOffM + 2 * 128 * 128 * 2;
-  static constexpr int kBarKFull = 0;                     // [2]
-  static constexpr int kBarKEmpty = 2;                    // [2]
-  static constexpr int kBarQFull = 4;                     // [kQStages]
-  static constexpr int kBarQEmpty = 4 + kQStages;         // [kQStages]
-  static constexpr int kBarAccFull = 4 + 2 * kQStages;    // [2]
-  static constexpr int kBarAccFree = 6 + 2 * kQStages;    // [2] accumulator, weights and mask buffer free
-  static constexpr int kBarAuxFull = 8 + 2 * kQStages;    // [2] weights and mask of an item landed
-  static constexpr int kBarMmaDone = 10 + 2 * kQStages;   // [1]
-  static constexpr int kNumBars = 11 + 2 * kQStages;
+  static constexpr int kOffM = kOffW + 2 * 128 * 4;                // pool mask [2][kMaskTokens][256 keys] f16
+  static constexpr int kOffBar = kOffM + 2 * kMaskTokens * 256 * 2;
+  static constexpr int kBarKFull = 0;                     // [1]
+  static constexpr int kBarKEmpty = 1;                    // [1]
+  static constexpr int kBarQFull = 2;                     // [kQStages]
+  static constexpr int kBarQEmpty = 2 + kQStages;         // [kQStages]
+  static constexpr int kBarAccFull = 2 + 2 * kQStages;    // [2] an item's two accumulators
+  static constexpr int kBarAccFree = 4 + 2 * kQStages;    // [2] ... free, and its weights and mask read
+  static constexpr int kBarAuxFull = 6 + 2 * kQStages;    // [2] weights and mask of an item landed
+  static constexpr int kBarMmaDone = 8 + 2 * kQStages;    // [1]
+  static constexpr int kNumBars = 9 + 2 * kQStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // +1024: manual 1 KB alignment
-  static constexpr int kEpiWarps = 8;                      // two per TMEM lane quarter
-  static constexpr int kThreads = 32 * (kEpiWarps + 2);
-  static constexpr int kProducerWarp = kEpiWarps;
+  static constexpr int kEpiWarps = 16;                     // four per TMEM lane quarter
+  static constexpr int kThreads = 32 * (kEpiWarps + 3);
+  static constexpr int kProducerWarp = kEpiWarps;   // key and query tiles
   static constexpr int kMmaWarp = kEpiWarps + 1;
-  static constexpr uint32_t kTmemCols = 256;  // two 128-column accumulators
+  static constexpr int kAuxWarp = kEpiWarps + 2;    // head weights and mask tiles
+  static constexpr uint32_t kTmemCols = 512;        // two items in flight x two 128-column accumulators
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
-// Item -> (b, key tile, token tile); the items of one key tile are consecutive, and
-// each CTA takes a contiguous range of items, so it loads a key tile once for all
-// the token tiles of that range.
+// Item -> (b, pair of key tiles, token tile); the items of one pair are consecutive, and
+// each CTA takes a contiguous range of items, so it loads a pair once for all the token
+// tiles of that range, and every query tile it loads serves 256 keys.
 struct IndexerItem {
-  int b, pt, tt;
+  int b, pp, tt;
 };
 
 __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int item) {
   IndexerItem it;
   it.tt = item % p.n_ttiles;
   const int bp = item / p.n_ttiles;
-  it.pt = bp % p.n_ptiles;
-  it.b = bp / p.n_ptiles;
+  it.pp = bp % p.n_pairs;
+  it.b = bp / p.n_pairs;
   return it;
+}
+
+// the item after it, without divisions
+__device__ __forceinline__ void indexer_next(const IndexerParams& p, IndexerItem& it) {
+  if (++it.tt == p.n_ttiles) {
+    it.tt = 0;
+    if (++it.pp == p.n_pairs) {
+      it.pp = 0;
+      ++it.b;
+    }
+  }
 }
 
 // Asynchronous 4-byte global -> shared copy (the LDGSTS path); bytes past src_bytes are
@@ -107,40 +122,43 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Epilogue of the score kernel: eight warps, thread = key (TMEM lane) of the tile; warp w
-// reads lanes 32 (w % 4) .. + 31 and accumulator columns 64 (w / 4) .. + 63.  H = 2^LGH heads,
-// so the 128 columns are 128 / H tokens of H heads each (column = token * H + head) and a
-// token's score is the weighted sum of its H rectified columns.  At H = 128 one token spans
-// all columns, and warps 0-3 take them all.  The head weights and the mask rows of the item
-// were put in shared memory by the producer warp; an aligned mask came by TMA, any other
-// is read from global memory here.
+// Epilogue of the score kernel: sixteen warps, thread = key (TMEM lane) of a tile.  Warp w
+// reads lanes 32 (w % 4) .. + 31 of the accumulator of key tile (w / 8) of the pair, columns
+// 64 ((w / 4) % 2) .. + 63.  H = 2^LGH heads, so the 128 columns are 128 / H tokens of H heads
+// each (column = token * H + head) and a token's score is the weighted sum of its H
+// rectified columns.  At H = 128 one token spans all 128 columns: the warp at column 0 takes
+// them all and the other only keeps the barrier count.  The head weights and the mask rows
+// of the item were put in shared memory by the auxiliary-load warp; the mask came by TMA
+// when its rows are 16-byte aligned and a tile has at most 32 tokens (H >= 4), else it is
+// read from global memory here.
 template <int D, int LGH>
 __device__ __forceinline__ void indexer_epilogue(const IndexerParams& p, uint8_t* smem, uint32_t tmem,
                                                  uint64_t* bars, const WaitCtx& wctx, int item0,
                                                  int item1) {
   using C = IndexerCfg<D>;
   constexpr int H = 1 << LGH;
-  constexpr int TPT = 128 / H;  // tokens per tile
+  constexpr int TPT = 128 / H;            // tokens per tile
+  constexpr int kSpan = H > 64 ? H : 64;  // columns one warp reduces
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = (warp & 3) * 32 + lane;  // key of the tile
+  const int kt = warp >> 3;                 // key tile of the pair
+  const int r = (warp & 3) * 32 + lane;     // key within the tile
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const int c_begin = LGH == 7 ? 0 : (warp >> 2) * 64;
-  const int c_end = LGH == 7 ? ((warp >> 2) == 0 ? 128 : 0) : c_begin + 64;
+  const int c_begin = ((warp >> 2) & 1) * 64;
+  const int c_end = (c_begin % kSpan) == 0 ? c_begin + kSpan : c_begin;
   const float* wbuf = reinterpret_cast<const float*>(smem + C::kOffW);        // [2][128]
-  const uint16_t* mbuf = reinterpret_cast<const uint16_t*>(smem + C::kOffM);  // [2][128 tokens][128 keys]
+  const uint16_t* mbuf = reinterpret_cast<const uint16_t*>(smem + C::kOffM);  // [2][kMaskTokens][256 keys]
 
-  int g = 0;
-  for (int item = item0; item < item1; ++item, ++g) {
-    const IndexerItem it = indexer_item(p, item);
-    const int ab = g & 1;
+  IndexerItem it = indexer_item(p, item0);
+  for (int item = item0, g = 0; item < item1; ++item, ++g, indexer_next(p, it)) {
+    const int j = g & 1;  // accumulator pair and weights / mask buffer of this item
     const int t0 = it.tt * TPT;
-    const int key = it.pt * 128 + r;
+    const int key = it.pp * 256 + kt * 128 + r;
     const bool key_ok = key < p.P;
     const bool full = t0 + TPT <= p.T;  // no token of the tile lies past T
     // this key's score for token 0 of the tile; token tl is P floats further on
     float* const srow = p.score + ((long long)it.b * p.T + t0) * p.P + key;
-    const float* wb = wbuf + ab * 128;
-    const uint16_t* mb = mbuf + ab * 128 * 128 + r;
+    const float* wb = wbuf + j * 128;
+    const uint16_t* mb = mbuf + j * C::kMaskTokens * 256 + kt * 128 + r;
     // n scores of consecutive tokens from tl0: the mask values are read before any store,
     // so those reads are not held behind the global stores
     auto emit = [&](int tl0, auto& v) {
@@ -149,78 +167,72 @@ __device__ __forceinline__ void indexer_epilogue(const IndexerParams& p, uint8_t
         float mv[n];
         if (p.mask_tma) {
 #pragma unroll
-          for (int j = 0; j < n; ++j) mv[j] = __half2float(__ushort_as_half(mb[(tl0 + j) * 128]));
+          for (int u = 0; u < n; ++u) mv[u] = __half2float(__ushort_as_half(mb[(tl0 + u) * 256]));
         } else {
           const uint16_t* mrow = p.mask + ((long long)it.b * p.T + t0 + tl0) * p.P + key;
 #pragma unroll
-          for (int j = 0; j < n; ++j)
-            mv[j] = (key_ok && t0 + tl0 + j < p.T) ? __half2float(__ushort_as_half(mrow[(long long)j * p.P])) : 0.f;
+          for (int u = 0; u < n; ++u)
+            mv[u] = (key_ok && t0 + tl0 + u < p.T) ? __half2float(__ushort_as_half(mrow[(long long)u * p.P])) : 0.f;
         }
 #pragma unroll
-        for (int j = 0; j < n; ++j) v[j] += mv[j];
+        for (int u = 0; u < n; ++u) v[u] += mv[u];
       }
       if (!key_ok) return;
       float* dst = srow + (long long)tl0 * p.P;
       if (full) {
 #pragma unroll
-        for (int j = 0; j < n; ++j, dst += p.P) *dst = v[j];
+        for (int u = 0; u < n; ++u, dst += p.P) *dst = v[u];
       } else {
 #pragma unroll
-        for (int j = 0; j < n; ++j, dst += p.P)
-          if (t0 + tl0 + j < p.T) *dst = v[j];
+        for (int u = 0; u < n; ++u, dst += p.P)
+          if (t0 + tl0 + u < p.T) *dst = v[u];
       }
     };
-    mbar_wait(smem_u32(&bars[C::kBarAuxFull + ab]), (g >> 1) & 1, wctx);
-    mbar_wait(smem_u32(&bars[C::kBarAccFull + ab]), (g >> 1) & 1, wctx);
+    mbar_wait(smem_u32(&bars[C::kBarAuxFull + j]), (g >> 1) & 1, wctx);
+    mbar_wait(smem_u32(&bars[C::kBarAccFull + j]), (g >> 1) & 1, wctx);
     __syncwarp();
     tc_fence_after_sync();
+    const uint32_t acc = tmem + lane_base + (uint32_t)(2 * j + kt) * 128u;
     float carry = 0.f;  // H > 32: a token spans several 32-column pieces
 #pragma unroll 1
-    for (int c0 = c_begin; c0 < c_end; c0 += 64) {
-      uint32_t s[2][32];
-      tmem_ld32(tmem + lane_base + ab * 128u + c0, s[0]);
-      tmem_ld32(tmem + lane_base + ab * 128u + c0 + 32, s[1]);
+    for (int cb = c_begin; cb < c_end; cb += 32) {
+      uint32_t sv[32];
+      tmem_ld32(acc + cb, sv);
       tmem_ld_wait();
-      reg_order_after_wait(s[0]);
-      reg_order_after_wait(s[1]);
+      reg_order_after_wait(sv);
+      float wv[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int cb = c0 + half * 32;
-        float wv[32];
+      for (int c = 0; c < 32; c += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(wb + cb + c);
+        wv[c] = w4.x;
+        wv[c + 1] = w4.y;
+        wv[c + 2] = w4.z;
+        wv[c + 3] = w4.w;
+      }
+      if constexpr (H <= 32) {
+        float v[32 / H];
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          const float4 w4 = *reinterpret_cast<const float4*>(wb + cb + c);
-          wv[c] = w4.x;
-          wv[c + 1] = w4.y;
-          wv[c + 2] = w4.z;
-          wv[c + 3] = w4.w;
+        for (int u = 0; u < 32 / H; ++u) {
+          float a = 0.f;
+#pragma unroll
+          for (int h = 0; h < H; ++h) a = fmaf(wv[u * H + h], fmaxf(__uint_as_float(sv[u * H + h]), 0.f), a);
+          v[u] = a;
         }
-        if constexpr (H <= 32) {
-          float v[32 / H];
+        emit(cb >> LGH, v);
+      } else {
 #pragma unroll
-          for (int j = 0; j < 32 / H; ++j) {
-            float a = 0.f;
-#pragma unroll
-            for (int h = 0; h < H; ++h)
-              a = fmaf(wv[j * H + h], fmaxf(__uint_as_float(s[half][j * H + h]), 0.f), a);
-            v[j] = a;
-          }
+        for (int c = 0; c < 32; ++c) carry = fmaf(wv[c], fmaxf(__uint_as_float(sv[c]), 0.f), carry);
+        if (((cb + 32) & (H - 1)) == 0) {
+          float v[1] = {carry};
           emit(cb >> LGH, v);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) carry = fmaf(wv[c], fmaxf(__uint_as_float(s[half][c]), 0.f), carry);
-          if (((cb + 32) & (H - 1)) == 0) {
-            float v[1] = {carry};
-            emit(cb >> LGH, v);
-            carry = 0.f;
-          }
+          carry = 0.f;
         }
       }
     }
-    // accumulator ab, and the weights and mask of buffer ab, are free for item g + 2
+    // accumulators 2j, 2j + 1 and weights / mask buffer j are free for item g + 2
     tc_fence_before_sync();
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&bars[C::kBarAccFree + ab]));
+    if (lane == 0) mbar_arrive(smem_u32(&bars[C::kBarAccFree + j]));
   }
 }
 
@@ -240,17 +252,17 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
-  // this CTA's items: a contiguous range, so consecutive items share a key tile
+  // this CTA's items: a contiguous range, so consecutive items share a pair of key tiles
   const int item0 = blockIdx.x * items_per_cta;
   const int item1 = min(p.n_items, item0 + items_per_cta);
 
   if (threadIdx.x == 0) {
+    mbar_init(BAR(C::kBarKFull), 1);
+    mbar_init(BAR(C::kBarKEmpty), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(BAR(C::kBarKFull + i), 1);
-      mbar_init(BAR(C::kBarKEmpty + i), 1);
       mbar_init(BAR(C::kBarAccFull + i), 1);
       mbar_init(BAR(C::kBarAccFree + i), C::kEpiWarps);  // one arrive per epilogue warp
-      mbar_init(BAR(C::kBarAuxFull + i), 33);  // the byte-count arrive + one cp.async arrive per producer lane
+      mbar_init(BAR(C::kBarAuxFull + i), 33);  // the byte-count arrive + one cp.async arrive per lane
     }
     for (int s = 0; s < C::kQStages; ++s) {
       mbar_init(BAR(C::kBarQFull + s), 1);
@@ -269,35 +281,30 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // key tiles along the item range: the r-th distinct key tile goes to key buffer r & 1
-  auto same_key_tile = [&](const IndexerItem& a, const IndexerItem& b) {
-    return a.b == b.b && a.pt == b.pt;
-  };
+  auto same_pair = [&](const IndexerItem& a, const IndexerItem& b) { return a.b == b.b && a.pp == b.pp; };
 
   if (warp == C::kProducerWarp) {
-    // ======================= producer: TMA tiles, weights, mask =======================
+    // ======================= producer: key-tile pairs and query tiles =======================
     if (lane == 0) {
       tma_prefetch_map(&p.tm_q);
       tma_prefetch_map(&p.tm_k);
-      if (p.mask_tma) tma_prefetch_map(&p.tm_mask);
     }
-    const int tpt = p.tok_per_tile;
-    const uint32_t mask_bytes = p.mask_tma ? (uint32_t)tpt * 128u * 2u : 0u;
-    int nk = 0;  // key tiles loaded
+    int nk = 0;  // pairs loaded
     int nq = 0;  // query tiles loaded
-    int na = 0;  // weight / mask buffers loaded
     IndexerItem prev{-1, -1, -1};
-    for (int item = item0, g = 0; item < item1; ++item, ++g) {
-      const IndexerItem it = indexer_item(p, item);
-      if (!same_key_tile(it, prev)) {
-        const int kb = nk & 1;
-        if (nk >= 2) mbar_wait(BAR(C::kBarKEmpty + kb), ((nk >> 1) - 1) & 1, wctx);
+    IndexerItem it = indexer_item(p, item0);
+    for (int item = item0, g = 0; item < item1; ++item, ++g, indexer_next(p, it)) {
+      if (!same_pair(it, prev)) {
+        // one buffer: a new pair waits until the MMAs are done with the previous one (once
+        // or twice per CTA).  The second tile of the last pair may lie past P: TMA fills zeros.
+        if (nk >= 1) mbar_wait(BAR(C::kBarKEmpty), (nk - 1) & 1, wctx);
         __syncwarp();
         if (warp_flag(abort_flag)) break;
-        mbar_arrive_expect_tx_w(BAR(C::kBarKFull + kb), C::kTileBytes);
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d_w(sbase + C::kOffK + kb * C::kTileBytes + bx * C::kBoxBytes, &p.tm_k,
-                        BAR(C::kBarKFull + kb), bx * 64, it.pt * 128, it.b);
+        mbar_arrive_expect_tx_w(BAR(C::kBarKFull), 2 * C::kTileBytes);
+        for (int kt = 0; kt < 2; ++kt)
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d_w(sbase + C::kOffK + kt * C::kTileBytes + bx * C::kBoxBytes, &p.tm_k,
+                          BAR(C::kBarKFull), bx * 64, (it.pp * 2 + kt) * 128, it.b);
         ++nk;
         prev = it;
       }
@@ -310,8 +317,23 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
         tma_load_3d_w(sbase + C::kOffQ + st * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
                       BAR(C::kBarQFull + st), bx * 64, it.tt * 128, it.b);
       ++nq;
-      // weights and mask of this item into buffer g & 1, free once the epilogue is done
-      // with item g - 2
+    }
+    if (lane == 0 && *abort_flag) {
+      // let every copy this warp started land before the CTA can exit
+      for (int i = max(0, nq - C::kQStages); i < nq; ++i)
+        mbar_wait_drain(BAR(C::kBarQFull + i % C::kQStages), (i / C::kQStages) & 1, p.timeout_ns);
+      if (nk > 0) mbar_wait_drain(BAR(C::kBarKFull), (nk - 1) & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == C::kAuxWarp) {
+    // ======================= head weights and mask tiles =======================
+    // item g's into buffer g & 1, free once the epilogue is done with item g - 2
+    if (lane == 0 && p.mask_tma) tma_prefetch_map(&p.tm_mask);
+    const int tpt = p.tok_per_tile;
+    const uint32_t mask_bytes = p.mask_tma ? (uint32_t)tpt * 256u * 2u : 0u;
+    int na = 0;  // buffers loaded
+    IndexerItem it = indexer_item(p, item0);
+    for (int item = item0, g = 0; item < item1; ++item, ++g, indexer_next(p, it)) {
       const int xb = g & 1;
       if (g >= 2) mbar_wait(BAR(C::kBarAccFree + xb), ((g >> 1) - 1) & 1, wctx);
       __syncwarp();
@@ -319,8 +341,8 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
       const int t0 = it.tt * tpt;
       mbar_arrive_expect_tx_w(BAR(C::kBarAuxFull + xb), mask_bytes);
       if (p.mask_tma)
-        tma_load_3d_w(sbase + C::kOffM + xb * (128 * 128 * 2), &p.tm_mask, BAR(C::kBarAuxFull + xb),
-                      it.pt * 128, t0, it.b);
+        tma_load_3d_w(sbase + C::kOffM + xb * (C::kMaskTokens * 256 * 2), &p.tm_mask, BAR(C::kBarAuxFull + xb),
+                      it.pp * 256, t0, it.b);
       const float* wrow = p.w + ((long long)it.b * p.T) * p.H;
 #pragma unroll
       for (int c = lane; c < 128; c += 32) {  // column c: token c / H, head c % H
@@ -334,11 +356,6 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
     }
     cp_async_wait_all();
     if (lane == 0 && *abort_flag) {
-      // let every copy this warp started land before the CTA can exit
-      for (int i = max(0, nq - C::kQStages); i < nq; ++i)
-        mbar_wait_drain(BAR(C::kBarQFull + i % C::kQStages), (i / C::kQStages) & 1, p.timeout_ns);
-      for (int i = max(0, nk - 2); i < nk; ++i)
-        mbar_wait_drain(BAR(C::kBarKFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
       for (int i = max(0, na - 2); i < na; ++i)
         mbar_wait_drain(BAR(C::kBarAuxFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
     }
@@ -348,41 +365,43 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
     constexpr uint32_t idesc = make_idesc_f16(128, 128, BF16, false);  // Kp Q^T, both K-major
     int nk = 0, g = 0;
     IndexerItem prev{-1, -1, -1};
-    for (int item = item0; item < item1; ++item, ++g) {
-      const IndexerItem it = indexer_item(p, item);
-      const bool new_key = !same_key_tile(it, prev);
-      if (new_key) {
-        if (nk > 0) tc_commit_w(BAR(C::kBarKEmpty + ((nk - 1) & 1)));  // previous key tile released
-        mbar_wait(BAR(C::kBarKFull + (nk & 1)), (nk >> 1) & 1, wctx);
+    IndexerItem it = indexer_item(p, item0);
+    for (int item = item0; item < item1; ++item, ++g, indexer_next(p, it)) {
+      if (!same_pair(it, prev)) {
+        if (nk > 0) tc_commit_w(BAR(C::kBarKEmpty));  // the previous pair is released
+        mbar_wait(BAR(C::kBarKFull), nk & 1, wctx);
         ++nk;
         prev = it;
       }
       const int st = g % C::kQStages;
-      const int ab = g & 1;
+      const int j = g & 1;
       mbar_wait(BAR(C::kBarQFull + st), (g / C::kQStages) & 1, wctx);
-      if (g >= 2) mbar_wait(BAR(C::kBarAccFree + ab), ((g >> 1) - 1) & 1, wctx);
+      if (g >= 2) mbar_wait(BAR(C::kBarAccFree + j), ((g >> 1) - 1) & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
-        const uint32_t sK = sbase + C::kOffK + ((nk - 1) & 1) * C::kTileBytes;
         const uint32_t sQ = sbase + C::kOffQ + st * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // 16 head-dim elements per k-step
-          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-          mma_f16_ss_w(tmem + ab * 128u, make_sdesc_sw128(sK + off, 16, 1024),
-                       make_sdesc_sw128(sQ + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        for (int kt = 0; kt < 2; ++kt) {
+          const uint32_t sK = sbase + C::kOffK + kt * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // 16 head-dim elements per k-step
+            const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+            mma_f16_ss_w(tmem + (uint32_t)(2 * j + kt) * 128u, make_sdesc_sw128(sK + off, 16, 1024),
+                         make_sdesc_sw128(sQ + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          }
         }
-        tc_commit_w(BAR(C::kBarAccFull + ab));
+        tc_commit_w(BAR(C::kBarAccFull + j));
         tc_commit_w(BAR(C::kBarQEmpty + st));
       }
     }
-    if (nk > 0) tc_commit_w(BAR(C::kBarKEmpty + ((nk - 1) & 1)));
+    if (nk > 0) tc_commit_w(BAR(C::kBarKEmpty));
     // every MMA (and every commit arrive) has landed before TMEM is released
     tc_commit_w(BAR(C::kBarMmaDone));
     mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    // ======================= epilogue warps 0-7 (thread = pooled key) ===========
+    // ======================= epilogue warps 0-15 (thread = pooled key) ===========
     switch (p.lg_h) {  // the head count fixes how columns group into tokens
       case 0: indexer_epilogue<D, 0>(p, smem, tmem, bars, wctx, item0, item1); break;
       case 1: indexer_epilogue<D, 1>(p, smem, tmem, bars, wctx, item0, item1); break;
