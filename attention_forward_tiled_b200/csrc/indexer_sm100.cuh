@@ -11,14 +11,14 @@
 // (token, head) pairs of 128 / H tokens its N = 128 columns, so the product lands
 // in TMEM with one thread per key holding every head of every token of the tile:
 // the rectifier, the head weights and the head sum stay inside a thread.  Work
-// items (b, key tile, token tile) go to persistent CTAs (608 threads):
-//   * warp 16, producer: TMA loads of a pair of key tiles (once per run of items on the
+// items (b, pair of key tiles, token tile) go to persistent CTAs (352 threads):
+//   * warp 8, producer: TMA loads of a pair of key tiles (once per run of items on the
 //     same pair) and of the query tiles (a four-deep ring) into shared memory;
-//   * warp 18, auxiliary loads: the item's mask tile by TMA and its head weights by
+//   * warp 10, auxiliary loads: the item's mask tile by TMA and its head weights by
 //     cp.async, double-buffered;
-//   * warp 17, MMA issuer: S^T = Kp Q^T for both key tiles of the pair (two TMEM
+//   * warp 9, MMA issuer: S^T = Kp Q^T for both key tiles of the pair (two TMEM
 //     accumulators per item, two items in flight), so each query tile serves 256 keys;
-//   * warps 0-15, epilogue: rectify, weight, sum over heads, add the f16 mask and
+//   * warps 0-7, epilogue: rectify, weight, sum over heads, add the f16 mask and
 //     store fp32 scores (one thread per key: consecutive keys, coalesced stores).
 //
 // Top-k (prhub.com.cn report "PR #45743 完整报告", section "实现拆解": the decode
@@ -73,7 +73,7 @@ struct IndexerCfg {
   static constexpr int kNumBars = 9 + 2 * kQStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // +1024: manual 1 KB alignment
-  static constexpr int kEpiWarps = 16;                     // four per TMEM lane quarter
+  static constexpr int kEpiWarps = 8;                      // one per (key tile, TMEM lane quarter)
   static constexpr int kThreads = 32 * (kEpiWarps + 3);
   static constexpr int kProducerWarp = kEpiWarps;   // key and query tiles
   static constexpr int kMmaWarp = kEpiWarps + 1;
@@ -122,12 +122,11 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Epilogue of the score kernel: sixteen warps, thread = key (TMEM lane) of a tile.  Warp w
-// reads lanes 32 (w % 4) .. + 31 of the accumulator of key tile (w / 8) of the pair, columns
-// 64 ((w / 4) % 2) .. + 63.  H = 2^LGH heads, so the 128 columns are 128 / H tokens of H heads
-// each (column = token * H + head) and a token's score is the weighted sum of its H
-// rectified columns.  At H = 128 one token spans all 128 columns: the warp at column 0 takes
-// them all and the other only keeps the barrier count.  The head weights and the mask rows
+// Epilogue of the score kernel: eight warps, thread = key (TMEM lane) of a tile.  Warp w
+// reads lanes 32 (w % 4) .. + 31 of the accumulator of key tile (w / 4) of the pair, all 128
+// columns.  H = 2^LGH heads, so the columns are 128 / H tokens of H heads each (column =
+// token * H + head) and a token's score is the weighted sum of its H rectified columns
+// (carried across 32-column pieces when H > 32).  The head weights and the mask rows
 // of the item were put in shared memory by the auxiliary-load warp; the mask came by TMA
 // when its rows are 16-byte aligned and a tile has at most 32 tokens (H >= 4), else it is
 // read from global memory here.
@@ -138,13 +137,10 @@ __device__ __forceinline__ void indexer_epilogue(const IndexerParams& p, uint8_t
   using C = IndexerCfg<D>;
   constexpr int H = 1 << LGH;
   constexpr int TPT = 128 / H;            // tokens per tile
-  constexpr int kSpan = H > 64 ? H : 64;  // columns one warp reduces
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = warp >> 3;                 // key tile of the pair
+  const int kt = warp >> 2;                 // key tile of the pair
   const int r = (warp & 3) * 32 + lane;     // key within the tile
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const int c_begin = ((warp >> 2) & 1) * 64;
-  const int c_end = (c_begin % kSpan) == 0 ? c_begin + kSpan : c_begin;
   const float* wbuf = reinterpret_cast<const float*>(smem + C::kOffW);        // [2][128]
   const uint16_t* mbuf = reinterpret_cast<const uint16_t*>(smem + C::kOffM);  // [2][kMaskTokens][256 keys]
 
@@ -194,12 +190,15 @@ __device__ __forceinline__ void indexer_epilogue(const IndexerParams& p, uint8_t
     tc_fence_after_sync();
     const uint32_t acc = tmem + lane_base + (uint32_t)(2 * j + kt) * 128u;
     float carry = 0.f;  // H > 32: a token spans several 32-column pieces
-#pragma unroll 1
-    for (int cb = c_begin; cb < c_end; cb += 32) {
-      uint32_t sv[32];
-      tmem_ld32(acc + cb, sv);
+    // four 32-column pieces; the TMEM load of piece i + 1 is in flight while piece i is reduced
+    uint32_t sv[2][32];
+    tmem_ld32(acc, sv[0]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int cb = i * 32;
       tmem_ld_wait();
-      reg_order_after_wait(sv);
+      reg_order_after_wait(sv[i & 1]);
+      if (i < 3) tmem_ld32(acc + cb + 32, sv[(i + 1) & 1]);
       float wv[32];
 #pragma unroll
       for (int c = 0; c < 32; c += 4) {
@@ -210,18 +209,24 @@ __device__ __forceinline__ void indexer_epilogue(const IndexerParams& p, uint8_t
         wv[c + 3] = w4.w;
       }
       if constexpr (H <= 32) {
-        float v[32 / H];
+        constexpr int NT = 32 / H;          // tokens in the piece
+        constexpr int G = NT < 8 ? NT : 8;  // ... emitted eight at a time
 #pragma unroll
-        for (int u = 0; u < 32 / H; ++u) {
-          float a = 0.f;
+        for (int u0 = 0; u0 < NT; u0 += G) {
+          float v[G];
 #pragma unroll
-          for (int h = 0; h < H; ++h) a = fmaf(wv[u * H + h], fmaxf(__uint_as_float(sv[u * H + h]), 0.f), a);
-          v[u] = a;
+          for (int u = 0; u < G; ++u) {
+            float a = 0.f;
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+              a = fmaf(wv[(u0 + u) * H + h], fmaxf(__uint_as_float(sv[i & 1][(u0 + u) * H + h]), 0.f), a);
+            v[u] = a;
+          }
+          emit((cb >> LGH) + u0, v);
         }
-        emit(cb >> LGH, v);
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) carry = fmaf(wv[c], fmaxf(__uint_as_float(sv[c]), 0.f), carry);
+        for (int c = 0; c < 32; ++c) carry = fmaf(wv[c], fmaxf(__uint_as_float(sv[i & 1][c]), 0.f), carry);
         if (((cb + 32) & (H - 1)) == 0) {
           float v[1] = {carry};
           emit(cb >> LGH, v);
@@ -401,7 +406,7 @@ __global__ void __launch_bounds__(IndexerCfg<D>::kThreads, 1)
     mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    // ======================= epilogue warps 0-15 (thread = pooled key) ===========
+    // ======================= epilogue warps 0-7 (thread = pooled key) ===========
     switch (p.lg_h) {  // the head count fixes how columns group into tokens
       case 0: indexer_epilogue<D, 0>(p, smem, tmem, bars, wctx, item0, item1); break;
       case 1: indexer_epilogue<D, 1>(p, smem, tmem, bars, wctx, item0, item1); break;
