@@ -591,9 +591,12 @@ __global__ void __launch_bounds__(kTopkThreads)
     cidx[i] = 0x7fffffff;
   }
   __syncthreads();
-  // ---- bitonic sort: key descending, then position ascending
+  // ---- bitonic sort: key descending, then position ascending.  Stages whose partner is
+  // 32 or more elements away go through shared memory; the rest of each merge (strides 16
+  // down to 1) runs in registers with warp shuffles, one element per thread and slot.
   for (int size = 2; size <= kp2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+    int stride = size >> 1;
+    for (; stride >= 32; stride >>= 1) {
       for (int i = tid; i < kp2; i += kTopkThreads) {
         const int j = i ^ stride;
         if (j > i) {
@@ -611,6 +614,31 @@ __global__ void __launch_bounds__(kTopkThreads)
       }
       __syncthreads();
     }
+#pragma unroll 1
+    for (int i0 = 0; i0 < kp2; i0 += kTopkThreads) {  // whole warps: kp2 is a power of two
+      const int i = i0 + tid;
+      const bool active = i < kp2;
+      uint32_t kx = active ? ckey[i] : 0u;
+      int ix = active ? cidx[i] : 0;
+      const bool desc = (i & size) == 0;
+      for (int st = stride; st >= 1; st >>= 1) {
+        const uint32_t ky = __shfl_xor_sync(0xffffffffu, kx, st);
+        const int iy = __shfl_xor_sync(0xffffffffu, ix, st);
+        const bool y_first = ky > kx || (ky == kx && iy < ix);
+        const bool lower = (i & st) == 0;
+        // the lower element of the pair keeps the one that comes first in this block's
+        // order, the upper one the other
+        if (lower == (desc == y_first)) {
+          kx = ky;
+          ix = iy;
+        }
+      }
+      if (active) {
+        ckey[i] = kx;
+        cidx[i] = ix;
+      }
+    }
+    __syncthreads();
   }
   int* out = idx + (long long)row * k;
   for (int i = tid; i < k; i += kTopkThreads) out[i] = (i < nsel) ? cidx[i] : -1;
