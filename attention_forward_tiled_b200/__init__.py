@@ -8,11 +8,11 @@ back to anything else.  ``inputs`` holds the seeded synthetic workloads.
 """
 from ._binding import (ATTN_BF16, ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_RANGE, ATTN_ERR_TIMEOUT,
                        ATTN_ERR_UNSUPPORTED, ATTN_F16, ATTN_OK, LIB_PATH, SIGNATURES, AttnError,
-                       HostRunner, attn_bwd, attn_fwd, attn_fwd_decode_paged, attn_fwd_paged, debug_set, error_string,
+                       HostRunner, attn_bwd, attn_fwd, attn_fwd_decode_paged, attn_fwd_paged, attn_fwd_relpos, debug_set, error_string,
                        get_status, indexer_score, load_library, topk, version)
 
 __all__ = [
-    "attn_fwd", "attn_bwd", "attn_fwd_decode_paged", "attn_fwd_paged", "indexer_score", "topk", "get_status", "error_string", "version", "debug_set", "load_library",
+    "attn_fwd", "attn_bwd", "attn_fwd_decode_paged", "attn_fwd_paged", "attn_fwd_relpos", "indexer_score", "topk", "get_status", "error_string", "version", "debug_set", "load_library",
     "HostRunner", "AttnError", "LIB_PATH", "SIGNATURES", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_RANGE", "ATTN_F16", "ATTN_BF16",
 ]

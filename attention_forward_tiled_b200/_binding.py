@@ -31,6 +31,7 @@ SIGNATURES = {
                                    _i, _vp]),
     "attn_fwd_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                             _i, _i, _vp]),
+    "attn_fwd_relpos": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_indexer_score": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "attn_topk": (_i, [_vp, _i, _i, _i, _vp, _vp]),
@@ -159,6 +160,39 @@ def attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_lse=T
             raise ValueError(f"unknown path {path!r}")
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_relpos(q, k, v, emb, R, causal=False, scale=None, out=None, lse=None, return_lse=True,
+                    stream=None):
+    """Attention whose scores carry the relative-position term scale * q_i . emb[dist(i, j)],
+    dist(i, j) = clamp(i - j, -R, R) + R (emb [n_emb, d] in q's dtype, n_emb >= 2R + 1).
+
+    q, k, v [B, N, H, d] as attn_fwd (B may be batch x blocks of a block-local model).
+    Returns (out, lse) as attn_fwd."""
+    import torch
+    lib = load_library()
+    B, H, Nq, Nk, d = _check(q, k, v)
+    if emb.dim() != 2 or emb.shape[1] != d or emb.dtype != q.dtype or emb.device != q.device:
+        raise ValueError("emb must be [n_emb, d] in q's dtype on q's device")
+    if not emb.is_contiguous():
+        raise ValueError("emb must be contiguous")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_buffer("lse", lse, (B, H, Nq), torch.float32, q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.attn_fwd_relpos(
+            ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+            ctypes.c_void_p(emb.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+            ctypes.c_void_p(lse.data_ptr() if lse is not None else 0), B, H, Nq, Nk, d, emb.shape[0],
+            int(R), int(bool(causal)), scale, _dtype_code(q.dtype), _stream_ptr(stream, q.device))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_relpos")
     return out, lse
 
 

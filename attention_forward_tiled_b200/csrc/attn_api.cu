@@ -18,6 +18,7 @@
 
 #include "attn.h"
 #include "backward_sm100.cuh"
+#include "relpos_sm100.cuh"
 #include "decode_mq_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "indexer_sm100.cuh"
@@ -53,7 +54,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int* status_ptr = nullptr;
-  bool attr_set[28] = {};  // per kernel instantiation: max dynamic shared memory raised
+  bool attr_set[32] = {};  // per kernel instantiation: max dynamic shared memory raised
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -542,6 +543,38 @@ int launch_indexer(DeviceState* ds, const void* q, const void* kp, const float* 
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+
+// Relative-position attention: one CTA per (128-query tile, head, batch).
+template <int D, bool BF16>
+int launch_relpos(DeviceState* ds, const void* q, const void* k, const void* v, const void* emb, void* out,
+                  float* lse, int B, int H, int Nq, int Nk, int n_emb, int R, int causal, float scale,
+                  cudaStream_t stream) {
+  using C = RelposCfg<D>;
+  auto kernel = attn_relpos_kernel<D, BF16>;
+  const int slot = 28 + (D == 128 ? 0 : 1) + (BF16 ? 2 : 0);
+  if (int rc = ensure_smem_attr(ds, slot, kernel, C::kSmemBytes)) return rc;
+  RelposParams p;
+  const int dtype = BF16 ? ATTN_BF16 : ATTN_F16;
+  if (int rc = encode_bnhd(&p.tm_q, q, B, Nq, H, D, dtype, 128)) return rc;
+  if (int rc = encode_bnhd(&p.tm_k, k, B, Nk, H, D, dtype, 64)) return rc;
+  if (int rc = encode_bnhd(&p.tm_v, v, B, Nk, H, D, dtype, 64)) return rc;
+  if (int rc = encode_rows3d(&p.tm_e, emb, 1, n_emb, D, dtype)) return rc;
+  p.out = out;
+  p.lse = lse;
+  p.status = ds->status_ptr;
+  p.B = B;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.R = R;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  const dim3 grid((unsigned)((Nq + 127) / 128), (unsigned)H, (unsigned)B);
+  kernel<<<grid, dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // Backward: D = rowsum(dO o O) and a zeroed fp32 dQ accumulator, the tiled gradient
 // kernel, then dQ = scale * accumulator cast to the input type.  Workspace taken
 // stream-ordered from the default pool and returned on the same stream.
@@ -802,6 +835,29 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
     return bf16 ? launch_bwd<128, true>(ATTN_BWD_ARGS) : launch_bwd<128, false>(ATTN_BWD_ARGS);
   return bf16 ? launch_bwd<64, true>(ATTN_BWD_ARGS) : launch_bwd<64, false>(ATTN_BWD_ARGS);
 #undef ATTN_BWD_ARGS
+}
+
+int attn_fwd_relpos(const void* q, const void* k, const void* v, const void* emb, void* out, float* lse,
+                    int B, int H, int Nq, int Nk, int d, int n_emb, int R, int causal, float scale,
+                    int dtype, attn_stream_t stream) {
+  if (int rc = validate(q, k, v, out, lse, B, H, Nq, Nk, d, causal, scale, dtype)) return rc;
+  if (!emb || R < 0 || n_emb < 2 * (long long)R + 1) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(emb) % 16 != 0) return ATTN_ERR_INVALID_ARG;
+  if ((unsigned long long)n_emb * d * 2 >= (1ull << 40)) return ATTN_ERR_INVALID_ARG;
+  if (Nq > 65535 * 128 || H > 65535 || B > 65535) return ATTN_ERR_INVALID_ARG;  // grid limits
+  const size_t q_bytes = (size_t)B * Nq * H * d * 2;
+  if (overlaps(out, q_bytes, emb, (size_t)n_emb * d * 2) ||
+      (lse && overlaps(lse, (size_t)B * H * Nq * 4, emb, (size_t)n_emb * d * 2)))
+    return ATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_BF16;
+#define ATTN_RELPOS_ARGS ds, q, k, v, emb, out, lse, B, H, Nq, Nk, n_emb, R, causal, scale, st
+  if (d == 128)
+    return bf16 ? launch_relpos<128, true>(ATTN_RELPOS_ARGS) : launch_relpos<128, false>(ATTN_RELPOS_ARGS);
+  return bf16 ? launch_relpos<64, true>(ATTN_RELPOS_ARGS) : launch_relpos<64, false>(ATTN_RELPOS_ARGS);
+#undef ATTN_RELPOS_ARGS
 }
 
 int attn_indexer_score(const void* q, const void* kp, const float* w, const void* mask, float* score,

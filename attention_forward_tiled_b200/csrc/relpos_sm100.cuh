@@ -1,0 +1,434 @@
+// relpos_sm100.cuh -- attention with a fused relative-position score term (sm_100a).
+//
+// vLLM page "PR #42933" (Granite-Speech conformer block attention), sections "实现拆解"
+// and "关键源码片段": the attention scores of a block carry, besides q_i . k_j, the term
+// q_i . emb[dist[i, j]] (the einsum "bnhid,ijd->bnhij" of the queries with the gathered
+// relative-position embeddings), both multiplied by the scale, before masking and the
+// softmax.  The distance table is the conformer's clamped relative distance,
+//   dist[i, j] = clamp(i - j, -R, R) + R,     emb row R = distance 0,
+// so the kernel takes R and never reads a table.
+//
+// One CTA per (b, h, 128-query tile); keys in steps of 64.  For a step the distances met
+// span at most 191 consecutive embedding rows (lo ... lo + 190, clamped at 0 and 2R), so
+// the tensor core computes G^T = E_win Q^T (two M = 128 products over 256 rows of the
+// window: TMEM lane = embedding row, column = query row) next to S = Q K^T.  The softmax
+// warps copy G^T to shared memory as Gs[c][row] with a 132-word row pitch and gather
+// bias[i, j] = Gs[dist(i, j) - lo][i]: a warp's 32 query rows read 32 different words of
+// different banks at every key (the 132 pitch makes the skewed read conflict-free), and a
+// thread keeps its own row in registers for nothing.  Roles (192 threads):
+//   * warp 4, producer: Q once, the K/V ring (two stages), the embedding window per step;
+//   * warp 5, MMA issuer: S and G of step t, then O += P V of step t - 1 once P is ready;
+//   * warps 0-3, softmax (thread = query row): copy G, gather the bias, online softmax
+//     (fp16 P into shared memory, O rescaled in TMEM when the row maximum grows), and the
+//     O / l epilogue.  For bf16 inputs they convert each V tile to fp16 in place first
+//     (P V runs in fp16, as in the plain kernel; magnitudes with no fp16 value set the
+//     range status).
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace attn_b200 {
+
+struct RelposParams {
+  CUtensorMap tm_q;  // q [B, Nq, H, D] as 4-D (D, H, Nq, B), box (64, 1, 128, 1), 128B swizzle
+  CUtensorMap tm_k;  // k [B, Nk, H, D] as 4-D (D, H, Nk, B), box (64, 1, 64, 1)
+  CUtensorMap tm_v;  // v, as k
+  CUtensorMap tm_e;  // emb [n_emb, D] as 3-D (D, n_emb, 1), box (64, 128, 1)
+  void* out;         // [B, Nq, H, D], the input dtype
+  float* lse;        // [B, H, Nq] natural log, or nullptr
+  int* status;
+  int B, H, Nq, Nk, R, causal;
+  float scale_log2;  // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct RelposCfg {
+  static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kQBytes = kBoxes * 128 * 128;   // 128 rows x D
+  static constexpr int kKVBytes = kBoxes * 64 * 128;   // 64 rows x D
+  static constexpr int kEBytes = 2 * kBoxes * 128 * 128;  // 256 embedding rows x D
+  static constexpr int kGsPitch = 132;                 // words per embedding row of Gs
+  static constexpr int kGsRows = 192;                  // rows a step can need (191) rounded up
+  static constexpr int kGsBytes = kGsRows * kGsPitch * 4;
+  static constexpr int kWinBytes = kEBytes > kGsBytes ? kEBytes : kGsBytes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;         // [2]
+  static constexpr int kOffV = kOffK + 2 * kKVBytes;    // [2]
+  static constexpr int kOffP = kOffV + 2 * kKVBytes;    // 128 x 64 fp16, 128B swizzle
+  static constexpr int kOffWin = kOffP + 128 * 128;     // embedding window, then Gs
+  static constexpr int kOffBar = kOffWin + kWinBytes;
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarKVFull = 1;   // [2]
+  static constexpr int kBarKVEmpty = 3;  // [2]
+  static constexpr int kBarEFull = 5;
+  static constexpr int kBarGsFree = 6;   // the softmax warps are done reading Gs (4 arrivals)
+  static constexpr int kBarSFull = 7;    // S and G of the step are in TMEM
+  static constexpr int kBarSFree = 8;    // ... and have been read (4 arrivals)
+  static constexpr int kBarPFull = 9;    // P written, O rescaled, V converted (4 arrivals)
+  static constexpr int kBarPVDone = 10;  // O += P V of the step has completed
+  static constexpr int kBarMmaDone = 11;
+  static constexpr int kNumBars = 12;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // +1024: manual 1 KB alignment
+  static constexpr int kThreads = 192;
+  static constexpr int kProducerWarp = 4;
+  static constexpr int kMmaWarp = 5;
+  // TMEM columns
+  static constexpr uint32_t kColO = 0;    // D columns
+  static constexpr uint32_t kColS = 128;  // 64 columns
+  static constexpr uint32_t kColG = 256;  // two 128-column accumulators
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+// Keys of the CTA's query tile: steps of 64 up to the last key any of its rows may see.
+__device__ __forceinline__ int relpos_steps(const RelposParams& p, int q0) {
+  int kend = p.Nk;  // one past the last key
+  if (p.causal) {
+    const int last_row = min(q0 + 127, p.Nq - 1);
+    kend = min(p.Nk, last_row + (p.Nk - p.Nq) + 1);
+  }
+  return kend <= 0 ? 0 : (kend + 63) / 64;
+}
+
+// First embedding row a step needs: the smallest clamped distance over the tile.
+__device__ __forceinline__ int relpos_lo(const RelposParams& p, int q0, int k0) {
+  return min(max(q0 - (k0 + 63), -p.R), p.R) + p.R;
+}
+
+
+// Softmax warps 0-3: thread = query row q0 + r of the tile (TMEM lane r).
+template <int D, bool BF16>
+__device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* smem, uint32_t tmem,
+                                               uint64_t* bars, const WaitCtx& wctx, int q0, int h, int b,
+                                               int nsteps) {
+  using C = RelposCfg<D>;
+  auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = threadIdx.x;  // row of the tile
+  const int i = q0 + r;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  float* gs = reinterpret_cast<float*>(smem + C::kOffWin);  // [kGsRows][kGsPitch]
+  uint8_t* sp = smem + C::kOffP;
+  const int shift = p.Nk - p.Nq;  // bottom-right causal alignment
+  float m = -INFINITY;            // running maximum of scale * log2(e) * score
+  float l0 = 0.f, l1 = 0.f;       // sum of the fp16-rounded P the tensor core multiplies
+  uint32_t vmag = 0;              // bf16: largest |V| bit pattern converted
+
+  for (int t = 0; t < nsteps; ++t) {
+    const int k0 = t * 64;
+    const int lo = relpos_lo(p, q0, k0);
+    const int hi = min(max(q0 + 127 - k0, -p.R), p.R) + p.R;
+    const int n_off = hi - lo + 1;  // embedding rows this step uses (<= 191)
+    mbar_wait(BAR(C::kBarSFull), t & 1, wctx);
+    __syncwarp();
+    tc_fence_after_sync();
+    // ---- G^T (lane = embedding row) -> Gs[row][query row]; the loads are warp-collective,
+    // so the condition is per warp
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      if (a * 128 + warp * 32 < n_off) {
+        const int c = a * 128 + warp * 32 + lane;  // < 192
+        float* dst = gs + c * C::kGsPitch;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t g[32];
+          tmem_ld32(tmem + lane_base + C::kColG + a * 128 + q * 32, g);
+          tmem_ld_wait();
+          reg_order_after_wait(g);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(dst + q * 32 + 4 * u) =
+                make_float4(__uint_as_float(g[4 * u]), __uint_as_float(g[4 * u + 1]),
+                            __uint_as_float(g[4 * u + 2]), __uint_as_float(g[4 * u + 3]));
+        }
+      }
+    }
+    // ---- this row's 64 raw scores
+    uint32_t sv[2][32];
+    tmem_ld32(tmem + lane_base + C::kColS, sv[0]);
+    tmem_ld32(tmem + lane_base + C::kColS + 32, sv[1]);
+    tmem_ld_wait();
+    reg_order_after_wait(sv[0]);
+    reg_order_after_wait(sv[1]);
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(C::kBarSFree));  // S and G may be overwritten
+    named_bar_sync(1, 128);                          // Gs is complete
+    // ---- add the gathered term, scale, mask
+    float x[64];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int jj = 0; jj < 64; ++jj) {
+      const int j = k0 + jj;
+      const bool allowed = i < p.Nq && j < p.Nk && (!p.causal || j <= i + shift);
+      const int c = min(max(i - j, -p.R), p.R) + p.R - lo;  // in [0, n_off) for every i, j of the tile
+      const float g = gs[c * C::kGsPitch + r];
+      x[jj] = allowed ? (__uint_as_float(sv[jj >> 5][jj & 31]) + g) * p.scale_log2 : -INFINITY;
+      mx = fmaxf(mx, x[jj]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(C::kBarGsFree));  // the window may be reloaded
+    // ---- online softmax: O and the P buffer are free once the previous P V is done
+    const float m_new = fmaxf(m, mx);
+    if (t >= 1) {
+      mbar_wait(BAR(C::kBarPVDone), (t - 1) & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      const bool grow = m_new > m && m > -INFINITY;
+      if (__any_sync(0xffffffffu, grow)) {  // TMEM loads and stores are warp-collective
+        const float f = grow ? ex2_approx(m - m_new) : 1.0f;
+        l0 *= f;
+        l1 *= f;
+#pragma unroll 1
+        for (int cq = 0; cq < D / 32; ++cq) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + C::kColO + cq * 32, o);
+          tmem_ld_wait();
+          reg_order_after_wait(o);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * f);
+          tmem_st32(tmem + lane_base + C::kColO + cq * 32, o);
+        }
+        tmem_st_wait();
+      }
+    }
+    m = m_new;
+    const float mu = m == -INFINITY ? 0.f : m;  // a row that saw no key yet: every P is 0
+    uint32_t pk[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      pk[u] = pack2<false>(ex2_approx(x[2 * u] - mu), ex2_approx(x[2 * u + 1] - mu));
+      add_f16x2_f32(l0, l1, pk[u]);
+    }
+    // P row r: 64 fp16 = eight 16-byte chunks, 128-byte swizzle (K-major A operand)
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc)
+      *reinterpret_cast<uint4*>(sp + r * 128 + ((cc ^ (r & 7)) << 4)) =
+          make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+    if constexpr (BF16) {  // V of this step to fp16, in place
+      mbar_wait(BAR(C::kBarKVFull + (t & 1)), (t >> 1) & 1, wctx);
+      uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffV + (t & 1) * C::kKVBytes);
+#pragma unroll 2
+      for (int c = r; c < C::kKVBytes / 16; c += 128) {
+        uint4 w = tile[c];
+        vmag = __vmaxu2(vmag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                       __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+        w.x = bf16x2_to_f16x2_sat(w.x);
+        w.y = bf16x2_to_f16x2_sat(w.y);
+        w.z = bf16x2_to_f16x2_sat(w.z);
+        w.w = bf16x2_to_f16x2_sat(w.w);
+        tile[c] = w;
+      }
+    }
+    fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(C::kBarPFull));
+  }
+
+  // ---- epilogue: O / l in the input dtype, lse = ln(sum exp(scale * score))
+  const float l = l0 + l1;
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+  const bool row_ok = i < p.Nq;
+  uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
+                                         ((((long long)b * p.Nq + (row_ok ? i : 0)) * p.H + h) * D) * 2);
+  if (nsteps > 0) {
+    mbar_wait(BAR(C::kBarPVDone), (nsteps - 1) & 1, wctx);
+    __syncwarp();
+    tc_fence_after_sync();
+#pragma unroll 1
+    for (int cq = 0; cq < D / 32; ++cq) {
+      uint32_t o[32];
+      tmem_ld32(tmem + lane_base + C::kColO + cq * 32, o);
+      tmem_ld_wait();
+      reg_order_after_wait(o);
+      if (row_ok) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          orow[cq * 4 + u] = make_uint4(
+              pack2<BF16>(__uint_as_float(o[8 * u]) * inv, __uint_as_float(o[8 * u + 1]) * inv),
+              pack2<BF16>(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv),
+              pack2<BF16>(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv),
+              pack2<BF16>(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv));
+      }
+    }
+  } else if (row_ok) {  // no key reaches this tile
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (row_ok && p.lse != nullptr)
+    p.lse[((long long)b * p.H + h) * p.Nq + i] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+  if constexpr (BF16) {
+    if (max(vmag & 0xFFFFu, vmag >> 16) >= kBf16NoF16) atomicCAS(p.status, 0, kStatusRange);
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
+    attn_relpos_kernel(const __grid_constant__ RelposParams p) {
+  using C = RelposCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
+  const int q0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
+  const int nsteps = relpos_steps(p, q0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::kBarQFull), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(C::kBarKVFull + s), 1);
+      mbar_init(BAR(C::kBarKVEmpty + s), 1);
+    }
+    mbar_init(BAR(C::kBarEFull), 1);
+    mbar_init(BAR(C::kBarGsFree), 4);
+    mbar_init(BAR(C::kBarSFull), 1);
+    mbar_init(BAR(C::kBarSFree), 4);
+    mbar_init(BAR(C::kBarPFull), 4);
+    mbar_init(BAR(C::kBarPVDone), 1);
+    mbar_init(BAR(C::kBarMmaDone), 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::kProducerWarp) {
+    // ======================= TMA producer =======================
+    int nkv = 0, ne = 0;
+    if (nsteps > 0) {
+      if (lane == 0) {
+        tma_prefetch_map(&p.tm_q);
+        tma_prefetch_map(&p.tm_k);
+        tma_prefetch_map(&p.tm_v);
+        tma_prefetch_map(&p.tm_e);
+      }
+      mbar_arrive_expect_tx_w(BAR(C::kBarQFull), C::kQBytes);
+      for (int bx = 0; bx < C::kBoxes; ++bx)
+        tma_load_4d_w(sbase + C::kOffQ + bx * 16384, &p.tm_q, BAR(C::kBarQFull), bx * 64, h, q0, b);
+      for (int t = 0; t < nsteps; ++t) {
+        const int s = t & 1, k0 = t * 64;
+        if (t >= 2) mbar_wait(BAR(C::kBarKVEmpty + s), ((t >> 1) - 1) & 1, wctx);
+        __syncwarp();
+        if (warp_flag(abort_flag)) break;
+        mbar_arrive_expect_tx_w(BAR(C::kBarKVFull + s), 2 * C::kKVBytes);
+        for (int bx = 0; bx < C::kBoxes; ++bx) {
+          tma_load_4d_w(sbase + C::kOffK + s * C::kKVBytes + bx * 8192, &p.tm_k, BAR(C::kBarKVFull + s),
+                        bx * 64, h, k0, b);
+          tma_load_4d_w(sbase + C::kOffV + s * C::kKVBytes + bx * 8192, &p.tm_v, BAR(C::kBarKVFull + s),
+                        bx * 64, h, k0, b);
+        }
+        ++nkv;
+        // the window shares its bytes with Gs: wait until the previous step's gather is done
+        if (t >= 1) mbar_wait(BAR(C::kBarGsFree), (t - 1) & 1, wctx);
+        __syncwarp();
+        if (warp_flag(abort_flag)) break;
+        const int lo = relpos_lo(p, q0, k0);
+        mbar_arrive_expect_tx_w(BAR(C::kBarEFull), C::kEBytes);
+        for (int rb = 0; rb < 2; ++rb)
+          for (int bx = 0; bx < C::kBoxes; ++bx)  // rows past n_emb read as zeros and are never used
+            tma_load_3d_w(sbase + C::kOffWin + (rb * C::kBoxes + bx) * 16384, &p.tm_e, BAR(C::kBarEFull),
+                          bx * 64, lo + rb * 128, 0);
+        ++ne;
+      }
+      if (lane == 0 && *abort_flag) {
+        // let every copy this warp started land before the CTA can exit
+        mbar_wait_drain(BAR(C::kBarQFull), 0, p.timeout_ns);
+        for (int i = max(0, nkv - 2); i < nkv; ++i)
+          mbar_wait_drain(BAR(C::kBarKVFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
+        if (ne > 0) mbar_wait_drain(BAR(C::kBarEFull), (ne - 1) & 1, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kMmaWarp) {
+    // ======================= tcgen05 MMA issuer =======================
+    constexpr uint32_t idesc_s = make_idesc_f16(128, 64, BF16, false);   // Q K^T, both K-major
+    constexpr uint32_t idesc_g = make_idesc_f16(128, 128, BF16, false);  // E_win Q^T, both K-major
+    constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);    // P V: fp16, V MN-major
+    auto issue_pv = [&](int t) {
+      mbar_wait(BAR(C::kBarPFull), t & 1, wctx);
+      __syncwarp();
+      tc_fence_after_sync();
+      if (!warp_flag(abort_flag)) {
+        const uint32_t sV = sbase + C::kOffV + (t & 1) * C::kKVBytes;
+        const uint32_t sP = sbase + C::kOffP;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // 16 keys per k-step
+          mma_f16_ss_w(tmem + C::kColO, make_sdesc_sw128(sP + kk * 32, 16, 1024),
+                       make_sdesc_sw128(sV + kk * 2048, 8192, 1024), idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit_w(BAR(C::kBarPVDone));
+        tc_commit_w(BAR(C::kBarKVEmpty + (t & 1)));
+      }
+    };
+    if (nsteps > 0) {
+      mbar_wait(BAR(C::kBarQFull), 0, wctx);
+      for (int t = 0; t < nsteps; ++t) {
+        const int s = t & 1;
+        mbar_wait(BAR(C::kBarKVFull + s), (t >> 1) & 1, wctx);
+        mbar_wait(BAR(C::kBarEFull), t & 1, wctx);
+        if (t >= 1) mbar_wait(BAR(C::kBarSFree), (t - 1) & 1, wctx);
+        __syncwarp();
+        tc_fence_after_sync();
+        if (!warp_flag(abort_flag)) {
+          const uint32_t sQ = sbase + C::kOffQ;
+          const uint32_t sK = sbase + C::kOffK + s * C::kKVBytes;
+          const uint32_t sE = sbase + C::kOffWin;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // 16 head-dim elements per k-step
+            const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_f16_ss_w(tmem + C::kColS, make_sdesc_sw128(sQ + oq, 16, 1024),
+                         make_sdesc_sw128(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idesc_s,
+                         kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t oe = (rb * C::kBoxes + (kk >> 2)) * 16384 + (kk & 3) * 32;
+              mma_f16_ss_w(tmem + C::kColG + rb * 128, make_sdesc_sw128(sE + oe, 16, 1024),
+                           make_sdesc_sw128(sQ + oq, 16, 1024), idesc_g, kk > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit_w(BAR(C::kBarSFull));
+        }
+        if (t >= 1) issue_pv(t - 1);
+      }
+      issue_pv(nsteps - 1);
+    }
+    // every MMA (and every commit arrive) has landed before TMEM is released
+    tc_commit_w(BAR(C::kBarMmaDone));
+    mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+    __syncwarp();
+  } else {
+    relpos_softmax<D, BF16>(p, smem, tmem, bars, wctx, q0, h, b, nsteps);
+  }
+
+  // ---- teardown: every role is done with TMEM
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace attn_b200

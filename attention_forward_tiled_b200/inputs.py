@@ -53,6 +53,16 @@ INDEXER_WORKLOADS = {
 }
 
 
+# Block-local attention with the relative-position term (the Granite-Speech conformer of the
+# vLLM "PR #42933" page): the sequence is cut into blocks of 200 tokens (B counts batch x
+# blocks), 8 heads of d 128, every distance within a block distinct (R = 199 -> 399
+# embedding rows).  The page gives no sizes; these are a plain reading of a block-local
+# speech encoder.
+RELPOS_WORKLOADS = {
+    "relpos_block200": dict(B=512, H=8, Nq=200, Nk=200, d=128, R=199, causal=False, dtype="f16",
+                            scale=1.0 / math.sqrt(128), seed=9),
+}
+
 def make_inputs(B, H, Nq, Nk, d, dtype="f16", seed=0, k_mult=1.0, **_):
     """Return CPU tensors (q, k, v) in [B, N, H, d] layout and the given dtype."""
     g = torch.Generator("cpu").manual_seed(int(seed))
@@ -126,3 +136,15 @@ def make_indexer_inputs(B, T, H, P, d, dtype="f16", seed=0, weights="random", ma
         mask = mask.expand(B, T, P).contiguous()
     dt = DTYPES[dtype]
     return q.to(dt), kp.to(dt), w, mask
+
+
+def make_relpos_inputs(B, H, Nq, Nk, d, R, dtype="f16", seed=0, **_):
+    """q, k, v as make_inputs and the relative-position table emb [2R + 1, d] (randn), CPU
+    tensors in the dtype.  Draw order: q, k, v, emb."""
+    g = torch.Generator("cpu").manual_seed(int(seed))
+    q = torch.randn(B, Nq, H, d, generator=g, dtype=torch.float32)
+    k = torch.randn(B, Nk, H, d, generator=g, dtype=torch.float32)
+    v = torch.randn(B, Nk, H, d, generator=g, dtype=torch.float32)
+    emb = torch.randn(2 * R + 1, d, generator=g, dtype=torch.float32)
+    dt = DTYPES[dtype]
+    return q.to(dt), k.to(dt), v.to(dt), emb.to(dt)

@@ -252,6 +252,35 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
                       int d, int causal, float scale, int dtype, attn_stream_t stream);
 
 /*
+ * attn_fwd_relpos -- attention with a fused relative-position score term.
+ *
+ * The Granite-Speech conformer block attention of the vLLM page "PR #42933"
+ * (sections "实现拆解" and "关键源码片段"): the scores carry, besides
+ * q_i . k_j, the einsum of the queries with the relative-position embeddings
+ * gathered by a distance table, both scaled, before masking and softmax:
+ *   S[i, j] = scale * (q_i . k_j + q_i . emb[dist(i, j)]),
+ *   dist(i, j) = clamp(i - j, -R, R) + R     (row R of emb is distance 0),
+ * then O and lse exactly as attn_fwd.  The table is the conformer's clamped
+ * relative distance, so it is given by R, not stored; a model whose table is
+ * clamp(i - j, -R, R) + M passes emb + (M - R) * d.  The term is formed on the
+ * tensor cores per 128 x 64 tile and never written to memory.
+ *
+ *   q, out       [B, Nq, H, d]   dtype      (read / written)
+ *   k, v         [B, Nk, H, d]   dtype      (read)
+ *   emb          [n_emb, d]      dtype      (read; n_emb >= 2R + 1; shared by
+ *                                            every batch element and head)
+ *   lse          [B, H, Nq]      float32    (written; may be NULL)
+ *   B (batch x blocks), H, Nq, Nk, d, causal, scale, dtype and alignment as
+ *   attn_fwd; emb 16-byte aligned, R >= 0.  For bf16 inputs P V runs in fp16 as
+ *   in attn_fwd, with the same value-range status (ATTN_ERR_RANGE).
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA;
+ * asynchronous like attn_fwd.
+ */
+ATTN_API int attn_fwd_relpos(const void* q, const void* k, const void* v, const void* emb, void* out,
+                             float* lse, int B, int H, int Nq, int Nk, int d, int n_emb, int R,
+                             int causal, float scale, int dtype, attn_stream_t stream);
+
+/*
  * attn_indexer_score -- lightning-indexer score on the tensor cores.
  *
  * The aispot.cmou.io report on llama.cpp release b11372 (entry "compute the

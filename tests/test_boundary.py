@@ -135,6 +135,29 @@ def test_prefill_entry_validation(lib):
     assert lib.attn_fwd_prefill(Q, K, V, O, L, 1, 2, 64, 64, 32, 0, 0.1, 1, NULL) == attn.ATTN_ERR_UNSUPPORTED
 
 
+EMB = ctypes.c_void_p(0x900000000)
+
+
+def relpos(lib, q=Q, k=K, v=V, emb=EMB, o=O, lse=L, B=2, H=4, Nq=200, Nk=200, d=128, n_emb=401,
+           R=200, causal=0, scale=0.1, dtype=0):
+    return lib.attn_fwd_relpos(q, k, v, emb, o, lse, B, H, Nq, Nk, d, n_emb, R, causal, scale, dtype, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(emb=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(R=-1), attn.ATTN_ERR_INVALID_ARG),
+    (dict(n_emb=400), attn.ATTN_ERR_INVALID_ARG),                          # fewer than 2R + 1 rows
+    (dict(emb=ctypes.c_void_p(0x900000008)), attn.ATTN_ERR_INVALID_ARG),   # 8-byte aligned only
+    (dict(emb=ctypes.c_void_p(0x400000000 + 1024)), attn.ATTN_ERR_INVALID_ARG),  # out overlaps emb
+    (dict(o=NULL), attn.ATTN_ERR_INVALID_ARG),
+    (dict(causal=3), attn.ATTN_ERR_INVALID_ARG),
+    (dict(d=32), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(dtype=5), attn.ATTN_ERR_UNSUPPORTED),
+])
+def test_relpos_entry_validation(lib, kw, code):
+    assert relpos(lib, **kw) == code
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     q = torch.zeros(1, 8, 1, 64, dtype=torch.float16)
