@@ -64,12 +64,14 @@ KERNEL_SOURCES = {
     "mq": ("decode_mq_sm100.cuh", "sm100_ptx.cuh"),
     "indexer": ("indexer_sm100.cuh", "sm100_ptx.cuh"),
     "bwd": ("backward_sm100.cuh", "sm100_ptx.cuh"),
+    "relpos": ("relpos_sm100.cuh", "sm100_ptx.cuh"),
 }
 
 
 def kernel_kind(workload):
     """Which kernel's sources a workload's traffic figure belongs to."""
-    for prefix, kind in (("decode", "decode"), ("spec", "mq"), ("indexer", "indexer"), ("bwd", "bwd")):
+    for prefix, kind in (("decode", "decode"), ("spec", "mq"), ("indexer", "indexer"), ("bwd", "bwd"),
+                         ("relpos", "relpos")):
         if workload.startswith(prefix):
             return kind
     return "prefill"
@@ -579,6 +581,60 @@ def measure_bwd(name, K, W, world, device, peaks):
             "clocks": sampler.summary(), "config": cfg}
 
 
+def measure_relpos(name, K, W, world, device, peaks):
+    """Attention with the relative-position term (attn_fwd_relpos): TFLOP/s counted from the
+    three products the definition takes per score (q.k, q.emb[dist] and p.v, 2d FLOP each),
+    6 B H Nq Nk d, on the block-local workload; the kernel's window product does more."""
+    import torch
+
+    import attention_forward_tiled_b200 as attn
+    from attention_forward_tiled_b200.inputs import RELPOS_WORKLOADS, make_relpos_inputs
+
+    w = RELPOS_WORKLOADS[name]
+    q, k, v, emb = (t.to(device) for t in make_relpos_inputs(**w))
+    out = torch.empty_like(q)
+    lse = torch.empty((w["B"], w["H"], w["Nq"]), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        attn.attn_fwd_relpos(q, k, v, emb, w["R"], causal=w["causal"], scale=w["scale"], out=out, lse=lse,
+                             stream=stream)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(device)
+    if attn.get_status(device=device) != 0:
+        raise RuntimeError("device status error during warm-up")
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    t_steps = time_gpu_steps(step, K, stream, None)
+    sampler.stop()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    if attn.get_status(device=device) != 0:
+        raise RuntimeError("device status error during the timed region")
+    elapsed_ms = max_over_ranks(sum(t_steps), world)
+    f = 6.0 * w["B"] * w["H"] * w["Nq"] * w["Nk"] * w["d"]
+    if w["causal"]:
+        f *= 0.5
+    achieved = f / (statistics.mean(t_steps) * 1e-3) / 1e12
+    nbytes = (2 * q.numel() + k.numel() + v.numel() + emb.numel()) * q.element_size() + lse.numel() * 4
+    del q, k, v, emb, out, lse
+    torch.cuda.empty_cache()
+    return {"value": world * K * f / (elapsed_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": elapsed_ms / K,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": committed_traffic(name), "algorithmic_flops_per_launch": f,
+                         "algorithmic_bytes_per_launch": nbytes},
+            "clocks": sampler.summary(),
+            "config": {"workload": name, "B": w["B"], "H": w["H"], "Nq": w["Nq"], "Nk": w["Nk"], "d": w["d"],
+                       "R": w["R"], "causal": w["causal"], "dtype": w["dtype"],
+                       "l2": "%.0f MB moved per call" % (nbytes / 1e6)}}
+
+
 def print_single(args, world, rank, r, dtype):
     """One JSON line for a workload timed on its own (profiling and single-kernel runs)."""
     line = {"metric": METRIC, "value": r["value"], "unit": r["unit"], "n_gpus": world, "steps": args.steps,
@@ -630,7 +686,11 @@ def run_ours(args):
     peaks = load_peaks()
     K, W = args.steps, max(3, args.warmup)
 
-    from attention_forward_tiled_b200.inputs import INDEXER_WORKLOADS, PAGED_WORKLOADS, WORKLOADS
+    from attention_forward_tiled_b200.inputs import (INDEXER_WORKLOADS, PAGED_WORKLOADS, RELPOS_WORKLOADS,
+                                                     WORKLOADS)
+    if args.workload in RELPOS_WORKLOADS:
+        r = measure_relpos(args.workload, K, W, world, device, peaks)
+        return print_single(args, world, rank, r, RELPOS_WORKLOADS[args.workload]["dtype"])
     if args.workload in INDEXER_WORKLOADS:
         r = measure_indexer(args.workload, K, W, world, device, peaks)
         r["score"]["extra"] = {"topk": r["topk"]}
@@ -670,6 +730,7 @@ def run_ours(args):
         extra["indexer_h4_score"] = r["score"]
         extra["indexer_h4_topk"] = r["topk"]
         extra["bwd_causal4k"] = measure_bwd("bwd_causal4k", K, W, world, device, peaks)
+        extra["relpos_block200"] = measure_relpos("relpos_block200", K, W, world, device, peaks)
     line = {
         "metric": METRIC,
         "value": main["value"],

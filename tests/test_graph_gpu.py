@@ -99,6 +99,15 @@ def test_graph_replay_indexer_and_topk():
     _replay_equals_eager(run, [score, idx])
 
 
+def test_graph_replay_relpos():
+    from attention_forward_tiled_b200 import attn_fwd_relpos
+    from attention_forward_tiled_b200.inputs import make_relpos_inputs
+    q, k, v, emb = (t.cuda() for t in make_relpos_inputs(2, 2, 200, 200, 128, 50, seed=12))
+    out = torch.empty_like(q)
+    lse = torch.empty((2, 2, 200), dtype=torch.float32, device="cuda")
+    _replay_equals_eager(lambda: attn_fwd_relpos(q, k, v, emb, 50, causal=True, out=out, lse=lse), [out, lse])
+
+
 def test_graph_replay_backward():
     from attention_forward_tiled_b200 import attn_bwd
     q, k, v = (t.cuda() for t in make_inputs(1, 2, 200, 300, 128, dtype="f16", seed=8))

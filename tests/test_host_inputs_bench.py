@@ -127,5 +127,6 @@ def test_traffic_figures_follow_their_kernel():
     assert bench.kernel_kind("decode") == "decode" and bench.kernel_kind("decode_paged16") == "decode"
     assert bench.kernel_kind("spec8_paged16") == "mq"
     assert bench.kernel_kind("indexer_h4") == "indexer" and bench.kernel_kind("bwd_causal4k") == "bwd"
+    assert bench.kernel_kind("relpos_block200") == "relpos"
     shas = {k: bench.kernel_source_sha(k) for k in bench.KERNEL_SOURCES}
     assert len(set(shas.values())) == len(shas)
