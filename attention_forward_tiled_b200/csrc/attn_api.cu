@@ -155,12 +155,13 @@ int encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d, i
 }
 
 // 3-D view (d, rows, B) of a contiguous [B, rows, d] tensor; box (64, 128, 1), 128B swizzle.
-int encode_rows3d(CUtensorMap* map, const void* ptr, int B, long long rows, int d, int dtype) {
+int encode_rows3d(CUtensorMap* map, const void* ptr, int B, long long rows, int d, int dtype,
+                  int box_rows = 128) {
   EncodeTiledFn encode = get_encode_fn();
   if (!encode) return ATTN_ERR_CUDA;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)B};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType ty =
       dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -558,7 +559,7 @@ int launch_relpos(DeviceState* ds, const void* q, const void* k, const void* v, 
   if (int rc = encode_bnhd(&p.tm_q, q, B, Nq, H, D, dtype, 128)) return rc;
   if (int rc = encode_bnhd(&p.tm_k, k, B, Nk, H, D, dtype, 64)) return rc;
   if (int rc = encode_bnhd(&p.tm_v, v, B, Nk, H, D, dtype, 64)) return rc;
-  if (int rc = encode_rows3d(&p.tm_e, emb, 1, n_emb, D, dtype)) return rc;
+  if (int rc = encode_rows3d(&p.tm_e, emb, 1, n_emb, D, dtype, C::kWinRows)) return rc;
   p.out = out;
   p.lse = lse;
   p.status = ds->status_ptr;

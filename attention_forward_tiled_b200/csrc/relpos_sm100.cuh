@@ -8,21 +8,23 @@
 //   dist[i, j] = clamp(i - j, -R, R) + R,     emb row R = distance 0,
 // so the kernel takes R and never reads a table.
 //
-// One CTA per (b, h, 128-query tile); keys in steps of 64.  For a step the distances met
-// span at most 191 consecutive embedding rows (lo ... lo + 190, clamped at 0 and 2R), so
-// the tensor core computes G^T = E_win Q^T (two M = 128 products over 256 rows of the
-// window: TMEM lane = embedding row, column = query row) next to S = Q K^T.  The softmax
-// warps copy G^T to shared memory as Gs[c][row] with a 132-word row pitch and gather
-// bias[i, j] = Gs[dist(i, j) - lo][i]: a warp's 32 query rows read 32 different words of
-// different banks at every key (the 132 pitch makes the skewed read conflict-free), and a
-// thread keeps its own row in registers for nothing.  Roles (192 threads):
-//   * warp 4, producer: Q once, the K/V ring (two stages), the embedding window per step;
-//   * warp 5, MMA issuer: S and G of step t, then O += P V of step t - 1 once P is ready;
-//   * warps 0-3, softmax (thread = query row): copy G, gather the bias, online softmax
-//     (fp16 P into shared memory, O rescaled in TMEM when the row maximum grows), and the
-//     O / l epilogue.  For bf16 inputs they convert each V tile to fp16 in place first
-//     (P V runs in fp16, as in the plain kernel; magnitudes with no fp16 value set the
-//     range status).
+// One CTA per (b, h, 128-query tile); keys in steps of 64.  For a pair of steps (128 keys)
+// the distances met span at most 255 consecutive embedding rows (lo ... lo + 254, clamped
+// at 0 and 2R), so on every other step the tensor core computes G = Q E_win^T (N = 256:
+// TMEM lane = query row, column = window row) next to S = Q K^T, and the next window has a
+// whole step to arrive.  Query row r needs the columns dist(r, j) - lo for its 64 keys of
+// a step, a run of at most 64 that starts at a row-dependent column: each softmax thread
+// copies the 112 columns that cover its warp's runs into its own shared-memory row (pitch
+// 116 words, so the copy and the skewed reads are free of bank conflicts) and gathers from
+// there; no other thread reads the row, so no barrier is needed.  Roles (192 threads):
+//   * warp 4, producer: Q once, the K/V ring (two stages), the embedding window of each
+//     step pair as soon as the previous pair's product has read the buffer;
+//   * warp 5, MMA issuer: S (and G) of step t, then O += P V of step t - 1 once P is ready;
+//   * warps 0-3, softmax (thread = query row): copy and gather G, online softmax (fp16 P
+//     into shared memory, in the K slot of the step at d = 128; O rescaled in TMEM when
+//     the row maximum grows), and the O / l epilogue.  For bf16 inputs they convert each V
+//     tile to fp16 in place first (P V runs in fp16, as in the plain kernel; magnitudes
+//     with no fp16 value set the range status).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -33,7 +35,7 @@ struct RelposParams {
   CUtensorMap tm_q;  // q [B, Nq, H, D] as 4-D (D, H, Nq, B), box (64, 1, 128, 1), 128B swizzle
   CUtensorMap tm_k;  // k [B, Nk, H, D] as 4-D (D, H, Nk, B), box (64, 1, 64, 1)
   CUtensorMap tm_v;  // v, as k
-  CUtensorMap tm_e;  // emb [n_emb, D] as 3-D (D, n_emb, 1), box (64, 128, 1)
+  CUtensorMap tm_e;  // emb [n_emb, D] as 3-D (D, n_emb, 1), box (64, 192, 1)
   void* out;         // [B, Nq, H, D], the input dtype
   float* lse;        // [B, H, Nq] natural log, or nullptr
   int* status;
@@ -48,37 +50,40 @@ struct RelposCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kQBytes = kBoxes * 128 * 128;   // 128 rows x D
   static constexpr int kKVBytes = kBoxes * 64 * 128;   // 64 rows x D
-  static constexpr int kEBytes = 2 * kBoxes * 128 * 128;  // 256 embedding rows x D
-  static constexpr int kGsPitch = 132;                 // words per embedding row of Gs
-  static constexpr int kGsRows = 192;                  // rows a step can need (191) rounded up
-  static constexpr int kGsBytes = kGsRows * kGsPitch * 4;
-  static constexpr int kWinBytes = kEBytes > kGsBytes ? kEBytes : kGsBytes;
+  static constexpr int kWinRows = 256;                  // embedding rows two steps can need (255)
+  static constexpr int kEBoxBytes = kWinRows * 128;     // 256 rows x 64 elements
+  static constexpr int kEBytes = kBoxes * kEBoxBytes;
+  static constexpr int kGCols = 112;                    // columns of G a thread keeps per step
+  static constexpr int kGPitch = 116;                   // words of a thread's row of G
+  static constexpr bool kPInK = D == 128;               // P (16 KB) fits the step's K slot
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;         // [2]
   static constexpr int kOffV = kOffK + 2 * kKVBytes;    // [2]
-  static constexpr int kOffP = kOffV + 2 * kKVBytes;    // 128 x 64 fp16, 128B swizzle
-  static constexpr int kOffWin = kOffP + 128 * 128;     // embedding window, then Gs
-  static constexpr int kOffBar = kOffWin + kWinBytes;
+  static constexpr int kOffE = kOffV + 2 * kKVBytes;    // embedding window
+  static constexpr int kOffP = kOffE + kEBytes;         // 128 x 64 fp16, 128B swizzle (D = 64)
+  static constexpr int kOffG = kOffP + (kPInK ? 0 : 128 * 128);  // [128 rows][kGPitch] fp32
+  static constexpr int kOffBar = kOffG + 128 * kGPitch * 4;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKVFull = 1;   // [2]
   static constexpr int kBarKVEmpty = 3;  // [2]
   static constexpr int kBarEFull = 5;
-  static constexpr int kBarGsFree = 6;   // the softmax warps are done reading Gs (4 arrivals)
-  static constexpr int kBarSFull = 7;    // S and G of the step are in TMEM
-  static constexpr int kBarSFree = 8;    // ... and have been read (4 arrivals)
-  static constexpr int kBarPFull = 9;    // P written, O rescaled, V converted (4 arrivals)
-  static constexpr int kBarPVDone = 10;  // O += P V of the step has completed
-  static constexpr int kBarMmaDone = 11;
+  static constexpr int kBarSFull = 6;    // S (and G, even steps) of the step are in TMEM
+  static constexpr int kBarSFree = 7;    // ... and have been read (4 arrivals)
+  static constexpr int kBarPFull = 8;    // P written, O rescaled, V converted (4 arrivals)
+  static constexpr int kBarPVDone = 9;   // O += P V of the step has completed
+  static constexpr int kBarMmaDone = 10;
+  static constexpr int kBarEFree = 11;   // the G product of a step pair has read the window
   static constexpr int kNumBars = 12;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // +1024: manual 1 KB alignment
   static constexpr int kThreads = 192;
   static constexpr int kProducerWarp = 4;
   static constexpr int kMmaWarp = 5;
-  // TMEM columns
+  // TMEM columns; a warp's G loads start at most 224 columns past kColG and read 128
+  // (past column 383 they read values no thread uses)
   static constexpr uint32_t kColO = 0;    // D columns
-  static constexpr uint32_t kColS = 128;  // 64 columns
-  static constexpr uint32_t kColG = 256;  // two 128-column accumulators
+  static constexpr uint32_t kColG = 128;  // 256 columns
+  static constexpr uint32_t kColS = 448;  // 64 columns
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -93,9 +98,11 @@ __device__ __forceinline__ int relpos_steps(const RelposParams& p, int q0) {
   return kend <= 0 ? 0 : (kend + 63) / 64;
 }
 
-// First embedding row a step needs: the smallest clamped distance over the tile.
+// First embedding row a pair of steps (128 keys from k0) needs: the smallest clamped
+// distance over the query tile and those keys.  The window lo ... lo + 255 covers the
+// pair (distances span 255 values).
 __device__ __forceinline__ int relpos_lo(const RelposParams& p, int q0, int k0) {
-  return min(max(q0 - (k0 + 63), -p.R), p.R) + p.R;
+  return min(max(q0 - (k0 + 127), -p.R), p.R) + p.R;
 }
 
 
@@ -110,8 +117,7 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
   const int r = threadIdx.x;  // row of the tile
   const int i = q0 + r;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  float* gs = reinterpret_cast<float*>(smem + C::kOffWin);  // [kGsRows][kGsPitch]
-  uint8_t* sp = smem + C::kOffP;
+  float* grow = reinterpret_cast<float*>(smem + C::kOffG) + r * C::kGPitch;  // this row's G
   const int shift = p.Nk - p.Nq;  // bottom-right causal alignment
   float m = -INFINITY;            // running maximum of scale * log2(e) * score
   float l0 = 0.f, l1 = 0.f;       // sum of the fp16-rounded P the tensor core multiplies
@@ -119,31 +125,29 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
 
   for (int t = 0; t < nsteps; ++t) {
     const int k0 = t * 64;
-    const int lo = relpos_lo(p, q0, k0);
-    const int hi = min(max(q0 + 127 - k0, -p.R), p.R) + p.R;
-    const int n_off = hi - lo + 1;  // embedding rows this step uses (<= 191)
+    const int lo = relpos_lo(p, q0, (t & ~1) * 64);  // window of the step pair
     mbar_wait(BAR(C::kBarSFull), t & 1, wctx);
     __syncwarp();
     tc_fence_after_sync();
-    // ---- G^T (lane = embedding row) -> Gs[row][query row]; the loads are warp-collective,
-    // so the condition is per warp
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      if (a * 128 + warp * 32 < n_off) {
-        const int c = a * 128 + warp * 32 + lane;  // < 192
-        float* dst = gs + c * C::kGsPitch;
+    // ---- this warp's rows need window columns cw ... cw + 94 (the clamp is monotone and
+    // moves by at most one per row or key): load the 128 from the 32-aligned column below
+    // and keep the 112 from base + s0, s0 = 0 or 16, which hold them
+    const int cw = min(max(q0 + warp * 32 - (k0 + 63), -p.R), p.R) + p.R - lo;
+    const int s0 = (cw & 31) & 16;
+    const int base = (cw & ~31) + s0;  // column of grow[0]
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t g[32];
-          tmem_ld32(tmem + lane_base + C::kColG + a * 128 + q * 32, g);
-          tmem_ld_wait();
-          reg_order_after_wait(g);
+    for (int q = 0; q < 4; ++q) {
+      uint32_t g[32];
+      tmem_ld32(tmem + lane_base + C::kColG + (cw & ~31) + q * 32, g);
+      tmem_ld_wait();
+      reg_order_after_wait(g);
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<float4*>(dst + q * 32 + 4 * u) =
-                make_float4(__uint_as_float(g[4 * u]), __uint_as_float(g[4 * u + 1]),
-                            __uint_as_float(g[4 * u + 2]), __uint_as_float(g[4 * u + 3]));
-        }
+      for (int u = 0; u < 8; ++u) {
+        const int dst = q * 32 + 4 * u - s0;
+        if (dst >= 0 && dst < C::kGCols)  // uniform over the warp
+          *reinterpret_cast<float4*>(grow + dst) =
+              make_float4(__uint_as_float(g[4 * u]), __uint_as_float(g[4 * u + 1]),
+                          __uint_as_float(g[4 * u + 2]), __uint_as_float(g[4 * u + 3]));
       }
     }
     // ---- this row's 64 raw scores
@@ -156,21 +160,38 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     tc_fence_before_sync();
     __syncwarp();
     if (lane == 0) mbar_arrive(BAR(C::kBarSFree));  // S and G may be overwritten
-    named_bar_sync(1, 128);                          // Gs is complete
     // ---- add the gathered term, scale, mask
     float x[64];
     float mx = -INFINITY;
+    // keys k0 + jj with jj < jlim are allowed for this row (tail and bottom-right causal)
+    const int jlim = i < p.Nq ? (p.causal ? min(p.Nk, i + shift + 1) : p.Nk) - k0 : 0;
+    // no allowed key of the step has a clamped distance; key k0 is then allowed and its
+    // column lies in the row, and a masked key reads at most 63 words below it (inside
+    // shared memory, a value of no use)
+    const bool unclamped = i - (k0 + min(63, jlim - 1)) >= -p.R && i - k0 <= p.R;
+    if (jlim <= 0) {  // the row sees no key of this step
 #pragma unroll
-    for (int jj = 0; jj < 64; ++jj) {
-      const int j = k0 + jj;
-      const bool allowed = i < p.Nq && j < p.Nk && (!p.causal || j <= i + shift);
-      const int c = min(max(i - j, -p.R), p.R) + p.R - lo;  // in [0, n_off) for every i, j of the tile
-      const float g = gs[c * C::kGsPitch + r];
-      x[jj] = allowed ? (__uint_as_float(sv[jj >> 5][jj & 31]) + g) * p.scale_log2 : -INFINITY;
-      mx = fmaxf(mx, x[jj]);
+      for (int jj = 0; jj < 64; ++jj) x[jj] = -INFINITY;
+    } else if (unclamped) {
+      // key jj's column is (key k0's column) - jj
+      const float* gp = grow + (i - k0 + p.R - lo - base);
+#pragma unroll
+      for (int jj = 0; jj < 64; ++jj) {
+        x[jj] = jj < jlim ? (__uint_as_float(sv[jj >> 5][jj & 31]) + gp[-jj]) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[jj]);
+      }
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < 64; ++jj) {
+        const int j = k0 + jj;
+        const bool allowed = i < p.Nq && j < p.Nk && (!p.causal || j <= i + shift);
+        // column of key j in this row's copy
+        const int c = min(max(i - j, -p.R), p.R) + p.R - lo - base;
+        const float g = grow[c];
+        x[jj] = allowed ? (__uint_as_float(sv[jj >> 5][jj & 31]) + g) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[jj]);
+      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(BAR(C::kBarGsFree));  // the window may be reloaded
     // ---- online softmax: O and the P buffer are free once the previous P V is done
     const float m_new = fmaxf(m, mx);
     if (t >= 1) {
@@ -203,7 +224,9 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
       pk[u] = pack2<false>(ex2_approx(x[2 * u] - mu), ex2_approx(x[2 * u + 1] - mu));
       add_f16x2_f32(l0, l1, pk[u]);
     }
-    // P row r: 64 fp16 = eight 16-byte chunks, 128-byte swizzle (K-major A operand)
+    // P row r: 64 fp16 = eight 16-byte chunks, 128-byte swizzle (K-major A operand); at
+    // d = 128 in the step's K slot, which S has finished reading
+    uint8_t* sp = smem + (C::kPInK ? C::kOffK + (t & 1) * C::kKVBytes : C::kOffP);
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc)
       *reinterpret_cast<uint4*>(sp + r * 128 + ((cc ^ (r & 7)) << 4)) =
@@ -292,12 +315,12 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
       mbar_init(BAR(C::kBarKVEmpty + s), 1);
     }
     mbar_init(BAR(C::kBarEFull), 1);
-    mbar_init(BAR(C::kBarGsFree), 4);
     mbar_init(BAR(C::kBarSFull), 1);
     mbar_init(BAR(C::kBarSFree), 4);
     mbar_init(BAR(C::kBarPFull), 4);
     mbar_init(BAR(C::kBarPVDone), 1);
     mbar_init(BAR(C::kBarMmaDone), 1);
+    mbar_init(BAR(C::kBarEFree), 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -336,16 +359,16 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
                         bx * 64, h, k0, b);
         }
         ++nkv;
-        // the window shares its bytes with Gs: wait until the previous step's gather is done
-        if (t >= 1) mbar_wait(BAR(C::kBarGsFree), (t - 1) & 1, wctx);
+        if (t & 1) continue;  // one window per step pair
+        // one window buffer: the previous pair's G product must have read it
+        const int pr = t >> 1;
+        if (pr >= 1) mbar_wait(BAR(C::kBarEFree), (pr - 1) & 1, wctx);
         __syncwarp();
         if (warp_flag(abort_flag)) break;
         const int lo = relpos_lo(p, q0, k0);
         mbar_arrive_expect_tx_w(BAR(C::kBarEFull), C::kEBytes);
-        for (int rb = 0; rb < 2; ++rb)
-          for (int bx = 0; bx < C::kBoxes; ++bx)  // rows past n_emb read as zeros and are never used
-            tma_load_3d_w(sbase + C::kOffWin + (rb * C::kBoxes + bx) * 16384, &p.tm_e, BAR(C::kBarEFull),
-                          bx * 64, lo + rb * 128, 0);
+        for (int bx = 0; bx < C::kBoxes; ++bx)  // rows past n_emb read as zeros and are never used
+          tma_load_3d_w(sbase + C::kOffE + bx * C::kEBoxBytes, &p.tm_e, BAR(C::kBarEFull), bx * 64, lo, 0);
         ++ne;
       }
       if (lane == 0 && *abort_flag) {
@@ -360,7 +383,7 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
   } else if (warp == C::kMmaWarp) {
     // ======================= tcgen05 MMA issuer =======================
     constexpr uint32_t idesc_s = make_idesc_f16(128, 64, BF16, false);   // Q K^T, both K-major
-    constexpr uint32_t idesc_g = make_idesc_f16(128, 128, BF16, false);  // E_win Q^T, both K-major
+    constexpr uint32_t idesc_g = make_idesc_f16(128, C::kWinRows, BF16, false);  // Q E_win^T, both K-major
     constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);    // P V: fp16, V MN-major
     auto issue_pv = [&](int t) {
       mbar_wait(BAR(C::kBarPFull), t & 1, wctx);
@@ -368,7 +391,7 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
         const uint32_t sV = sbase + C::kOffV + (t & 1) * C::kKVBytes;
-        const uint32_t sP = sbase + C::kOffP;
+        const uint32_t sP = sbase + (C::kPInK ? C::kOffK + (t & 1) * C::kKVBytes : C::kOffP);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 16 keys per k-step
           mma_f16_ss_w(tmem + C::kColO, make_sdesc_sw128(sP + kk * 32, 16, 1024),
@@ -382,14 +405,14 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
       for (int t = 0; t < nsteps; ++t) {
         const int s = t & 1;
         mbar_wait(BAR(C::kBarKVFull + s), (t >> 1) & 1, wctx);
-        mbar_wait(BAR(C::kBarEFull), t & 1, wctx);
+        if (!(t & 1)) mbar_wait(BAR(C::kBarEFull), (t >> 1) & 1, wctx);
         if (t >= 1) mbar_wait(BAR(C::kBarSFree), (t - 1) & 1, wctx);
         __syncwarp();
         tc_fence_after_sync();
         if (!warp_flag(abort_flag)) {
           const uint32_t sQ = sbase + C::kOffQ;
           const uint32_t sK = sbase + C::kOffK + s * C::kKVBytes;
-          const uint32_t sE = sbase + C::kOffWin;
+          const uint32_t sE = sbase + C::kOffE;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {  // 16 head-dim elements per k-step
             const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -397,15 +420,15 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
                          make_sdesc_sw128(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idesc_s,
                          kk > 0 ? 1u : 0u);
           }
-#pragma unroll
-          for (int rb = 0; rb < 2; ++rb) {
+          if (!(t & 1)) {  // G of the step pair
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t oe = (rb * C::kBoxes + (kk >> 2)) * 16384 + (kk & 3) * 32;
-              mma_f16_ss_w(tmem + C::kColG + rb * 128, make_sdesc_sw128(sE + oe, 16, 1024),
-                           make_sdesc_sw128(sQ + oq, 16, 1024), idesc_g, kk > 0 ? 1u : 0u);
+              mma_f16_ss_w(tmem + C::kColG, make_sdesc_sw128(sQ + oq, 16, 1024),
+                           make_sdesc_sw128(sE + (kk >> 2) * C::kEBoxBytes + (kk & 3) * 32, 16, 1024),
+                           idesc_g, kk > 0 ? 1u : 0u);
             }
+            tc_commit_w(BAR(C::kBarEFree));
           }
           tc_commit_w(BAR(C::kBarSFull));
         }
