@@ -545,7 +545,7 @@ int launch_indexer(DeviceState* ds, const void* q, const void* kp, const float* 
 }
 
 
-// Relative-position attention: one CTA per (128-query tile, head, batch).
+// Relative-position attention: persistent CTAs over the (batch, head, 128-query tile) units.
 template <int D, bool BF16>
 int launch_relpos(DeviceState* ds, const void* q, const void* k, const void* v, const void* emb, void* out,
                   float* lse, int B, int H, int Nq, int Nk, int n_emb, int R, int causal, float scale,
@@ -571,8 +571,12 @@ int launch_relpos(DeviceState* ds, const void* q, const void* k, const void* v, 
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
-  const dim3 grid((unsigned)((Nq + 127) / 128), (unsigned)H, (unsigned)B);
-  kernel<<<grid, dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
+  p.n_qtiles = (Nq + 127) / 128;
+  const long long units = (long long)B * H * p.n_qtiles;
+  if (units >= (1LL << 31)) return ATTN_ERR_INVALID_ARG;
+  p.n_units = (int)units;
+  const int grid = (int)std::min<long long>(units, ds->sm_count);  // persistent CTAs
+  kernel<<<dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -845,7 +849,6 @@ int attn_fwd_relpos(const void* q, const void* k, const void* v, const void* emb
   if (!emb || R < 0 || n_emb < 2 * (long long)R + 1) return ATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(emb) % 16 != 0) return ATTN_ERR_INVALID_ARG;
   if ((unsigned long long)n_emb * d * 2 >= (1ull << 40)) return ATTN_ERR_INVALID_ARG;
-  if (Nq > 65535 * 128 || H > 65535 || B > 65535) return ATTN_ERR_INVALID_ARG;  // grid limits
   const size_t q_bytes = (size_t)B * Nq * H * d * 2;
   if (overlaps(out, q_bytes, emb, (size_t)n_emb * d * 2) ||
       (lse && overlaps(lse, (size_t)B * H * Nq * 4, emb, (size_t)n_emb * d * 2)))

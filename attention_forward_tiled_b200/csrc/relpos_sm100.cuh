@@ -8,17 +8,19 @@
 //   dist[i, j] = clamp(i - j, -R, R) + R,     emb row R = distance 0,
 // so the kernel takes R and never reads a table.
 //
-// One CTA per (b, h, 128-query tile); keys in steps of 64.  For a pair of steps (128 keys)
-// the distances met span at most 255 consecutive embedding rows (lo ... lo + 254, clamped
-// at 0 and 2R), so on every other step the tensor core computes G = Q E_win^T (N = 256:
-// TMEM lane = query row, column = window row) next to S = Q K^T, and the next window has a
-// whole step to arrive.  Query row r needs the columns dist(r, j) - lo for its 64 keys of
+// Persistent CTAs over units (b, h, 128-query tile); keys in steps of 64.  For a pair of
+// steps (128 keys) the distances met span at most 255 consecutive embedding rows
+// (lo ... lo + 254, clamped at 0 and 2R), so on every other step the tensor core computes
+// G = Q E_win^T (N = 256: TMEM lane = query row, column = window row) next to S = Q K^T,
+// and the next window has a whole step to arrive.  Query row r needs the columns dist(r, j) - lo for its 64 keys of
 // a step, a run of at most 64 that starts at a row-dependent column: each softmax thread
 // copies the 112 columns that cover its warp's runs into its own shared-memory row (pitch
 // 116 words, so the copy and the skewed reads are free of bank conflicts) and gathers from
 // there; no other thread reads the row, so no barrier is needed.  Roles (192 threads):
-//   * warp 4, producer: Q once, the K/V ring (two stages), the embedding window of each
-//     step pair as soon as the previous pair's product has read the buffer;
+//   * warp 4, producer: Q of each unit as soon as the previous unit's last product has read
+//     it, the K/V ring (two stages), the embedding window of each step pair as soon as the
+//     previous pair's product has read the buffer (so the next unit's loads run behind the
+//     current unit's last step and epilogue);
 //   * warp 5, MMA issuer: S (and G) of step t, then O += P V of step t - 1 once P is ready;
 //   * warps 0-3, softmax (thread = query row): copy and gather G, online softmax (fp16 P
 //     into shared memory, in the K slot of the step at d = 128; O rescaled in TMEM when
@@ -40,6 +42,7 @@ struct RelposParams {
   float* lse;        // [B, H, Nq] natural log, or nullptr
   int* status;
   int B, H, Nq, Nk, R, causal;
+  int n_qtiles, n_units;  // 128-query tiles per (b, h); units (b, h, tile)
   float scale_log2;  // scale * log2(e)
   unsigned long long timeout_ns;
 };
@@ -73,7 +76,9 @@ struct RelposCfg {
   static constexpr int kBarPVDone = 9;   // O += P V of the step has completed
   static constexpr int kBarMmaDone = 10;
   static constexpr int kBarEFree = 11;   // the G product of a step pair has read the window
-  static constexpr int kNumBars = 12;
+  static constexpr int kBarQFree = 12;   // the last product of a unit has read Q
+  static constexpr int kBarOFree = 13;   // the epilogue of a unit has read O (4 arrivals)
+  static constexpr int kNumBars = 14;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // +1024: manual 1 KB alignment
   static constexpr int kThreads = 192;
@@ -109,24 +114,29 @@ __device__ __forceinline__ int relpos_lo(const RelposParams& p, int q0, int k0) 
 // Softmax warps 0-3: thread = query row q0 + r of the tile (TMEM lane r).
 template <int D, bool BF16>
 __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* smem, uint32_t tmem,
-                                               uint64_t* bars, const WaitCtx& wctx, int q0, int h, int b,
-                                               int nsteps) {
+                                               uint64_t* bars, const WaitCtx& wctx) {
   using C = RelposCfg<D>;
   auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = threadIdx.x;  // row of the tile
-  const int i = q0 + r;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
   float* grow = reinterpret_cast<float*>(smem + C::kOffG) + r * C::kGPitch;  // this row's G
   const int shift = p.Nk - p.Nq;  // bottom-right causal alignment
+  uint32_t vmag = 0;              // bf16: largest |V| bit pattern converted
+  int g = 0;                      // steps of this CTA so far (barrier phases)
+
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+  const int q0 = (u % p.n_qtiles) * 128;
+  const int h = (u / p.n_qtiles) % p.H, b = u / (p.n_qtiles * p.H);
+  const int i = q0 + r;
+  const int nsteps = relpos_steps(p, q0);
   float m = -INFINITY;            // running maximum of scale * log2(e) * score
   float l0 = 0.f, l1 = 0.f;       // sum of the fp16-rounded P the tensor core multiplies
-  uint32_t vmag = 0;              // bf16: largest |V| bit pattern converted
 
-  for (int t = 0; t < nsteps; ++t) {
+  for (int t = 0; t < nsteps; ++t, ++g) {
     const int k0 = t * 64;
     const int lo = relpos_lo(p, q0, (t & ~1) * 64);  // window of the step pair
-    mbar_wait(BAR(C::kBarSFull), t & 1, wctx);
+    mbar_wait(BAR(C::kBarSFull), g & 1, wctx);
     __syncwarp();
     tc_fence_after_sync();
     // ---- this warp's rows need window columns cw ... cw + 94 (the clamp is monotone and
@@ -195,7 +205,7 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     // ---- online softmax: O and the P buffer are free once the previous P V is done
     const float m_new = fmaxf(m, mx);
     if (t >= 1) {
-      mbar_wait(BAR(C::kBarPVDone), (t - 1) & 1, wctx);
+      mbar_wait(BAR(C::kBarPVDone), (g - 1) & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
       const bool grow = m_new > m && m > -INFINITY;
@@ -226,14 +236,14 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     }
     // P row r: 64 fp16 = eight 16-byte chunks, 128-byte swizzle (K-major A operand); at
     // d = 128 in the step's K slot, which S has finished reading
-    uint8_t* sp = smem + (C::kPInK ? C::kOffK + (t & 1) * C::kKVBytes : C::kOffP);
+    uint8_t* sp = smem + (C::kPInK ? C::kOffK + (g & 1) * C::kKVBytes : C::kOffP);
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc)
       *reinterpret_cast<uint4*>(sp + r * 128 + ((cc ^ (r & 7)) << 4)) =
           make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
     if constexpr (BF16) {  // V of this step to fp16, in place
-      mbar_wait(BAR(C::kBarKVFull + (t & 1)), (t >> 1) & 1, wctx);
-      uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffV + (t & 1) * C::kKVBytes);
+      mbar_wait(BAR(C::kBarKVFull + (g & 1)), (g >> 1) & 1, wctx);
+      uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffV + (g & 1) * C::kKVBytes);
 #pragma unroll 2
       for (int c = r; c < C::kKVBytes / 16; c += 128) {
         uint4 w = tile[c];
@@ -259,7 +269,7 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
   uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
                                          ((((long long)b * p.Nq + (row_ok ? i : 0)) * p.H + h) * D) * 2);
   if (nsteps > 0) {
-    mbar_wait(BAR(C::kBarPVDone), (nsteps - 1) & 1, wctx);
+    mbar_wait(BAR(C::kBarPVDone), (g - 1) & 1, wctx);
     __syncwarp();
     tc_fence_after_sync();
 #pragma unroll 1
@@ -278,12 +288,17 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
               pack2<BF16>(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv));
       }
     }
+    // O may be overwritten by the next unit's first P V
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(C::kBarOFree));
   } else if (row_ok) {  // no key reaches this tile
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (row_ok && p.lse != nullptr)
     p.lse[((long long)b * p.H + h) * p.Nq + i] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }  // units
   if constexpr (BF16) {
     if (max(vmag & 0xFFFFu, vmag >> 16) >= kBf16NoF16) atomicCAS(p.status, 0, kStatusRange);
   }
@@ -305,8 +320,13 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
-  const int q0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
-  const int nsteps = relpos_steps(p, q0);
+  // persistent CTAs: units u = (b, h, tile) in steps of gridDim.x; every role walks the
+  // same units, and barrier phases count steps, pairs and units over the whole walk
+  auto unit = [&](int u, int& q0, int& h, int& b) {
+    q0 = (u % p.n_qtiles) * 128;
+    h = (u / p.n_qtiles) % p.H;
+    b = u / (p.n_qtiles * p.H);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::kBarQFull), 1);
@@ -321,6 +341,8 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
     mbar_init(BAR(C::kBarPVDone), 1);
     mbar_init(BAR(C::kBarMmaDone), 1);
     mbar_init(BAR(C::kBarEFree), 1);
+    mbar_init(BAR(C::kBarQFree), 1);
+    mbar_init(BAR(C::kBarOFree), 4);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -335,22 +357,35 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
 
   if (warp == C::kProducerWarp) {
     // ======================= TMA producer =======================
-    int nkv = 0, ne = 0;
-    if (nsteps > 0) {
-      if (lane == 0) {
-        tma_prefetch_map(&p.tm_q);
-        tma_prefetch_map(&p.tm_k);
-        tma_prefetch_map(&p.tm_v);
-        tma_prefetch_map(&p.tm_e);
-      }
+    if (lane == 0) {
+      tma_prefetch_map(&p.tm_q);
+      tma_prefetch_map(&p.tm_k);
+      tma_prefetch_map(&p.tm_v);
+      tma_prefetch_map(&p.tm_e);
+    }
+    int g = 0, ge = 0, nu = 0;  // steps, step pairs and units (with keys) loaded
+    bool stop = false;
+    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
+      int q0, h, b;
+      unit(u, q0, h, b);
+      const int nsteps = relpos_steps(p, q0);
+      if (nsteps == 0) continue;
+      // one Q buffer: the previous unit's last product must have read it
+      if (nu >= 1) mbar_wait(BAR(C::kBarQFree), (nu - 1) & 1, wctx);
+      __syncwarp();
+      if (warp_flag(abort_flag)) break;
       mbar_arrive_expect_tx_w(BAR(C::kBarQFull), C::kQBytes);
       for (int bx = 0; bx < C::kBoxes; ++bx)
         tma_load_4d_w(sbase + C::kOffQ + bx * 16384, &p.tm_q, BAR(C::kBarQFull), bx * 64, h, q0, b);
-      for (int t = 0; t < nsteps; ++t) {
-        const int s = t & 1, k0 = t * 64;
-        if (t >= 2) mbar_wait(BAR(C::kBarKVEmpty + s), ((t >> 1) - 1) & 1, wctx);
+      ++nu;
+      for (int t = 0; t < nsteps; ++t, ++g) {
+        const int s = g & 1, k0 = t * 64;
+        if (g >= 2) mbar_wait(BAR(C::kBarKVEmpty + s), ((g >> 1) - 1) & 1, wctx);
         __syncwarp();
-        if (warp_flag(abort_flag)) break;
+        if (warp_flag(abort_flag)) {
+          stop = true;
+          break;
+        }
         mbar_arrive_expect_tx_w(BAR(C::kBarKVFull + s), 2 * C::kKVBytes);
         for (int bx = 0; bx < C::kBoxes; ++bx) {
           tma_load_4d_w(sbase + C::kOffK + s * C::kKVBytes + bx * 8192, &p.tm_k, BAR(C::kBarKVFull + s),
@@ -358,26 +393,28 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
           tma_load_4d_w(sbase + C::kOffV + s * C::kKVBytes + bx * 8192, &p.tm_v, BAR(C::kBarKVFull + s),
                         bx * 64, h, k0, b);
         }
-        ++nkv;
         if (t & 1) continue;  // one window per step pair
         // one window buffer: the previous pair's G product must have read it
-        const int pr = t >> 1;
-        if (pr >= 1) mbar_wait(BAR(C::kBarEFree), (pr - 1) & 1, wctx);
+        if (ge >= 1) mbar_wait(BAR(C::kBarEFree), (ge - 1) & 1, wctx);
         __syncwarp();
-        if (warp_flag(abort_flag)) break;
+        if (warp_flag(abort_flag)) {
+          ++g;  // this step's K/V copy is in flight
+          stop = true;
+          break;
+        }
         const int lo = relpos_lo(p, q0, k0);
         mbar_arrive_expect_tx_w(BAR(C::kBarEFull), C::kEBytes);
         for (int bx = 0; bx < C::kBoxes; ++bx)  // rows past n_emb read as zeros and are never used
           tma_load_3d_w(sbase + C::kOffE + bx * C::kEBoxBytes, &p.tm_e, BAR(C::kBarEFull), bx * 64, lo, 0);
-        ++ne;
+        ++ge;
       }
-      if (lane == 0 && *abort_flag) {
-        // let every copy this warp started land before the CTA can exit
-        mbar_wait_drain(BAR(C::kBarQFull), 0, p.timeout_ns);
-        for (int i = max(0, nkv - 2); i < nkv; ++i)
-          mbar_wait_drain(BAR(C::kBarKVFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
-        if (ne > 0) mbar_wait_drain(BAR(C::kBarEFull), (ne - 1) & 1, p.timeout_ns);
-      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // let every copy this warp started land before the CTA can exit
+      if (nu > 0) mbar_wait_drain(BAR(C::kBarQFull), (nu - 1) & 1, p.timeout_ns);
+      for (int i = max(0, g - 2); i < g; ++i)
+        mbar_wait_drain(BAR(C::kBarKVFull + (i & 1)), (i >> 1) & 1, p.timeout_ns);
+      if (ge > 0) mbar_wait_drain(BAR(C::kBarEFull), (ge - 1) & 1, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
@@ -385,28 +422,38 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
     constexpr uint32_t idesc_s = make_idesc_f16(128, 64, BF16, false);   // Q K^T, both K-major
     constexpr uint32_t idesc_g = make_idesc_f16(128, C::kWinRows, BF16, false);  // Q E_win^T, both K-major
     constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);    // P V: fp16, V MN-major
-    auto issue_pv = [&](int t) {
-      mbar_wait(BAR(C::kBarPFull), t & 1, wctx);
+    int nu = 0;  // units (with keys) whose products were issued
+    // O += P V of step g (t-th of its unit); the first of a unit waits until the previous
+    // unit's epilogue has read O
+    auto issue_pv = [&](int g, int t) {
+      if (t == 0 && nu >= 2) mbar_wait(BAR(C::kBarOFree), (nu - 2) & 1, wctx);
+      mbar_wait(BAR(C::kBarPFull), g & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
       if (!warp_flag(abort_flag)) {
-        const uint32_t sV = sbase + C::kOffV + (t & 1) * C::kKVBytes;
-        const uint32_t sP = sbase + (C::kPInK ? C::kOffK + (t & 1) * C::kKVBytes : C::kOffP);
+        const uint32_t sV = sbase + C::kOffV + (g & 1) * C::kKVBytes;
+        const uint32_t sP = sbase + (C::kPInK ? C::kOffK + (g & 1) * C::kKVBytes : C::kOffP);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 16 keys per k-step
           mma_f16_ss_w(tmem + C::kColO, make_sdesc_sw128(sP + kk * 32, 16, 1024),
                        make_sdesc_sw128(sV + kk * 2048, 8192, 1024), idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit_w(BAR(C::kBarPVDone));
-        tc_commit_w(BAR(C::kBarKVEmpty + (t & 1)));
+        tc_commit_w(BAR(C::kBarKVEmpty + (g & 1)));
       }
     };
-    if (nsteps > 0) {
-      mbar_wait(BAR(C::kBarQFull), 0, wctx);
-      for (int t = 0; t < nsteps; ++t) {
-        const int s = t & 1;
-        mbar_wait(BAR(C::kBarKVFull + s), (t >> 1) & 1, wctx);
-        if (!(t & 1)) mbar_wait(BAR(C::kBarEFull), (t >> 1) & 1, wctx);
-        if (t >= 1) mbar_wait(BAR(C::kBarSFree), (t - 1) & 1, wctx);
+    int g = 0, ge = 0;
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      int q0, h, b;
+      unit(u, q0, h, b);
+      const int nsteps = relpos_steps(p, q0);
+      if (nsteps == 0) continue;
+      mbar_wait(BAR(C::kBarQFull), nu & 1, wctx);
+      ++nu;
+      for (int t = 0; t < nsteps; ++t, ++g) {
+        const int s = g & 1;
+        mbar_wait(BAR(C::kBarKVFull + s), (g >> 1) & 1, wctx);
+        if (!(t & 1)) mbar_wait(BAR(C::kBarEFull), ge & 1, wctx);
+        if (g >= 1) mbar_wait(BAR(C::kBarSFree), (g - 1) & 1, wctx);
         __syncwarp();
         tc_fence_after_sync();
         if (!warp_flag(abort_flag)) {
@@ -431,17 +478,19 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
             tc_commit_w(BAR(C::kBarEFree));
           }
           tc_commit_w(BAR(C::kBarSFull));
+          if (t == nsteps - 1) tc_commit_w(BAR(C::kBarQFree));  // Q of this unit is read
         }
-        if (t >= 1) issue_pv(t - 1);
+        if (!(t & 1)) ++ge;
+        if (t >= 1) issue_pv(g - 1, t - 1);
       }
-      issue_pv(nsteps - 1);
+      issue_pv(g - 1, nsteps - 1);
     }
     // every MMA (and every commit arrive) has landed before TMEM is released
     tc_commit_w(BAR(C::kBarMmaDone));
     mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    relpos_softmax<D, BF16>(p, smem, tmem, bars, wctx, q0, h, b, nsteps);
+    relpos_softmax<D, BF16>(p, smem, tmem, bars, wctx);
   }
 
   // ---- teardown: every role is done with TMEM

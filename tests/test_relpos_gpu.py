@@ -53,6 +53,27 @@ def test_relpos_matches_oracle(B, H, Nq, Nk, d, R, causal, dtype):
     assert_lse_close(lse, ref_lse, what)
 
 
+@pytest.mark.parametrize("B,H,Nq,Nk,R,causal", [
+    (40, 4, 300, 300, 20, True),   # 480 units on 148 persistent CTAs, 1 to 5 key steps each
+    (80, 2, 300, 100, 30, True),   # ... and units whose rows see no key, interleaved
+])
+def test_relpos_persistent_units(B, H, Nq, Nk, R, causal):
+    """More units than SMs: every CTA walks several (b, h, tile) units with their barrier
+    phases carried across; five batch elements spread over the walk against the oracle."""
+    q, k, v, emb = make_relpos_inputs(B, H, Nq, Nk, 128, R, seed=B + Nk)
+    scale = 1.0 / math.sqrt(128)
+    out, lse = attn_fwd_relpos(q.cuda(), k.cuda(), v.cuda(), emb.cuda(), R, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    dist = clamped_dist(Nq, Nk, R)
+    for bb in (0, 1, B // 3, B // 2 + 1, B - 1):
+        ref_o, ref_lse = oracle.attn_fwd_relpos(q[bb:bb + 1], k[bb:bb + 1], v[bb:bb + 1], emb, dist,
+                                                causal=causal, scale=scale)
+        what = f"relpos persistent B{B} {Nq}x{Nk} batch {bb}"
+        assert_o_close(out[bb:bb + 1].cpu(), ref_o, q.dtype, what)
+        assert_lse_close(lse[bb:bb + 1].cpu(), ref_lse, what)
+
+
 def test_relpos_term_matters():
     """The same inputs with the term dropped (emb = 0) differ from the result with it, and
     equal plain attention: the kernel really adds the gathered term."""
