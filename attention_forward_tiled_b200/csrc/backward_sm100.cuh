@@ -18,8 +18,9 @@
 // dQ^T (lane = head-dim element, column = query) is staged in shared memory and added to
 // an fp32 accumulator in global memory with one TMA reduce-add per tile (other key tiles
 // add to the same rows);
-// dV and dK are written once at the end.  Roles (192 threads): warps 0-3 elementwise
-// and epilogues, warp 4 TMA producer, warp 5 MMA issuer.
+// dV and dK are written once at the end.  Roles (320 threads): warps 0-7 elementwise and
+// epilogues (two warps per TMEM lane quarter, each taking 32 of a tile's 64 query columns),
+// warp 8 TMA producer, warp 9 MMA issuer.
 //
 // TMEM columns: S^T [0,64) (P^T packed in [0,32)), dP^T [64,128) (dS^T packed in
 // [64,96)), dQ^T [128,192), dV [256,256+D), dK [384,384+D).
@@ -70,16 +71,17 @@ struct BwdCfg {
   static constexpr int kBarQFull = 1;                      // [2]
   static constexpr int kBarQEmpty = 3;                     // [2]
   static constexpr int kBarSFull = 5;                      // S^T and dP^T landed
-  static constexpr int kBarPDone = 6;                      // P^T, dS^T written (4 warps)
+  static constexpr int kBarPDone = 6;                      // P^T, dS^T written (8 warps)
   static constexpr int kBarDQFull = 7;                     // dQ^T landed
-  static constexpr int kBarDQFree = 8;                     // dQ^T read (4 warps)
+  static constexpr int kBarDQFree = 8;                     // dQ^T read (8 warps)
   static constexpr int kBarMmaDone = 9;
   static constexpr int kNumBars = 10;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
-  static constexpr int kThreads = 192;
-  static constexpr int kProducerWarp = 4;
-  static constexpr int kMmaWarp = 5;
+  static constexpr int kEwWarps = 8;  // elementwise: two per TMEM lane quarter, 32 query columns each
+  static constexpr int kThreads = 32 * (kEwWarps + 2);
+  static constexpr int kProducerWarp = kEwWarps;
+  static constexpr int kMmaWarp = kEwWarps + 1;
   static constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 128, kColDV = 256, kColDK = 384;
   static_assert(kOffQ % 1024 == 0 && kOffDS % 1024 == 0 && kQTile % 1024 == 0, "swizzle atoms");
   static_assert(kOffDQ % 128 == 0, "bulk-copy source alignment");
@@ -124,9 +126,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       mbar_init(BAR(C::kBarQEmpty + i), 1);
     }
     mbar_init(BAR(C::kBarSFull), 1);
-    mbar_init(BAR(C::kBarPDone), 4);
+    mbar_init(BAR(C::kBarPDone), C::kEwWarps);
     mbar_init(BAR(C::kBarDQFull), 1);
-    mbar_init(BAR(C::kBarDQFree), 4);
+    mbar_init(BAR(C::kBarDQFree), C::kEwWarps);
     mbar_init(BAR(C::kBarMmaDone), 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -236,9 +238,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    // ======================= elementwise warps 0-3 (thread = key of the tile) ==========
-    const int r = threadIdx.x;  // key of the tile (S^T, dP^T, dV, dK lanes); head-dim element of dQ^T
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ======================= elementwise warps 0-7 ==========
+    // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (keys for S^T, dP^T, dV, dK; head-dim
+    // elements for dQ^T) and takes query columns 32 hf .. + 31, hf = w / 4, of each tile
+    // (and half of the head-dim columns of dV and dK at the end).
+    const int hf = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;  // TMEM lane: key of the tile / head-dim element of dQ^T
+    const int tid = threadIdx.x;           // 0..255
+    const int c_off = hf * 32;             // this warp's query columns
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int key = j * 128 + r;
     const long long diag = (long long)p.Nk - p.Nq;
     float* rowbuf = reinterpret_cast<float*>(smem + C::kOffRow);  // [2][2][64]: lse2, D
@@ -247,67 +255,75 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // per-query lse (base 2) and D of query tile i into rowbuf[i & 1]: loaded a tile ahead,
     // stored to shared memory after this tile's work, so the load latency is hidden
     auto row_load = [&](int i, float& l2, float& dd) {
-      const int q = (qt0 + i) * 64 + r;
+      const int q = (qt0 + i) * 64 + tid;
       const long long o = ((long long)b * p.H + h) * p.Nq + q;
-      l2 = (r < 64 && q < p.Nq) ? __ldg(p.lse + o) * 1.4426950408889634f : 0.f;
-      dd = (r < 64 && q < p.Nq) ? __ldg(p.dsum + o) : 0.f;
+      l2 = (tid < 64 && q < p.Nq) ? __ldg(p.lse + o) * 1.4426950408889634f : 0.f;
+      dd = (tid < 64 && q < p.Nq) ? __ldg(p.dsum + o) : 0.f;
     };
     float nl2 = 0.f, ndd = 0.f;
     if (nqt > 0) {
       row_load(0, nl2, ndd);
-      if (r < 64) {
-        rowbuf[r] = nl2;
-        rowbuf[64 + r] = ndd;
+      if (tid < 64) {
+        rowbuf[tid] = nl2;
+        rowbuf[64 + tid] = ndd;
       }
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(1, 32 * C::kEwWarps);
     for (int i = 0; i < nqt; ++i) {
       const int q0 = (qt0 + i) * 64;
-      float* lse2 = rowbuf + (i & 1) * 128;
-      float* dsm = lse2 + 64;
+      const float* lse2 = rowbuf + (i & 1) * 128 + c_off;
+      const float* dsm = rowbuf + (i & 1) * 128 + 64 + c_off;
       if (i + 1 < nqt) row_load(i + 1, nl2, ndd);
       mbar_wait(BAR(C::kBarSFull), i & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
-      uint32_t s[2][32], dp[2][32];
-      tmem_ld32(tmem + lane_base + C::kColS, s[0]);
-      tmem_ld32(tmem + lane_base + C::kColS + 32, s[1]);
-      tmem_ld32(tmem + lane_base + C::kColDP, dp[0]);
-      tmem_ld32(tmem + lane_base + C::kColDP + 32, dp[1]);
+      uint32_t s[32], dp[32];
+      tmem_ld32(tmem + lane_base + C::kColS + c_off, s);
+      tmem_ld32(tmem + lane_base + C::kColDP + c_off, dp);
       tmem_ld_wait();
-      reg_order_after_wait(s[0]);
-      reg_order_after_wait(s[1]);
-      reg_order_after_wait(dp[0]);
-      reg_order_after_wait(dp[1]);
-      // query q0 + c sees this key iff key < Nk, q0 + c < Nq and (causal) key <= q0 + c + Nk - Nq
-      uint32_t pk[2][16], dk2[2][16];
+      reg_order_after_wait(s);
+      reg_order_after_wait(dp);
+      // query q0 + c sees this key iff key < Nk, q0 + c < Nq and (causal) key <= q0 + c + Nk - Nq;
+      // a key that every query of this warp's columns sees takes no per-element test
+      const int qa = q0 + c_off;
+      const bool all_see = key < p.Nk && qa + 31 < p.Nq && (!p.causal || (long long)key <= qa + diag);
+      uint32_t pk[16], dk2[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float pv[2], dv2[2];
+      for (int c8 = 0; c8 < 32; c8 += 8) {
+        const float4 la = *reinterpret_cast<const float4*>(lse2 + c8);
+        const float4 lb = *reinterpret_cast<const float4*>(lse2 + c8 + 4);
+        const float4 da = *reinterpret_cast<const float4*>(dsm + c8);
+        const float4 db = *reinterpret_cast<const float4*>(dsm + c8 + 4);
+        const float l8[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+        const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+        float pv[8], dv8[8];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = c + e;
-          const int q = q0 + col;
-          const bool ok = key < p.Nk && q < p.Nq && (!p.causal || (long long)key <= q + diag);
-          const float x = __uint_as_float(s[col >> 5][col & 31]) * p.scale_log2 - lse2[col];
-          const float pr = ok ? ex2_approx(x) : 0.f;
+        for (int e = 0; e < 8; ++e) {
+          const int col = c8 + e;
+          float pr = ex2_approx(__uint_as_float(s[col]) * p.scale_log2 - l8[e]);
+          if (!all_see) {
+            const int q = qa + col;
+            const bool ok = key < p.Nk && q < p.Nq && (!p.causal || (long long)key <= q + diag);
+            pr = ok ? pr : 0.f;
+          }
           pv[e] = pr;
-          dv2[e] = pr * (__uint_as_float(dp[col >> 5][col & 31]) - dsm[col]);
+          dv8[e] = pr * (__uint_as_float(dp[col]) - d8[e]);
         }
-        pk[c >> 5][(c & 31) >> 1] = pack2<BF16>(pv[0], pv[1]);
-        dk2[c >> 5][(c & 31) >> 1] = pack2<BF16>(dv2[0], dv2[1]);
-      }
-      // P^T and dS^T (packed pairs) into the consumed S^T / dP^T columns
-      tmem_st16(tmem + lane_base + C::kColS, pk[0]);
-      tmem_st16(tmem + lane_base + C::kColS + 16, pk[1]);
-      tmem_st16(tmem + lane_base + C::kColDP, dk2[0]);
-      tmem_st16(tmem + lane_base + C::kColDP + 16, dk2[1]);
-      // dS^T row (64 queries, 128 bytes) into shared memory, 128-byte swizzle (MN-major B)
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const uint4 w = make_uint4(dk2[cc >> 2][(cc & 3) * 4 + 0], dk2[cc >> 2][(cc & 3) * 4 + 1],
-                                   dk2[cc >> 2][(cc & 3) * 4 + 2], dk2[cc >> 2][(cc & 3) * 4 + 3]);
-        *reinterpret_cast<uint4*>(ds_row + ((cc ^ (r & 7)) << 4)) = w;
+        for (int e = 0; e < 8; e += 2) {
+          pk[(c8 + e) >> 1] = pack2<BF16>(pv[e], pv[e + 1]);
+          dk2[(c8 + e) >> 1] = pack2<BF16>(dv8[e], dv8[e + 1]);
+        }
+      }
+      // P^T and dS^T (packed pairs) into the consumed S^T / dP^T columns of this warp's queries
+      tmem_st16(tmem + lane_base + C::kColS + hf * 16, pk);
+      tmem_st16(tmem + lane_base + C::kColDP + hf * 16, dk2);
+      // dS^T row (64 queries, 128 bytes) into shared memory, 128-byte swizzle (MN-major B):
+      // this warp's four 16-byte chunks
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint4 w = make_uint4(dk2[cc * 4 + 0], dk2[cc * 4 + 1], dk2[cc * 4 + 2], dk2[cc * 4 + 3]);
+        *reinterpret_cast<uint4*>(ds_row + (((hf * 4 + cc) ^ (r & 7)) << 4)) = w;
       }
       tmem_st_wait();
       fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
@@ -315,45 +331,45 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarPDone));
 
-      // dQ^T of this tile (lane = head-dim element, 64 query columns) -> shared memory as
-      // [query][D] -> one TMA reduce-add into the fp32 accumulator (rows past Nq are skipped)
+      // dQ^T of this tile (lane = head-dim element; this warp's 32 query columns) -> shared
+      // memory as [query][D] -> one TMA reduce-add into the fp32 accumulator (rows past Nq
+      // are skipped)
       mbar_wait(BAR(C::kBarDQFull), i & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
-      uint32_t dq[2][32];
-      tmem_ld32(tmem + lane_base + C::kColDQ, dq[0]);
-      tmem_ld32(tmem + lane_base + C::kColDQ + 32, dq[1]);
+      uint32_t dq[32];
+      tmem_ld32(tmem + lane_base + C::kColDQ + c_off, dq);
       tmem_ld_wait();
-      reg_order_after_wait(dq[0]);
-      reg_order_after_wait(dq[1]);
+      reg_order_after_wait(dq);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarDQFree));
-      if (r == 0) bulk_wait_group_read0();  // the previous tile's reduce has read the stage
-      named_bar_sync(1, 128);
+      if (tid == 0) bulk_wait_group_read0();  // the previous tile's reduce has read the stage
+      named_bar_sync(1, 32 * C::kEwWarps);
       if (r < D) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) dq_stage[c * D + r] = __uint_as_float(dq[c >> 5][c & 31]);
+        for (int c = 0; c < 32; ++c) dq_stage[(c_off + c) * D + r] = __uint_as_float(dq[c]);
       }
       fence_proxy_async_smem();  // generic-proxy writes -> visible to the TMA
       // next tile's per-query rows, loaded at the top of this iteration
-      if (i + 1 < nqt && r < 64) {
-        rowbuf[((i + 1) & 1) * 128 + r] = nl2;
-        rowbuf[((i + 1) & 1) * 128 + 64 + r] = ndd;
+      if (i + 1 < nqt && tid < 64) {
+        rowbuf[((i + 1) & 1) * 128 + tid] = nl2;
+        rowbuf[((i + 1) & 1) * 128 + 64 + tid] = ndd;
       }
-      named_bar_sync(1, 128);
-      if (r == 0 && !*abort_flag) {
+      named_bar_sync(1, 32 * C::kEwWarps);
+      if (tid == 0 && !*abort_flag) {
         tma_reduce_add_4d(&p.tm_dq, sbase + C::kOffDQ, 0, h, q0, b);
         bulk_commit_group();
       }
     }
-    if (r == 0) bulk_wait_group_read0();  // ... and the last one before the CTA exits
-    if (r == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (tid == 0) bulk_wait_group_read0();  // ... and the last one before the CTA exits
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 
-    // ---- epilogue: dV and scale * dK (lane = key) -> 16-bit -> global.  The last tile's
-    // dQ^T commit covered every earlier product, so dV and dK are final here.  The TMEM
-    // loads are warp-collective: every lane takes part, and only rows of keys below Nk
-    // are stored (the last key tile may be partial).
+    // ---- epilogue: dV and scale * dK (lane = key) -> 16-bit -> global; this warp takes
+    // head-dim columns hf * D / 2 .. + D / 2.  The last tile's dQ^T commit covered every
+    // earlier product, so dV and dK are final here.  The TMEM loads are warp-collective:
+    // every lane takes part, and only rows of keys below Nk are stored (the last key tile
+    // may be partial).
     const bool key_row = key < p.Nk;
     const long long row = (((long long)b * p.Nk + (key_row ? key : 0)) * p.H + h) * D;
     uint4* dvrow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dv) + row * 2);
@@ -361,7 +377,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     if (nqt == 0) {  // no query sees this key tile
       if (key_row) {
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
+        for (int c = hf * D / 16; c < (hf + 1) * D / 16; ++c) {
           dvrow[c] = make_uint4(0u, 0u, 0u, 0u);
           dkrow[c] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -369,7 +385,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     } else {
       tc_fence_after_sync();
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = hf * D / 64; c < (hf + 1) * D / 64; ++c) {
         uint32_t a[32], k2[32];
         tmem_ld32(tmem + lane_base + C::kColDV + c * 32, a);
         tmem_ld32(tmem + lane_base + C::kColDK + c * 32, k2);
