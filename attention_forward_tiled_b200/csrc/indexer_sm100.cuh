@@ -492,6 +492,7 @@ __global__ void __launch_bounds__(kTopkThreads)
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;   // entries still to choose among those matching the prefix
   bool take_all = false;
+  bool few = false;    // the prefix is shared by at most 32 keys: they are sorted by one warp
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
     __syncthreads();
@@ -550,15 +551,71 @@ __global__ void __launch_bounds__(kTopkThreads)
     remaining = ctl[1];
     prefix |= (uint32_t)sel << shift;
     pmask |= 255u << shift;
+    if (shift > 0 && shift <= 16 && ctl[2] <= 32) {  // the rest of the digits are not needed
+      few = true;
+      break;
+    }
   }
   const uint32_t thr = prefix;  // the k-th largest key (unless take_all)
   const int eq_total = ctl[2];   // entries equal to thr (last pass)
   __syncthreads();
+  if (few) {
+    // ---- gather: keys whose decided top digits exceed the prefix (all chosen, any order)
+    // and the <= 32 keys that share it, of which one warp keeps the `remaining` first in
+    // the output order (larger key, then lower position)
+    uint32_t* candk = hist;                                 // [32]
+    int* candi = reinterpret_cast<int*>(hist + 32);         // [32]
+    if (tid == 0) {
+      ctl[3] = 0;
+      ctl[4] = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < P; i += kTopkThreads) {
+      const uint32_t u = key_at(i);
+      const uint32_t hb = u & pmask;
+      if (u != 0u && hb > prefix) {
+        const int slot = atomicAdd(&ctl[3], 1);
+        ckey[slot] = u;
+        cidx[slot] = i;
+      } else if (u != 0u && hb == prefix) {
+        const int slot = atomicAdd(&ctl[4], 1);
+        candk[slot] = u;
+        candi[slot] = i;
+      }
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const int nc = ctl[4], above = ctl[3];
+      uint32_t kx = tid < nc ? candk[tid] : 0u;
+      int ix = tid < nc ? candi[tid] : 0x7fffffff;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+        const bool desc = (tid & size) == 0;
+#pragma unroll
+        for (int st = size >> 1; st >= 1; st >>= 1) {
+          const uint32_t ky = __shfl_xor_sync(0xffffffffu, kx, st);
+          const int iy = __shfl_xor_sync(0xffffffffu, ix, st);
+          const bool y_first = ky > kx || (ky == kx && iy < ix);
+          if (((tid & st) == 0) == (desc == y_first)) {
+            kx = ky;
+            ix = iy;
+          }
+        }
+      }
+      if (tid < remaining) {
+        ckey[above + tid] = kx;
+        cidx[above + tid] = ix;
+      }
+      __syncwarp();
+      if (tid == 0) ctl[3] = above + remaining;
+    }
+    __syncthreads();
+  }
   // ---- gather: keys above thr in any order, then the `remaining` lowest positions with key thr
-  if (tid == 0) ctl[3] = 0;
+  if (!few && tid == 0) ctl[3] = 0;
   __syncthreads();
   const bool ties_all = take_all || eq_total == remaining;
-  for (int i = tid; i < P; i += kTopkThreads) {
+  for (int i = few ? P : tid; i < P; i += kTopkThreads) {
     const uint32_t u = key_at(i);
     if (u != 0u && (take_all ? true : (u > thr || (ties_all && u == thr)))) {
       const int slot = atomicAdd(&ctl[3], 1);
@@ -567,7 +624,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     }
   }
   __syncthreads();
-  if (!ties_all) {  // ties at thr: the lowest positions, in position order
+  if (!few && !ties_all) {  // ties at thr: the lowest positions, in position order
     int base = 0;
     const int above = ctl[3];
     for (int c0 = 0; c0 < P; c0 += kTopkThreads) {
