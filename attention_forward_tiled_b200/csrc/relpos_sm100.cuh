@@ -12,21 +12,21 @@
 // steps (128 keys) the distances met span at most 255 consecutive embedding rows
 // (lo ... lo + 254, clamped at 0 and 2R), so on every other step the tensor core computes
 // G = Q E_win^T (N = 256: TMEM lane = query row, column = window row) next to S = Q K^T,
-// and the next window has a whole step to arrive.  Query row r needs the columns dist(r, j) - lo for its 64 keys of
-// a step, a run of at most 64 that starts at a row-dependent column: each softmax thread
-// copies the 112 columns that cover its warp's runs into its own shared-memory row (pitch
-// 116 words, so the copy and the skewed reads are free of bank conflicts) and gathers from
-// there; no other thread reads the row, so no barrier is needed.  Roles (192 threads):
-//   * warp 4, producer: Q of each unit as soon as the previous unit's last product has read
+// and the next window has a whole step to arrive.  Query row r needs the columns
+// dist(r, j) - lo for its 64 keys of a step, a run of at most 64 that starts at a
+// row-dependent column: the two softmax warps of a row copy the 112 columns that cover
+// their runs into the row's shared-memory line (pitch 116 words, so the copy and the
+// skewed reads are free of bank conflicts) and gather from there.  Roles (320 threads):
+//   * warp 8, producer: Q of each unit as soon as the previous unit's last product has read
 //     it, the K/V ring (two stages), the embedding window of each step pair as soon as the
 //     previous pair's product has read the buffer (so the next unit's loads run behind the
 //     current unit's last step and epilogue);
-//   * warp 5, MMA issuer: S (and G) of step t, then O += P V of step t - 1 once P is ready;
-//   * warps 0-3, softmax (thread = query row): copy and gather G, online softmax (fp16 P
-//     into shared memory, in the K slot of the step at d = 128; O rescaled in TMEM when
-//     the row maximum grows), and the O / l epilogue.  For bf16 inputs they convert each V
-//     tile to fp16 in place first (P V runs in fp16, as in the plain kernel; magnitudes
-//     with no fp16 value set the range status).
+//   * warp 9, MMA issuer: S (and G) of step t, then O += P V of step t - 1 once P is ready;
+//   * warps 0-7, softmax (two warps per query row, 32 keys of a step each): copy and
+//     gather G, online softmax (fp16 P into shared memory, in the K slot of the step at
+//     d = 128; O rescaled in TMEM when the row maximum grows), and the O / l epilogue.  For
+//     bf16 inputs they convert each V tile to fp16 in place first (P V runs in fp16, as in
+//     the plain kernel; magnitudes with no fp16 value set the range status).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -65,25 +65,27 @@ struct RelposCfg {
   static constexpr int kOffE = kOffV + 2 * kKVBytes;    // embedding window
   static constexpr int kOffP = kOffE + kEBytes;         // 128 x 64 fp16, 128B swizzle (D = 64)
   static constexpr int kOffG = kOffP + (kPInK ? 0 : 128 * 128);  // [128 rows][kGPitch] fp32
-  static constexpr int kOffBar = kOffG + 128 * kGPitch * 4;
+  static constexpr int kOffX = kOffG + 128 * kGPitch * 4;  // [max, sum][half][128 rows] fp32
+  static constexpr int kOffBar = kOffX + 2 * 2 * 128 * 4;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKVFull = 1;   // [2]
   static constexpr int kBarKVEmpty = 3;  // [2]
   static constexpr int kBarEFull = 5;
   static constexpr int kBarSFull = 6;    // S (and G, even steps) of the step are in TMEM
-  static constexpr int kBarSFree = 7;    // ... and have been read (4 arrivals)
-  static constexpr int kBarPFull = 8;    // P written, O rescaled, V converted (4 arrivals)
+  static constexpr int kBarSFree = 7;    // ... and have been read (8 arrivals)
+  static constexpr int kBarPFull = 8;    // P written, O rescaled, V converted (8 arrivals)
   static constexpr int kBarPVDone = 9;   // O += P V of the step has completed
   static constexpr int kBarMmaDone = 10;
   static constexpr int kBarEFree = 11;   // the G product of a step pair has read the window
   static constexpr int kBarQFree = 12;   // the last product of a unit has read Q
-  static constexpr int kBarOFree = 13;   // the epilogue of a unit has read O (4 arrivals)
+  static constexpr int kBarOFree = 13;   // the epilogue of a unit has read O (8 arrivals)
   static constexpr int kNumBars = 14;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // +1024: manual 1 KB alignment
-  static constexpr int kThreads = 192;
-  static constexpr int kProducerWarp = 4;
-  static constexpr int kMmaWarp = 5;
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
   // TMEM columns; a warp's G loads start at most 224 columns past kColG and read 128
   // (past column 383 they read values no thread uses)
   static constexpr uint32_t kColO = 0;    // D columns
@@ -111,16 +113,24 @@ __device__ __forceinline__ int relpos_lo(const RelposParams& p, int q0, int k0) 
 }
 
 
-// Softmax warps 0-3: thread = query row q0 + r of the tile (TMEM lane r).
+// Softmax warps 0-7: warps w and w + 4 share query rows 32 (w % 4) .. + 31 (TMEM lanes)
+// and take keys 32 hf .. + 31 of each 64-key step, hf = w / 4.  The pair copies the two
+// halves of its rows' G window, exchanges the half-row maxima and the final row sums
+// through shared memory (64-thread named barriers 2 + w % 4), and splits the O rescale and
+// the epilogue by head-dim halves.
 template <int D, bool BF16>
 __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* smem, uint32_t tmem,
                                                uint64_t* bars, const WaitCtx& wctx) {
   using C = RelposCfg<D>;
   auto BAR = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = threadIdx.x;  // row of the tile
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int qw = warp & 3, hf = warp >> 2;
+  const int r = qw * 32 + lane;  // row of the tile
+  const int tid = threadIdx.x;   // 0..255
+  const uint32_t pair_bar = 2 + qw;
+  const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
   float* grow = reinterpret_cast<float*>(smem + C::kOffG) + r * C::kGPitch;  // this row's G
+  float* xch = reinterpret_cast<float*>(smem + C::kOffX);  // [max, sum][half][128 rows]
   const int shift = p.Nk - p.Nq;  // bottom-right causal alignment
   uint32_t vmag = 0;              // bf16: largest |V| bit pattern converted
   int g = 0;                      // steps of this CTA so far (barrier phases)
@@ -130,8 +140,8 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
   const int h = (u / p.n_qtiles) % p.H, b = u / (p.n_qtiles * p.H);
   const int i = q0 + r;
   const int nsteps = relpos_steps(p, q0);
-  float m = -INFINITY;            // running maximum of scale * log2(e) * score
-  float l0 = 0.f, l1 = 0.f;       // sum of the fp16-rounded P the tensor core multiplies
+  float m = -INFINITY;            // running maximum of scale * log2(e) * score (whole row)
+  float l0 = 0.f, l1 = 0.f;       // this warp's sum of the fp16-rounded P
 
   for (int t = 0; t < nsteps; ++t, ++g) {
     const int k0 = t * 64;
@@ -139,39 +149,38 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     mbar_wait(BAR(C::kBarSFull), g & 1, wctx);
     __syncwarp();
     tc_fence_after_sync();
-    // ---- this warp's rows need window columns cw ... cw + 94 (the clamp is monotone and
-    // moves by at most one per row or key): load the 128 from the 32-aligned column below
-    // and keep the 112 from base + s0, s0 = 0 or 16, which hold them
-    const int cw = min(max(q0 + warp * 32 - (k0 + 63), -p.R), p.R) + p.R - lo;
+    // ---- these rows need window columns cw ... cw + 94 (the clamp is monotone and moves
+    // by at most one per row or key): of the 128 from the 32-aligned column below, the 112
+    // from base + s0 (s0 = 0 or 16) hold them; this warp copies the half hf of the 128
+    const int cw = min(max(q0 + qw * 32 - (k0 + 63), -p.R), p.R) + p.R - lo;
     const int s0 = (cw & 31) & 16;
     const int base = (cw & ~31) + s0;  // column of grow[0]
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-      uint32_t g[32];
-      tmem_ld32(tmem + lane_base + C::kColG + (cw & ~31) + q * 32, g);
+    for (int q = 2 * hf; q < 2 * hf + 2; ++q) {
+      uint32_t gv[32];
+      tmem_ld32(tmem + lane_base + C::kColG + (cw & ~31) + q * 32, gv);
       tmem_ld_wait();
-      reg_order_after_wait(g);
+      reg_order_after_wait(gv);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int dst = q * 32 + 4 * u - s0;
+      for (int e = 0; e < 8; ++e) {
+        const int dst = q * 32 + 4 * e - s0;
         if (dst >= 0 && dst < C::kGCols)  // uniform over the warp
           *reinterpret_cast<float4*>(grow + dst) =
-              make_float4(__uint_as_float(g[4 * u]), __uint_as_float(g[4 * u + 1]),
-                          __uint_as_float(g[4 * u + 2]), __uint_as_float(g[4 * u + 3]));
+              make_float4(__uint_as_float(gv[4 * e]), __uint_as_float(gv[4 * e + 1]),
+                          __uint_as_float(gv[4 * e + 2]), __uint_as_float(gv[4 * e + 3]));
       }
     }
-    // ---- this row's 64 raw scores
-    uint32_t sv[2][32];
-    tmem_ld32(tmem + lane_base + C::kColS, sv[0]);
-    tmem_ld32(tmem + lane_base + C::kColS + 32, sv[1]);
+    // ---- this row's 32 raw scores of this warp's keys
+    uint32_t sv[32];
+    tmem_ld32(tmem + lane_base + C::kColS + hf * 32, sv);
     tmem_ld_wait();
-    reg_order_after_wait(sv[0]);
-    reg_order_after_wait(sv[1]);
+    reg_order_after_wait(sv);
     tc_fence_before_sync();
     __syncwarp();
     if (lane == 0) mbar_arrive(BAR(C::kBarSFree));  // S and G may be overwritten
+    named_bar_sync(pair_bar, 64);                    // both halves of the rows are copied
     // ---- add the gathered term, scale, mask
-    float x[64];
+    float x[32];
     float mx = -INFINITY;
     // keys k0 + jj with jj < jlim are allowed for this row (tail and bottom-right causal)
     const int jlim = i < p.Nq ? (p.causal ? min(p.Nk, i + shift + 1) : p.Nk) - k0 : 0;
@@ -181,46 +190,50 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     const bool unclamped = i - (k0 + min(63, jlim - 1)) >= -p.R && i - k0 <= p.R;
     if (jlim <= 0) {  // the row sees no key of this step
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) x[jj] = -INFINITY;
+      for (int e = 0; e < 32; ++e) x[e] = -INFINITY;
     } else if (unclamped) {
       // key jj's column is (key k0's column) - jj
-      const float* gp = grow + (i - k0 + p.R - lo - base);
+      const float* gp = grow + (i - k0 + p.R - lo - base) - hf * 32;
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        x[jj] = jj < jlim ? (__uint_as_float(sv[jj >> 5][jj & 31]) + gp[-jj]) * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[jj]);
+      for (int e = 0; e < 32; ++e) {
+        x[e] = hf * 32 + e < jlim ? (__uint_as_float(sv[e]) + gp[-e]) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[e]);
       }
     } else {
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        const int j = k0 + jj;
+      for (int e = 0; e < 32; ++e) {
+        const int j = k0 + hf * 32 + e;
         const bool allowed = i < p.Nq && j < p.Nk && (!p.causal || j <= i + shift);
         // column of key j in this row's copy
         const int c = min(max(i - j, -p.R), p.R) + p.R - lo - base;
-        const float g = grow[c];
-        x[jj] = allowed ? (__uint_as_float(sv[jj >> 5][jj & 31]) + g) * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[jj]);
+        const float gg = grow[c];
+        x[e] = allowed ? (__uint_as_float(sv[e]) + gg) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[e]);
       }
     }
+    // ---- the row maximum from both halves (after this barrier both warps are also done
+    // reading the copied row)
+    xch[hf * 128 + r] = mx;
+    named_bar_sync(pair_bar, 64);
+    const float m_new = fmaxf(m, fmaxf(mx, xch[(hf ^ 1) * 128 + r]));
     // ---- online softmax: O and the P buffer are free once the previous P V is done
-    const float m_new = fmaxf(m, mx);
     if (t >= 1) {
       mbar_wait(BAR(C::kBarPVDone), (g - 1) & 1, wctx);
       __syncwarp();
       tc_fence_after_sync();
-      const bool grow = m_new > m && m > -INFINITY;
-      if (__any_sync(0xffffffffu, grow)) {  // TMEM loads and stores are warp-collective
-        const float f = grow ? ex2_approx(m - m_new) : 1.0f;
+      const bool grow_m = m_new > m && m > -INFINITY;
+      if (__any_sync(0xffffffffu, grow_m)) {  // TMEM loads and stores are warp-collective
+        const float f = grow_m ? ex2_approx(m - m_new) : 1.0f;
         l0 *= f;
         l1 *= f;
 #pragma unroll 1
-        for (int cq = 0; cq < D / 32; ++cq) {
+        for (int cq = hf * (D / 64); cq < (hf + 1) * (D / 64); ++cq) {  // this warp's half of O
           uint32_t o[32];
           tmem_ld32(tmem + lane_base + C::kColO + cq * 32, o);
           tmem_ld_wait();
           reg_order_after_wait(o);
 #pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * f);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
           tmem_st32(tmem + lane_base + C::kColO + cq * 32, o);
         }
         tmem_st_wait();
@@ -228,24 +241,24 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     }
     m = m_new;
     const float mu = m == -INFINITY ? 0.f : m;  // a row that saw no key yet: every P is 0
-    uint32_t pk[32];
+    uint32_t pk[16];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      pk[u] = pack2<false>(ex2_approx(x[2 * u] - mu), ex2_approx(x[2 * u + 1] - mu));
-      add_f16x2_f32(l0, l1, pk[u]);
+    for (int e = 0; e < 16; ++e) {
+      pk[e] = pack2<false>(ex2_approx(x[2 * e] - mu), ex2_approx(x[2 * e + 1] - mu));
+      add_f16x2_f32(l0, l1, pk[e]);
     }
-    // P row r: 64 fp16 = eight 16-byte chunks, 128-byte swizzle (K-major A operand); at
-    // d = 128 in the step's K slot, which S has finished reading
+    // P row r: 64 fp16 = eight 16-byte chunks, 128-byte swizzle (K-major A operand); this
+    // warp's four; at d = 128 in the step's K slot, which S has finished reading
     uint8_t* sp = smem + (C::kPInK ? C::kOffK + (g & 1) * C::kKVBytes : C::kOffP);
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc)
-      *reinterpret_cast<uint4*>(sp + r * 128 + ((cc ^ (r & 7)) << 4)) =
+    for (int cc = 0; cc < 4; ++cc)
+      *reinterpret_cast<uint4*>(sp + r * 128 + (((hf * 4 + cc) ^ (r & 7)) << 4)) =
           make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
     if constexpr (BF16) {  // V of this step to fp16, in place
       mbar_wait(BAR(C::kBarKVFull + (g & 1)), (g >> 1) & 1, wctx);
       uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffV + (g & 1) * C::kKVBytes);
 #pragma unroll 2
-      for (int c = r; c < C::kKVBytes / 16; c += 128) {
+      for (int c = tid; c < C::kKVBytes / 16; c += 256) {
         uint4 w = tile[c];
         vmag = __vmaxu2(vmag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
                                        __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
@@ -262,8 +275,11 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     if (lane == 0) mbar_arrive(BAR(C::kBarPFull));
   }
 
-  // ---- epilogue: O / l in the input dtype, lse = ln(sum exp(scale * score))
-  const float l = l0 + l1;
+  // ---- epilogue: O / l in the input dtype (this warp's half of the head dim), lse =
+  // ln(sum exp(scale * score)); the row sum adds both warps' halves
+  xch[256 + hf * 128 + r] = l0 + l1;
+  named_bar_sync(pair_bar, 64);
+  const float l = l0 + l1 + xch[256 + (hf ^ 1) * 128 + r];
   const float inv = l > 0.f ? 1.0f / l : 0.f;
   const bool row_ok = i < p.Nq;
   uint4* orow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) +
@@ -273,19 +289,19 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     __syncwarp();
     tc_fence_after_sync();
 #pragma unroll 1
-    for (int cq = 0; cq < D / 32; ++cq) {
+    for (int cq = hf * (D / 64); cq < (hf + 1) * (D / 64); ++cq) {
       uint32_t o[32];
       tmem_ld32(tmem + lane_base + C::kColO + cq * 32, o);
       tmem_ld_wait();
       reg_order_after_wait(o);
       if (row_ok) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          orow[cq * 4 + u] = make_uint4(
-              pack2<BF16>(__uint_as_float(o[8 * u]) * inv, __uint_as_float(o[8 * u + 1]) * inv),
-              pack2<BF16>(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv),
-              pack2<BF16>(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv),
-              pack2<BF16>(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv));
+        for (int e = 0; e < 4; ++e)
+          orow[cq * 4 + e] = make_uint4(
+              pack2<BF16>(__uint_as_float(o[8 * e]) * inv, __uint_as_float(o[8 * e + 1]) * inv),
+              pack2<BF16>(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv),
+              pack2<BF16>(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv),
+              pack2<BF16>(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
       }
     }
     // O may be overwritten by the next unit's first P V
@@ -294,9 +310,9 @@ __device__ __forceinline__ void relpos_softmax(const RelposParams& p, uint8_t* s
     if (lane == 0) mbar_arrive(BAR(C::kBarOFree));
   } else if (row_ok) {  // no key reaches this tile
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+    for (int c = hf * (D / 16); c < (hf + 1) * (D / 16); ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
   }
-  if (row_ok && p.lse != nullptr)
+  if (row_ok && hf == 0 && p.lse != nullptr)
     p.lse[((long long)b * p.H + h) * p.Nq + i] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
   }  // units
   if constexpr (BF16) {
@@ -336,13 +352,13 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
     }
     mbar_init(BAR(C::kBarEFull), 1);
     mbar_init(BAR(C::kBarSFull), 1);
-    mbar_init(BAR(C::kBarSFree), 4);
-    mbar_init(BAR(C::kBarPFull), 4);
+    mbar_init(BAR(C::kBarSFree), C::kSoftmaxWarps);
+    mbar_init(BAR(C::kBarPFull), C::kSoftmaxWarps);
     mbar_init(BAR(C::kBarPVDone), 1);
     mbar_init(BAR(C::kBarMmaDone), 1);
     mbar_init(BAR(C::kBarEFree), 1);
     mbar_init(BAR(C::kBarQFree), 1);
-    mbar_init(BAR(C::kBarOFree), 4);
+    mbar_init(BAR(C::kBarOFree), C::kSoftmaxWarps);
     *abort_flag = 0;
     mbar_init_fence();
   }

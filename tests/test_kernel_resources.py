@@ -21,7 +21,7 @@ THREADS = {"attn_prefill_kernel": 384, "attn_decode_partial_kernel": 160,
            "attn_decode_combine_kernel": 128, "attn_mq_partial_kernel": 192,
            "attn_mq_combine_kernel": 128, "attn_indexer_score_kernel": 352,
            "attn_topk_kernel": 512, "attn_bwd_kernel": 320, "attn_bwd_pre_kernel": 128,
-           "attn_bwd_dq_kernel": 256, "attn_relpos_kernel": 192}
+           "attn_bwd_dq_kernel": 256, "attn_relpos_kernel": 320}
 # bytes of spill stores / loads per prefill instantiation (head_dim, bf16) at this version
 PREFILL_SPILL_CEILING = {(64, False): (112, 168), (64, True): (152, 300),
                          (128, False): (8, 8), (128, True): (16, 16)}
