@@ -409,20 +409,44 @@ __global__ void __launch_bounds__(RelposCfg<D>::kThreads, 1)
           tma_load_4d_w(sbase + C::kOffV + s * C::kKVBytes + bx * 8192, &p.tm_v, BAR(C::kBarKVFull + s),
                         bx * 64, h, k0, b);
         }
-        if (t & 1) continue;  // one window per step pair
-        // one window buffer: the previous pair's G product must have read it
-        if (ge >= 1) mbar_wait(BAR(C::kBarEFree), (ge - 1) & 1, wctx);
-        __syncwarp();
-        if (warp_flag(abort_flag)) {
+        // embedding windows, one per step pair, in the order the products take them: the
+        // first before any product needs it, then the next pair's as soon as this pair's
+        // K/V loads are issued (it only waits for this pair's G product to read the buffer)
+        auto load_window = [&](int lo) {
+          if (ge >= 1) mbar_wait(BAR(C::kBarEFree), (ge - 1) & 1, wctx);
+          __syncwarp();
+          if (warp_flag(abort_flag)) return false;
+          mbar_arrive_expect_tx_w(BAR(C::kBarEFull), C::kEBytes);
+          for (int bx = 0; bx < C::kBoxes; ++bx)  // rows past n_emb read as zeros and are never used
+            tma_load_3d_w(sbase + C::kOffE + bx * C::kEBoxBytes, &p.tm_e, BAR(C::kBarEFull), bx * 64, lo, 0);
+          ++ge;
+          return true;
+        };
+        bool ok = true;
+        if (ge == 0) ok = load_window(relpos_lo(p, q0, k0));
+        if (ok && ((t & 1) || t == nsteps - 1)) {  // last step of its pair
+          int lon = 0;
+          bool has_next = false;
+          if (t + 1 < nsteps) {
+            lon = relpos_lo(p, q0, (t + 1) * 64);
+            has_next = true;
+          } else {
+            for (int u2 = u + (int)gridDim.x; u2 < p.n_units; u2 += gridDim.x) {
+              const int q2 = (u2 % p.n_qtiles) * 128;
+              if (relpos_steps(p, q2) > 0) {
+                lon = relpos_lo(p, q2, 0);
+                has_next = true;
+                break;
+              }
+            }
+          }
+          if (has_next) ok = load_window(lon);
+        }
+        if (!ok) {
           ++g;  // this step's K/V copy is in flight
           stop = true;
           break;
         }
-        const int lo = relpos_lo(p, q0, k0);
-        mbar_arrive_expect_tx_w(BAR(C::kBarEFull), C::kEBytes);
-        for (int bx = 0; bx < C::kBoxes; ++bx)  // rows past n_emb read as zeros and are never used
-          tma_load_3d_w(sbase + C::kOffE + bx * C::kEBoxBytes, &p.tm_e, BAR(C::kBarEFull), bx * 64, lo, 0);
-        ++ge;
       }
     }
     if (lane == 0 && *abort_flag) {
