@@ -102,3 +102,48 @@ def test_topk_distinct_scores_large_rows():
     idx = topk(s.cuda(), 300)
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), oracle.topk(s.double().numpy(), 300))
+
+
+def _rows_few_candidates(P, k, seed):
+    """Rows whose k-th largest score falls in a radix bin of at most 32 keys after the
+    second (or third) 8-bit digit, so the selection sorts those candidates in one warp:
+    a background well below, `above` scores that are all chosen, and candidates that
+    share the decided top digits (1 + m 2^-15 + j 2^-23 is exact in fp32)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    rows = []
+    one = 1.0
+    for above, cand in [
+        (k - 1, [one + j * 2.0 ** -20 for j in range(20)]),                  # one of 20 distinct
+        (k - 7, [one + j * 2.0 ** -20 for j in (5, 5, 5, 3, 3, 9, 1, 1, 0, 7, 7, 7, 2)]),
+        (k - 32, [one + j * 2.0 ** -21 for j in range(32)]),                  # every candidate
+        (k - 10, [one] * 16),                                                 # equal: by position
+    ]:
+        s = torch.randn(P, generator=g) * 0.1 - 4.0
+        vals = torch.cat([2.0 + torch.rand(above, generator=g), torch.tensor(cand)])
+        pos = torch.randperm(P, generator=g)[: vals.numel()]
+        s[pos] = vals
+        rows.append(s)
+    # third digit: 100 keys share the top 16 bits; the k-th falls in a bin of 20 of them
+    s = torch.randn(P, generator=g) * 0.1 - 4.0
+    m_above = [one + m * 2.0 ** -15 for m in range(100 - (k - 11), 100)]   # k - 11 above
+    m_below = [one + m * 2.0 ** -15 for m in range(0, 40)]
+    cand = [one + 50 * 2.0 ** -15 + j * 2.0 ** -23 for j in (4, 4, 0, 19, 7, 7, 7, 3, 12, 12, 1, 5,
+                                                             6, 8, 9, 10, 11, 13, 14, 15)]
+    vals = torch.tensor(m_above + m_below + cand)
+    pos = torch.randperm(P, generator=g)[: vals.numel()]
+    s[pos] = vals
+    rows.append(s)
+    return torch.stack(rows).float()
+
+
+@pytest.mark.parametrize("P", [5000, 60000])
+def test_topk_few_candidates(P):
+    """The selection's short path (<= 32 keys left after two or three digits), with ties
+    among the candidates and on either side of the cut, from shared memory (P = 5000) and
+    from global memory (P = 60000), against the oracle bit for bit."""
+    k = 60
+    s = _rows_few_candidates(P, k, seed=P)
+    idx = topk(s.cuda(), k)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(s.double().numpy(), k))

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from attention_forward_tiled_b200 import attn_fwd_relpos, get_status
+from attention_forward_tiled_b200 import ATTN_ERR_RANGE, attn_fwd_relpos, get_status
 from attention_forward_tiled_b200.inputs import RELPOS_WORKLOADS, make_relpos_inputs
 from parity import assert_lse_close, assert_o_close
 
@@ -107,3 +107,26 @@ def test_relpos_full_workload_sampled():
         what = f"relpos_block200 block {bb}"
         assert_o_close(out[bb:bb + 1].cpu(), ref_o, q.dtype, what)
         assert_lse_close(lse[bb:bb + 1].cpu(), ref_lse, what)
+
+
+def test_relpos_bf16_values_outside_the_fp16_range():
+    """P V runs in fp16 here as in the plain kernel: a bf16 V element with no fp16 value
+    records ATTN_ERR_RANGE; the largest bf16 value below fp16's limit (65280) does not.  The
+    other head's output and every lse then match the oracle."""
+    q, k, v, emb = make_relpos_inputs(1, 2, 200, 200, 128, 30, dtype="bf16", seed=21)
+    qd, kd, ed = q.cuda(), k.cuda(), emb.cuda()
+    for bad in (1e5, -1e5, float("inf"), 65536.0):
+        vb = v.clone()
+        vb[0, 150, 1, 77] = bad
+        attn_fwd_relpos(qd, kd, vb.cuda(), ed, 30)
+        torch.cuda.synchronize()
+        assert get_status() == ATTN_ERR_RANGE, bad
+    vb = v.clone()
+    vb[0, 150, 1, 77] = 65280.0
+    out, lse = attn_fwd_relpos(qd, kd, vb.cuda(), ed, 30)
+    torch.cuda.synchronize()
+    assert get_status() == 0
+    ref_o, ref_lse = oracle.attn_fwd_relpos(q, k, vb, emb, clamped_dist(200, 200, 30),
+                                            scale=1.0 / math.sqrt(128))
+    assert_o_close(out[:, :, :1], ref_o[:, :, :1], q.dtype, "relpos bf16 V at 65280, head 0")
+    assert_lse_close(lse, ref_lse, "relpos bf16 V at 65280")
