@@ -97,6 +97,16 @@ struct PrefillCfg {
   static constexpr int kMmaWarp = 9;
   static constexpr int kConvWarp0 = 10;
   static constexpr int kUnitReaders = 11;  // warps that read each published unit: 8 softmax, MMA, 2 converter
+  // Registers per thread: 168 at launch (the 64 K file over 384 threads).  The file is split
+  // into four 16 K sub-partitions, and warp w runs on sub-partition w % 4, so each one holds
+  // two softmax warps and one warp of warpgroup 2 (producer, MMA issuer, converters).  At
+  // d = 64 warpgroup 2 gives registers up and the softmax warps take them, sub-partition by
+  // sub-partition: 2 x 208 + 88 = 3 x 168, so every thread keeps its 128 scores in registers.
+  static constexpr int kLaunchRegs = 168;
+  static constexpr int kRegsSoftmax = 208;
+  static constexpr int kRegsAux = 88;
+  static_assert(2 * kRegsSoftmax + kRegsAux == 3 * kLaunchRegs && kLaunchRegs * kThreads <= 65536,
+                "register split must add up to the launch's registers");
   // barrier indices
   static constexpr int kBarQFull = 0;      // [2] Q_t landed
   static constexpr int kBarQEmpty = 2;     // [2] last S_t of the unit done: Q_t buffer free
@@ -431,7 +441,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
   // Returns the k-th unit (nmax < 0: no more) after this warp has read it and released
   // its slot.
   auto next_unit = [&](int k) -> PrefillUnit {
-    mbar_wait(BAR(C::kBarUnitFull + (k & 1)), (k >> 1) & 1, wctx);
+    mbar_wait_inline(BAR(C::kBarUnitFull + (k & 1)), (k >> 1) & 1, wctx);
     __syncwarp();
     const volatile int* us = unit_slot + (k & 1) * kUnitInts;
     PrefillUnit u;
@@ -450,345 +460,353 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
 
   static_assert(C::kProducerWarp == 8 && C::kMmaWarp == 9 && C::kConvWarp0 == 10 && C::kThreads == 384,
                 "warpgroup 2 = producer, MMA issuer, two converter warps");
-  if (warp == C::kProducerWarp) {
-    // ======================= producer: unit claims + TMA loads ======================
-    if (lane == 0) {
-      tma_prefetch_map(&p.tm_q);
-      tma_prefetch_map(&p.tm_k);
-      tma_prefetch_map(&p.tm_v);
-      tma_prefetch_map(&p.tm_o);
-    }
-    __syncwarp();
-    int unit = blockIdx.x;  // the first unit is this CTA's own
-    int nq[2] = {0, 0};     // Q loads issued per tile
-    bool q_pending[2] = {false, false};
-    int g = 0;              // ring items issued
-    int nclaim = 0;
-    for (int k = 0;; ++k) {
-      PrefillUnit u;
-      if (unit >= 0) {
-        u = prefill_unit(p, unit);
-      } else {
-        u.id = -1;
-        u.b = u.h = u.row0[0] = u.row0[1] = u.nkv[0] = u.nkv[1] = 0;
-        u.nmax = -1;
-      }
-      if (k >= 2) mbar_wait(BAR(C::kBarUnitEmpty + (k & 1)), ((k >> 1) - 1) & 1, wctx);
-      __syncwarp();
+  // Roles.  setmaxnreg must dominate the code it governs, so each warpgroup's re-balance
+  // (d = 64) opens its branch and the return to the launch's count closes it.
+  if (warp >= C::kProducerWarp) {
+    // warpgroup 2: producer, MMA issuer, converters
+    if constexpr (C::kDecoupled) warpgroup_reg_dealloc<C::kRegsAux>();
+    if (warp == C::kProducerWarp) {
+      // ======================= producer: unit claims + TMA loads ======================
       if (lane == 0) {
-        volatile int* us = unit_slot + (k & 1) * kUnitInts;
-        us[0] = u.id;
-        us[1] = u.b;
-        us[2] = u.h;
-        us[3] = u.row0[0];
-        us[4] = u.row0[1];
-        us[5] = u.nkv[0];
-        us[6] = u.nkv[1];
-        us[7] = u.nmax;
-        mbar_arrive(BAR(C::kBarUnitFull + (k & 1)));
+        tma_prefetch_map(&p.tm_q);
+        tma_prefetch_map(&p.tm_k);
+        tma_prefetch_map(&p.tm_v);
+        tma_prefetch_map(&p.tm_o);
       }
       __syncwarp();
-      if (unit < 0) break;
-      // The next unit is claimed late in this one (kClaimLead ring items before its last
-      // load), so units go to the CTAs that are about to run out of work: claiming a
-      // whole unit ahead leaves a tail of up to one long causal unit between SMs.
-      bool claimed = false;
-      const int claim_at = max(0, 2 * u.nmax - C::kClaimLead);
-      auto claim_next = [&]() {
-        if (!claimed && !warp_flag(abort_flag)) {
-          mbar_arrive_expect_tx_w(BAR(C::kBarClc), 16);
-          clc_try_cancel_w(clc_resp, BAR(C::kBarClc));
-          claimed = true;
+      int unit = blockIdx.x;  // the first unit is this CTA's own
+      int nq[2] = {0, 0};     // Q loads issued per tile
+      bool q_pending[2] = {false, false};
+      int g = 0;              // ring items issued
+      int nclaim = 0;
+      for (int k = 0;; ++k) {
+        PrefillUnit u;
+        if (unit >= 0) {
+          u = prefill_unit(p, unit);
+        } else {
+          u.id = -1;
+          u.b = u.h = u.row0[0] = u.row0[1] = u.nkv[0] = u.nkv[1] = 0;
+          u.nmax = -1;
         }
-      };
-      for (int t = 0; t < 2; ++t) {
-        if (u.nkv[t] == 0) continue;
-        if (nq[t] > 0) mbar_wait(BAR(C::kBarQEmpty + t), (nq[t] - 1) & 1, wctx);
+        if (k >= 2) mbar_wait_inline(BAR(C::kBarUnitEmpty + (k & 1)), ((k >> 1) - 1) & 1, wctx);
         __syncwarp();
-        if (!(p.inject == 1 && t == 0) && !warp_flag(abort_flag)) {
-          mbar_arrive_expect_tx_w(BAR(C::kBarQFull + t), C::kTileBytes);
-          for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_4d_w(sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
-                          BAR(C::kBarQFull + t), bx * 64, u.h, u.row0[t], u.b);
-          q_pending[t] = true;
+        if (lane == 0) {
+          volatile int* us = unit_slot + (k & 1) * kUnitInts;
+          us[0] = u.id;
+          us[1] = u.b;
+          us[2] = u.h;
+          us[3] = u.row0[0];
+          us[4] = u.row0[1];
+          us[5] = u.nkv[0];
+          us[6] = u.nkv[1];
+          us[7] = u.nmax;
+          mbar_arrive(BAR(C::kBarUnitFull + (k & 1)));
         }
-        ++nq[t];
-      }
-      for (int i = 0; i < 2 * u.nmax; ++i, ++g) {
-        if (i == claim_at) claim_next();
-        const int stage = g % C::kStages;
-        const int round = g / C::kStages;
-        if (round > 0) mbar_wait(BAR(C::kBarKVEmpty + stage), (round - 1) & 1, wctx);
         __syncwarp();
-        if (warp_flag(abort_flag)) continue;
-        mbar_arrive_expect_tx_w(BAR(C::kBarKVFull + stage), C::kTileBytes);
-        const CUtensorMap* map = (i & 1) ? &p.tm_v : &p.tm_k;
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_4d_w(sbase + C::kOffKV + stage * C::kTileBytes + bx * C::kBoxBytes, map,
-                        BAR(C::kBarKVFull + stage), bx * 64, u.h, (i >> 1) * 128, u.b);
-      }
-      claim_next();  // units without K/V tiles
-      int next = -1;
-      if (claimed) {
-        if (mbar_wait(BAR(C::kBarClc), nclaim & 1, wctx)) next = clc_response_ctaid_x(clc_resp);
-        else mbar_wait_drain(BAR(C::kBarClc), nclaim & 1, p.timeout_ns);
-        ++nclaim;
-      }
-      __syncwarp();
-      unit = __shfl_sync(0xffffffffu, next, 0);
-    }
-    if (warp_flag(abort_flag)) {
-      // Let every copy this warp started land before the CTA can exit.
-      for (int t = 0; t < 2; ++t)
-        if (q_pending[t]) mbar_wait_drain(BAR(C::kBarQFull + t), (nq[t] - 1) & 1, p.timeout_ns);
-      const int first = g > C::kStages ? g - C::kStages : 0;
-      for (int i = first; i < g; ++i)
-        mbar_wait_drain(BAR(C::kBarKVFull + i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
-      __syncwarp();
-    }
-  } else if (warp == C::kMmaWarp) {
-    if constexpr (C::kDecoupled) {
-    // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
-    constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
-    // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
-    constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
-    const uint32_t colS[2] = {0u, 128u};
-    const uint32_t colO[2] = {256u, 256u + D};
-    const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
-    // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
-    auto issue_s = [&](int t, uint32_t sK) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-        mma_f16_ss_w(tmem + colS[t], make_sdesc_sw128(sQ[t] + off, 16, 1024),
-                     make_sdesc_sw128(sK + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-      }
-    };
-    // O_t += P_t V_j over 8 k-steps of 16 keys; P_t in its own TMEM columns.
-    auto issue_pv = [&](int t, uint32_t sV, bool accumulate_first) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t bdesc = make_sdesc_sw128(sV + kk * 2048, C::kBoxBytes, 1024);
-        const uint32_t acc = (accumulate_first || kk > 0) ? 1u : 0u;
-        mma_f16_ts_w(tmem + colO[t], tmem + C::kColP + 64 * t + kk * 8, bdesc, idesc_o, acc);
-      }
-    };
-    auto stage_addr = [&](int item) -> uint32_t {
-      return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;
-    };
-    int nq[2] = {0, 0};   // units seen per tile (q_full / q_empty phases)
-    int nsf[2] = {0, 0};  // S tiles released by the softmax (s_free phases)
-    int npf[2] = {0, 0};  // P tiles written by the softmax (p_full phases)
-    int g = 0;            // ring items consumed
-    for (int k = 0;; ++k) {
-      const PrefillUnit u = next_unit(k);
-      if (u.nmax < 0) break;
-      if (u.nmax == 0) continue;
-      for (int t = 0; t < 2; ++t)
-        if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
-      // prologue: S_t(0) for both tiles from K_0
-      mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
-      __syncwarp();
-      tc_fence_after_sync();
-      if (!warp_flag(abort_flag)) {
-        for (int t = 0; t < 2; ++t)
-          if (u.nkv[t] > 0) {
-            issue_s(t, stage_addr(g));
-            tc_commit_w(BAR(C::kBarSFull + t));
-            if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
+        if (unit < 0) break;
+        // The next unit is claimed late in this one (kClaimLead ring items before its last
+        // load), so units go to the CTAs that are about to run out of work: claiming a
+        // whole unit ahead leaves a tail of up to one long causal unit between SMs.
+        bool claimed = false;
+        const int claim_at = max(0, 2 * u.nmax - C::kClaimLead);
+        auto claim_next = [&]() {
+          if (!claimed && !warp_flag(abort_flag)) {
+            mbar_arrive_expect_tx_w(BAR(C::kBarClc), 16);
+            clc_try_cancel_w(clc_resp, BAR(C::kBarClc));
+            claimed = true;
           }
-        tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
-      }
-      for (int j = 0; j < u.nmax; ++j) {
-        // next score tiles: S_t(j+1) as soon as the softmax has read S_t(j) out of TMEM
-        const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
-        bool k_ready = false;
+        };
         for (int t = 0; t < 2; ++t) {
-          if (j >= u.nkv[t]) continue;
-          mbar_wait(BAR(C::kBarSFree + t), nsf[t] & 1, wctx);
-          ++nsf[t];
+          if (u.nkv[t] == 0) continue;
+          if (nq[t] > 0) mbar_wait_inline(BAR(C::kBarQEmpty + t), (nq[t] - 1) & 1, wctx);
           __syncwarp();
-          if (j + 1 < u.nkv[t]) {
-            if (!k_ready) {
-              mbar_wait(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
-              __syncwarp();
-              k_ready = true;
+          if (!(p.inject == 1 && t == 0) && !warp_flag(abort_flag)) {
+            mbar_arrive_expect_tx_w(BAR(C::kBarQFull + t), C::kTileBytes);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_4d_w(sbase + C::kOffQ + t * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q,
+                            BAR(C::kBarQFull + t), bx * 64, u.h, u.row0[t], u.b);
+            q_pending[t] = true;
+          }
+          ++nq[t];
+        }
+        for (int i = 0; i < 2 * u.nmax; ++i, ++g) {
+          if (i == claim_at) claim_next();
+          const int stage = g % C::kStages;
+          const int round = g / C::kStages;
+          if (round > 0) mbar_wait_inline(BAR(C::kBarKVEmpty + stage), (round - 1) & 1, wctx);
+          __syncwarp();
+          if (warp_flag(abort_flag)) continue;
+          mbar_arrive_expect_tx_w(BAR(C::kBarKVFull + stage), C::kTileBytes);
+          const CUtensorMap* map = (i & 1) ? &p.tm_v : &p.tm_k;
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_4d_w(sbase + C::kOffKV + stage * C::kTileBytes + bx * C::kBoxBytes, map,
+                          BAR(C::kBarKVFull + stage), bx * 64, u.h, (i >> 1) * 128, u.b);
+        }
+        claim_next();  // units without K/V tiles
+        int next = -1;
+        if (claimed) {
+          if (mbar_wait_inline(BAR(C::kBarClc), nclaim & 1, wctx)) next = clc_response_ctaid_x(clc_resp);
+          else mbar_wait_drain_inline(BAR(C::kBarClc), nclaim & 1, p.timeout_ns);
+          ++nclaim;
+        }
+        __syncwarp();
+        unit = __shfl_sync(0xffffffffu, next, 0);
+      }
+      if (warp_flag(abort_flag)) {
+        // Let every copy this warp started land before the CTA can exit.
+        for (int t = 0; t < 2; ++t)
+          if (q_pending[t]) mbar_wait_drain_inline(BAR(C::kBarQFull + t), (nq[t] - 1) & 1, p.timeout_ns);
+        const int first = g > C::kStages ? g - C::kStages : 0;
+        for (int i = first; i < g; ++i)
+          mbar_wait_drain_inline(BAR(C::kBarKVFull + i % C::kStages), (i / C::kStages) & 1, p.timeout_ns);
+        __syncwarp();
+      }
+    } else if (warp == C::kMmaWarp) {
+      if constexpr (C::kDecoupled) {
+      // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
+      constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
+      // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
+      constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
+      const uint32_t colS[2] = {0u, 128u};
+      const uint32_t colO[2] = {256u, 256u + D};
+      const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+      // S_t = Q_t K_j^T: the D / 16 = 4 k-steps of 16 elements (32 bytes apart inside the
+      // 128-byte swizzle rows of one box), issued in one batch.
+      static_assert(D == 64, "the decoupled pipeline runs at head_dim 64");
+      auto issue_s = [&](int t, uint32_t sK) {
+        mma_f16_ss_k64_w(tmem + colS[t], make_sdesc_sw128(sQ[t], 16, 1024), make_sdesc_sw128(sK, 16, 1024),
+                         idesc_s, 0u);
+      };
+      // O_t += P_t V_j over 8 k-steps of 16 keys (P_t in its own TMEM columns), issued in two
+      // batches of four.
+      auto issue_pv = [&](int t, uint32_t sV, bool accumulate_first) {
+        mma_f16_ts_k64_w<2048>(tmem + colO[t], tmem + C::kColP + 64 * t,
+                               make_sdesc_sw128(sV, C::kBoxBytes, 1024), idesc_o, accumulate_first ? 1u : 0u);
+        mma_f16_ts_k64_w<2048>(tmem + colO[t], tmem + C::kColP + 64 * t + 32,
+                               make_sdesc_sw128(sV + 4 * 2048, C::kBoxBytes, 1024), idesc_o, 1u);
+      };
+      auto stage_addr = [&](int item) -> uint32_t {
+        return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;
+      };
+      int nq[2] = {0, 0};   // units seen per tile (q_full / q_empty phases)
+      int nsf[2] = {0, 0};  // S tiles released by the softmax (s_free phases)
+      int npf[2] = {0, 0};  // P tiles written by the softmax (p_full phases)
+      int g = 0;            // ring items consumed
+      for (int k = 0;; ++k) {
+        const PrefillUnit u = next_unit(k);
+        if (u.nmax < 0) break;
+        if (u.nmax == 0) continue;
+        for (int t = 0; t < 2; ++t)
+          if (u.nkv[t] > 0) mbar_wait_inline(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
+        // prologue: S_t(0) for both tiles from K_0
+        mbar_wait_inline(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
+        __syncwarp();
+        tc_fence_after_sync();
+        if (!warp_flag(abort_flag)) {
+          for (int t = 0; t < 2; ++t)
+            if (u.nkv[t] > 0) {
+              issue_s(t, stage_addr(g));
+              tc_commit_w(BAR(C::kBarSFull + t));
+              if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
             }
+          tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
+        }
+        for (int j = 0; j < u.nmax; ++j) {
+          // next score tiles: S_t(j+1) as soon as the softmax has read S_t(j) out of TMEM
+          const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
+          bool k_ready = false;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= u.nkv[t]) continue;
+            mbar_wait_inline(BAR(C::kBarSFree + t), nsf[t] & 1, wctx);
+            ++nsf[t];
+            __syncwarp();
+            if (j + 1 < u.nkv[t]) {
+              if (!k_ready) {
+                mbar_wait_inline(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
+                __syncwarp();
+                k_ready = true;
+              }
+              tc_fence_after_sync();
+              if (warp_flag(abort_flag)) continue;
+              issue_s(t, stage_addr(ik));
+              tc_commit_w(BAR(C::kBarSFull + t));
+              if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
+            }
+          }
+          if (k_ready && !warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
+          // O_t += P_t(j) V_j once the softmax has written P_t(j)
+          const int iv = g + 2 * j + 1;  // ring item of V_j
+          mbar_wait_inline(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + iv % C::kStages), (iv / C::kStages) & 1,
+                    wctx);
+          __syncwarp();
+          for (int t = 0; t < 2; ++t) {
+            if (j >= u.nkv[t]) continue;
+            mbar_wait_inline(BAR(C::kBarPFull + t), npf[t] & 1, wctx);
+            ++npf[t];
+            __syncwarp();
             tc_fence_after_sync();
             if (warp_flag(abort_flag)) continue;
-            issue_s(t, stage_addr(ik));
-            tc_commit_w(BAR(C::kBarSFull + t));
-            if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
-          }
-        }
-        if (k_ready && !warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
-        // O_t += P_t(j) V_j once the softmax has written P_t(j)
-        const int iv = g + 2 * j + 1;  // ring item of V_j
-        mbar_wait(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + iv % C::kStages), (iv / C::kStages) & 1,
-                  wctx);
-        __syncwarp();
-        for (int t = 0; t < 2; ++t) {
-          if (j >= u.nkv[t]) continue;
-          mbar_wait(BAR(C::kBarPFull + t), npf[t] & 1, wctx);
-          ++npf[t];
-          __syncwarp();
-          tc_fence_after_sync();
-          if (warp_flag(abort_flag)) continue;
-          issue_pv(t, stage_addr(iv), j > 0);
-          tc_commit_w(BAR(C::kBarPVDone + t));
-        }
-        if (!warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + iv % C::kStages));
-      }
-      g += 2 * u.nmax;
-      for (int t = 0; t < 2; ++t)
-        if (u.nkv[t] > 0) ++nq[t];
-    }
-    // every MMA (and every commit arrive) has landed before TMEM is released
-    tc_commit_w(BAR(C::kBarMmaDone));
-    mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
-    __syncwarp();
-    } else {
-    // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
-    constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
-    // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
-    constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
-    const uint32_t colS[2] = {0u, 128u};
-    const uint32_t colO[2] = {256u, 256u + D};
-    const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
-    // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
-    // S_t = Q_t K_j^T: 8 k-steps of 16 elements, issued in one batch.
-    auto issue_s = [&](int t, uint32_t sK) {
-      mma_f16_ss_k128_w<C::kBoxBytes>(tmem + colS[t], make_sdesc_sw128(sQ[t], 16, 1024),
-                                      make_sdesc_sw128(sK, 16, 1024), idesc_s, 0u);
-    };
-    // k-steps kk0 .. kk0+3 of O_t += P_t V_j (keys 16*kk0 .. 16*kk0+63; P_t is in TMEM
-    // columns [64,128) of S_t), issued in one batch; the first k-step of the unit starts
-    // the accumulator.
-    auto issue_pv4 = [&](int t, uint32_t sV, int kk0, bool accumulate_first) {
-      mma_f16_ts_k64_w<2048>(tmem + colO[t], tmem + colS[t] + 64 + kk0 * 8,
-                             make_sdesc_sw128(sV + kk0 * 2048, C::kBoxBytes, 1024), idesc_o,
-                             accumulate_first ? 1u : 0u);
-    };
-    auto stage_addr = [&](int item) -> uint32_t {
-      return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;
-    };
-    int nq[2] = {0, 0};  // units seen per tile (q_full / q_empty phases)
-    int np[2] = {0, 0};  // P tiles consumed per tile (p_ready phases)
-    int g = 0;           // ring items consumed
-    for (int k = 0;; ++k) {
-      const PrefillUnit u = next_unit(k);
-      if (u.nmax < 0) break;
-      if (u.nmax == 0) continue;
-      for (int t = 0; t < 2; ++t)
-        if (u.nkv[t] > 0) mbar_wait(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
-      // prologue: S_t(0) for both tiles from K_0
-      mbar_wait(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
-      __syncwarp();
-      tc_fence_after_sync();
-      if (!warp_flag(abort_flag)) {
-        for (int t = 0; t < 2; ++t)
-          if (u.nkv[t] > 0) {
-            issue_s(t, stage_addr(g));
-            tc_commit_w(BAR(C::kBarSFull + t));
-            if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
-          }
-        tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
-      }
-      for (int j = 0; j < u.nmax; ++j) {
-        const int iv = g + 2 * j + 1;  // ring item of V_j
-        mbar_wait(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + iv % C::kStages), (iv / C::kStages) & 1,
-                  wctx);
-        __syncwarp();
-        const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
-        bool k_ready = false;
-        for (int t = 0; t < 2; ++t) {
-          if (j >= u.nkv[t]) continue;
-          // keys 64..127 as soon as that half of P_t(j) is written, then keys 0..63
-          mbar_wait(BAR(C::kBarPHalf + t), np[t] & 1, wctx);
-          __syncwarp();
-          tc_fence_after_sync();
-          if (!warp_flag(abort_flag)) issue_pv4(t, stage_addr(iv), 4, j > 0);
-          mbar_wait(BAR(C::kBarPFull + t), np[t] & 1, wctx);
-          ++np[t];
-          __syncwarp();
-          tc_fence_after_sync();
-          if (warp_flag(abort_flag)) continue;
-          issue_pv4(t, stage_addr(iv), 0, true);
-          if (j + 1 < u.nkv[t]) {
-            if (!k_ready) {
-              mbar_wait(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
-              __syncwarp();
-              k_ready = true;
-            }
-            if (warp_flag(abort_flag)) continue;
-            issue_s(t, stage_addr(ik));
-            tc_commit_w(BAR(C::kBarSFull + t));
-            if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
-          } else {
+            issue_pv(t, stage_addr(iv), j > 0);
             tc_commit_w(BAR(C::kBarPVDone + t));
           }
+          if (!warp_flag(abort_flag)) tc_commit_w(BAR(C::kBarKVEmpty + iv % C::kStages));
         }
+        g += 2 * u.nmax;
+        for (int t = 0; t < 2; ++t)
+          if (u.nkv[t] > 0) ++nq[t];
+      }
+      // every MMA (and every commit arrive) has landed before TMEM is released
+      tc_commit_w(BAR(C::kBarMmaDone));
+      mbar_wait_drain_inline(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+      __syncwarp();
+      } else {
+      // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
+      constexpr uint32_t idesc_s = make_idesc_f16(128, 128, BF16, false);  // Q K^T, both K-major
+      // P V always runs in fp16 (bf16 V tiles are converted in shared memory first); V is MN-major
+      constexpr uint32_t idesc_o = make_idesc_f16(128, D, false, true);
+      const uint32_t colS[2] = {0u, 128u};
+      const uint32_t colO[2] = {256u, 256u + D};
+      const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+      // S_t = Q_t K_j^T over D/16 k-steps of 16 elements (32 bytes inside a 128-byte swizzle row).
+      // S_t = Q_t K_j^T: 8 k-steps of 16 elements, issued in one batch.
+      auto issue_s = [&](int t, uint32_t sK) {
+        mma_f16_ss_k128_w<C::kBoxBytes>(tmem + colS[t], make_sdesc_sw128(sQ[t], 16, 1024),
+                                        make_sdesc_sw128(sK, 16, 1024), idesc_s, 0u);
+      };
+      // k-steps kk0 .. kk0+3 of O_t += P_t V_j (keys 16*kk0 .. 16*kk0+63; P_t is in TMEM
+      // columns [64,128) of S_t), issued in one batch; the first k-step of the unit starts
+      // the accumulator.
+      auto issue_pv4 = [&](int t, uint32_t sV, int kk0, bool accumulate_first) {
+        mma_f16_ts_k64_w<2048>(tmem + colO[t], tmem + colS[t] + 64 + kk0 * 8,
+                               make_sdesc_sw128(sV + kk0 * 2048, C::kBoxBytes, 1024), idesc_o,
+                               accumulate_first ? 1u : 0u);
+      };
+      auto stage_addr = [&](int item) -> uint32_t {
+        return sbase + C::kOffKV + (item % C::kStages) * C::kTileBytes;
+      };
+      int nq[2] = {0, 0};  // units seen per tile (q_full / q_empty phases)
+      int np[2] = {0, 0};  // P tiles consumed per tile (p_ready phases)
+      int g = 0;           // ring items consumed
+      for (int k = 0;; ++k) {
+        const PrefillUnit u = next_unit(k);
+        if (u.nmax < 0) break;
+        if (u.nmax == 0) continue;
+        for (int t = 0; t < 2; ++t)
+          if (u.nkv[t] > 0) mbar_wait_inline(BAR(C::kBarQFull + t), nq[t] & 1, wctx);
+        // prologue: S_t(0) for both tiles from K_0
+        mbar_wait_inline(BAR(C::kBarKVFull + g % C::kStages), (g / C::kStages) & 1, wctx);
+        __syncwarp();
+        tc_fence_after_sync();
         if (!warp_flag(abort_flag)) {
-          tc_commit_w(BAR(C::kBarKVEmpty + iv % C::kStages));
-          if (k_ready) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
-        }
-      }
-      g += 2 * u.nmax;
-      for (int t = 0; t < 2; ++t)
-        if (u.nkv[t] > 0) ++nq[t];
-    }
-    // every MMA (and every commit arrive) has landed before TMEM is released
-    tc_commit_w(BAR(C::kBarMmaDone));
-    mbar_wait_drain(BAR(C::kBarMmaDone), 0, p.timeout_ns);
-    __syncwarp();
-    }
-  } else if (warp >= C::kConvWarp0) {
-    // ======================= bf16 -> fp16 conversion of V tiles (bf16 inputs) ======
-    // Walks every ring item in order: waits for it to land, converts it if it is a V
-    // tile, then arrives on its v_conv barrier (the MMA issuer waits on that for V
-    // tiles) and on its empty barrier (the producer refills a stage only after both the
-    // tensor core and the converters are done with it).
-    // A V element of magnitude 65536 or more (or inf / NaN) has no fp16 value: the
-    // largest magnitude bit pattern met is tracked per thread and, if any such element
-    // was converted, the call's status word records kStatusRange.
-    const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
-    uint32_t vmag = 0;  // per-halfword max of |bf16 bits| over every V element converted
-    int g = 0;
-    for (int k = 0;; ++k) {
-      const PrefillUnit u = next_unit(k);
-      if (u.nmax < 0) break;
-      if constexpr (BF16) {
-        for (int i = 0; i < 2 * u.nmax; ++i) {
-          const int item = g + i;
-          const int st = item % C::kStages;
-          mbar_wait(BAR(C::kBarKVFull + st), (item / C::kStages) & 1, wctx);
-          __syncwarp();
-          if (i & 1) {
-            uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + st * C::kTileBytes);
-#pragma unroll 4
-            for (int c = ct; c < C::kTileBytes / 16; c += 64) {
-              uint4 w = tile[c];
-              vmag = __vmaxu2(vmag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
-                                             __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
-              w.x = bf16x2_to_f16x2_sat(w.x);
-              w.y = bf16x2_to_f16x2_sat(w.y);
-              w.z = bf16x2_to_f16x2_sat(w.z);
-              w.w = bf16x2_to_f16x2_sat(w.w);
-              tile[c] = w;
+          for (int t = 0; t < 2; ++t)
+            if (u.nkv[t] > 0) {
+              issue_s(t, stage_addr(g));
+              tc_commit_w(BAR(C::kBarSFull + t));
+              if (u.nkv[t] == 1) tc_commit_w(BAR(C::kBarQEmpty + t));
             }
-            fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-          }
+          tc_commit_w(BAR(C::kBarKVEmpty + g % C::kStages));
+        }
+        for (int j = 0; j < u.nmax; ++j) {
+          const int iv = g + 2 * j + 1;  // ring item of V_j
+          mbar_wait_inline(BAR((BF16 ? C::kBarVConv : C::kBarKVFull) + iv % C::kStages), (iv / C::kStages) & 1,
+                    wctx);
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(BAR(C::kBarVConv + st));
-            mbar_arrive(BAR(C::kBarKVEmpty + st));
+          const int ik = g + 2 * j + 2;  // ring item of K_{j+1}
+          bool k_ready = false;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= u.nkv[t]) continue;
+            // keys 64..127 as soon as that half of P_t(j) is written, then keys 0..63
+            mbar_wait_inline(BAR(C::kBarPHalf + t), np[t] & 1, wctx);
+            __syncwarp();
+            tc_fence_after_sync();
+            if (!warp_flag(abort_flag)) issue_pv4(t, stage_addr(iv), 4, j > 0);
+            mbar_wait_inline(BAR(C::kBarPFull + t), np[t] & 1, wctx);
+            ++np[t];
+            __syncwarp();
+            tc_fence_after_sync();
+            if (warp_flag(abort_flag)) continue;
+            issue_pv4(t, stage_addr(iv), 0, true);
+            if (j + 1 < u.nkv[t]) {
+              if (!k_ready) {
+                mbar_wait_inline(BAR(C::kBarKVFull + ik % C::kStages), (ik / C::kStages) & 1, wctx);
+                __syncwarp();
+                k_ready = true;
+              }
+              if (warp_flag(abort_flag)) continue;
+              issue_s(t, stage_addr(ik));
+              tc_commit_w(BAR(C::kBarSFull + t));
+              if (j + 2 == u.nkv[t]) tc_commit_w(BAR(C::kBarQEmpty + t));
+            } else {
+              tc_commit_w(BAR(C::kBarPVDone + t));
+            }
+          }
+          if (!warp_flag(abort_flag)) {
+            tc_commit_w(BAR(C::kBarKVEmpty + iv % C::kStages));
+            if (k_ready) tc_commit_w(BAR(C::kBarKVEmpty + ik % C::kStages));
           }
         }
+        g += 2 * u.nmax;
+        for (int t = 0; t < 2; ++t)
+          if (u.nkv[t] > 0) ++nq[t];
       }
-      g += 2 * u.nmax;
+      // every MMA (and every commit arrive) has landed before TMEM is released
+      tc_commit_w(BAR(C::kBarMmaDone));
+      mbar_wait_drain_inline(BAR(C::kBarMmaDone), 0, p.timeout_ns);
+      __syncwarp();
+      }
+    } else if (warp >= C::kConvWarp0) {
+      // ======================= bf16 -> fp16 conversion of V tiles (bf16 inputs) ======
+      // Walks every ring item in order: waits for it to land, converts it if it is a V
+      // tile, then arrives on its v_conv barrier (the MMA issuer waits on that for V
+      // tiles) and on its empty barrier (the producer refills a stage only after both the
+      // tensor core and the converters are done with it).
+      // A V element of magnitude 65536 or more (or inf / NaN) has no fp16 value: the
+      // largest magnitude bit pattern met is tracked per thread and, if any such element
+      // was converted, the call's status word records kStatusRange.
+      const int ct = threadIdx.x - C::kConvWarp0 * 32;  // 0..63
+      uint32_t vmag = 0;  // per-halfword max of |bf16 bits| over every V element converted
+      int g = 0;
+      for (int k = 0;; ++k) {
+        const PrefillUnit u = next_unit(k);
+        if (u.nmax < 0) break;
+        if constexpr (BF16) {
+          for (int i = 0; i < 2 * u.nmax; ++i) {
+            const int item = g + i;
+            const int st = item % C::kStages;
+            mbar_wait_inline(BAR(C::kBarKVFull + st), (item / C::kStages) & 1, wctx);
+            __syncwarp();
+            if (i & 1) {
+              uint4* tile = reinterpret_cast<uint4*>(smem + C::kOffKV + st * C::kTileBytes);
+#pragma unroll 4
+              for (int c = ct; c < C::kTileBytes / 16; c += 64) {
+                uint4 w = tile[c];
+                vmag = __vmaxu2(vmag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                               __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+                w.x = bf16x2_to_f16x2_sat(w.x);
+                w.y = bf16x2_to_f16x2_sat(w.y);
+                w.z = bf16x2_to_f16x2_sat(w.z);
+                w.w = bf16x2_to_f16x2_sat(w.w);
+                tile[c] = w;
+              }
+              fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+            }
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(BAR(C::kBarVConv + st));
+              mbar_arrive(BAR(C::kBarKVEmpty + st));
+            }
+          }
+        }
+        g += 2 * u.nmax;
+      }
+      if (max(vmag & 0xFFFFu, vmag >> 16) >= kBf16NoF16) atomicCAS(p.status, 0, kStatusRange);
     }
-    if (max(vmag & 0xFFFFu, vmag >> 16) >= kBf16NoF16) atomicCAS(p.status, 0, kStatusRange);
+    // back to the launch's registers (waits until the softmax warps have given theirs back)
+    __syncwarp();
+    if constexpr (C::kDecoupled) warpgroup_reg_alloc<C::kLaunchRegs>();
   } else {
+    // warpgroups 0 and 1: softmax
+    if constexpr (C::kDecoupled) warpgroup_reg_alloc<C::kRegsSoftmax>();
     if constexpr (C::kDecoupled) {
     // ======================= softmax warpgroups (warps 0-3: tile 0, 4-7: tile 1) ======
     const int t = warp >> 2;
@@ -827,7 +845,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazy: may lag the true max by <= 8)
       float l_run = 0.f;        // running sum of 2^(cs*s - m_run)
       for (int j = 0; j < nkv; ++j) {
-        mbar_wait(BAR(C::kBarSFull + t), ns & 1, wctx);
+        mbar_wait_inline(BAR(C::kBarSFull + t), ns & 1, wctx);
         ++ns;
         __syncwarp();  // lanes may leave the bounded wait on different polls
         tc_fence_after_sync();
@@ -867,7 +885,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
 
         if (j > 0) {
           // P_t(j-1) V must be done: its P buffer is about to be overwritten and O_t may be rescaled
-          mbar_wait(BAR(C::kBarPVDone + t), (npv + j - 1) & 1, wctx);
+          mbar_wait_inline(BAR(C::kBarPVDone + t), (npv + j - 1) & 1, wctx);
           __syncwarp();
           tc_fence_after_sync();
           if (__any_sync(0xffffffffu, rescale)) {  // lazy rescale of O (rare after the first tiles)
@@ -893,7 +911,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       }
 
       // ---- epilogue: O / l -> 16-bit -> swizzled staging (this tile's buffer) -> TMA store
-      mbar_wait(BAR(C::kBarPVDone + t), (npv + nkv - 1) & 1, wctx);
+      mbar_wait_inline(BAR(C::kBarPVDone + t), (npv + nkv - 1) & 1, wctx);
       npv += nkv;
       __syncwarp();
       tc_fence_after_sync();
@@ -906,7 +924,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
         bulk_wait_group_read0();
         mbar_arrive(BAR(C::kBarOFree + t));
       }
-      mbar_wait(BAR(C::kBarOFree + t), nout & 1, wctx);
+      mbar_wait_inline(BAR(C::kBarOFree + t), nout & 1, wctx);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) reg_order_after_wait(o[c]);
@@ -928,7 +946,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarOReady + t));
       if (quarter == 0) {
-        mbar_wait(BAR(C::kBarOReady + t), nout & 1, wctx);
+        mbar_wait_inline(BAR(C::kBarOReady + t), nout & 1, wctx);
         if (r == 0 && !*abort_flag) {
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_store_4d(&p.tm_o, sbase + C::kOffO + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64,
@@ -961,8 +979,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     // unit 0, tile 1 of unit 0, tile 0 of unit 1, ...: a turn starts when the previous
     // turn's TMA store has finished reading the buffer (an inactive tile passes its turn).
     auto ostage_acquire = [&](int k) {
-      if (t == 0 && k > 0) mbar_wait(BAR(C::kBarOStage + 1), (k - 1) & 1, wctx);
-      if (t == 1) mbar_wait(BAR(C::kBarOStage + 0), k & 1, wctx);
+      if (t == 0 && k > 0) mbar_wait_inline(BAR(C::kBarOStage + 1), (k - 1) & 1, wctx);
+      if (t == 1) mbar_wait_inline(BAR(C::kBarOStage + 0), k & 1, wctx);
       __syncwarp();
     };
     int ns = 0;  // S tiles consumed (s_full phases)
@@ -998,7 +1016,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       float m_run = -INFINITY;  // running max of scale*log2(e)*s (lazy: may lag the true max by <= 8)
       float l_run = 0.f;        // running sum of 2^(cs*s - m_run)
       for (int j = 0; j < nkv; ++j) {
-        mbar_wait(BAR(C::kBarSFull + t), ns & 1, wctx);
+        mbar_wait_inline(BAR(C::kBarSFull + t), ns & 1, wctx);
         ++ns;
         __syncwarp();  // lanes may leave the bounded wait on different polls
         tc_fence_after_sync();
@@ -1124,7 +1142,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       }
 
       // ---- epilogue: O / l -> 16-bit -> swizzled staging buffer -> TMA store
-      mbar_wait(BAR(C::kBarPVDone + t), no & 1, wctx);
+      mbar_wait_inline(BAR(C::kBarPVDone + t), no & 1, wctx);
       ++no;
       __syncwarp();
       tc_fence_after_sync();
@@ -1156,7 +1174,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarOReady + t));
       if (quarter == 0) {
-        mbar_wait(BAR(C::kBarOReady + t), (no - 1) & 1, wctx);
+        mbar_wait_inline(BAR(C::kBarOReady + t), (no - 1) & 1, wctx);
         if (r == 0 && !*abort_flag) {
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_store_4d(&p.tm_o, sbase + C::kOffO + bx * C::kBoxBytes, bx * 64, u.h, row0, u.b);
@@ -1171,6 +1189,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       }
     }
     }
+    __syncwarp();
+    if constexpr (C::kDecoupled) warpgroup_reg_dealloc<C::kLaunchRegs>();
   }
 
   // ---- teardown: every role is done with TMEM

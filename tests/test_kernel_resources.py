@@ -23,8 +23,11 @@ THREADS = {"attn_prefill_kernel": 384, "attn_decode_partial_kernel": 160,
            "attn_topk_kernel": 512, "attn_bwd_kernel": 320, "attn_bwd_pre_kernel": 128,
            "attn_bwd_dq_kernel": 256, "attn_relpos_kernel": 320}
 # bytes of spill stores / loads per prefill instantiation (head_dim, bf16) at this version
-PREFILL_SPILL_CEILING = {(64, False): (112, 168), (64, True): (152, 300),
-                         (128, False): (8, 8), (128, True): (16, 16)}
+# (d = 64: the softmax warps' scores stay in registers; what is left is outside the step loop)
+PREFILL_SPILL_CEILING = {(64, False): (8, 44), (64, True): (8, 48),
+                         (128, False): (8, 8), (128, True): (8, 8)}
+# d = 64 re-balances registers between warpgroups (setmaxnreg) from exactly this count at launch
+PREFILL_LAUNCH_REGS = 168
 
 
 @pytest.fixture(scope="module")
@@ -96,6 +99,14 @@ def test_non_prefill_kernels_do_not_spill(ptxas_report):
     for name, info in ptxas_report.items():
         if kernel_kind(name) != "attn_prefill_kernel":
             assert info["spill_stores"] == 0 and info["spill_loads"] == 0, (name, info)
+
+
+def test_prefill_launch_registers_match_the_split(ptxas_report):
+    """The d = 64 kernel's warpgroups trade registers (2 x 208 + 88 = 3 x 168 per sub-
+    partition); that only adds up if ptxas gives the kernel exactly 168 at launch."""
+    for name, info in ptxas_report.items():
+        if kernel_kind(name) == "attn_prefill_kernel" and template_args(name)[0] == 64:
+            assert info["registers"] == PREFILL_LAUNCH_REGS, (name, info)
 
 
 def test_prefill_spills_do_not_grow(ptxas_report):
