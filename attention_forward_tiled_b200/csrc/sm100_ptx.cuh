@@ -227,33 +227,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   return mbar_wait_slow(bar, parity, w.abort_flag, w.status, w.timeout_ns);
 }
 
-// The same waits with the polling loop inline, for kernels that re-balance registers
-// between warpgroups (setmaxnreg): ptxas allocates such a kernel only when it makes no
-// calls, and a call would also make the caller save its live registers around it.
-__device__ __forceinline__ bool mbar_wait_inline(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long limit = wait_limit_cycles(w.timeout_ns);
-  const long long c0 = clock64();
-  for (uint32_t it = 0; it < (1u << 30); ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*w.abort_flag) return false;
-    if (clock64() - c0 > limit) break;
-  }
-  *w.abort_flag = 1;
-  atomicCAS(w.status, 0, kStatusTimeout);
-  return false;
-}
-
-__device__ __forceinline__ bool mbar_wait_drain_inline(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
-  const long long limit = wait_limit_cycles(timeout_ns);
-  const long long c0 = clock64();
-  for (uint32_t it = 0; it < (1u << 30); ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - c0 > limit) return false;
-  }
-  return false;
-}
-
 // Drain wait used on the way out after an abort: ignores the abort flag but is
 // still bounded by the time limit.
 __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -467,29 +440,6 @@ __device__ __forceinline__ void mma_f16_ss_k128_w(uint32_t d_tmem, uint64_t a_de
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kStep), "n"(2 * kStep),
       "n"(3 * kStep), "n"(kBox), "n"(kBox + kStep), "n"(kBox + 2 * kStep), "n"(kBox + 3 * kStep)
-      : "memory");
-}
-
-// Four k-steps of D = A B with A and B K-major in shared memory (128-byte swizzle, one
-// 64-element box along K): one elected lane issues all four, advancing both descriptors'
-// start address by 32 B per k-step.
-__device__ __forceinline__ void mma_f16_ss_k64_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                 uint32_t idesc, uint32_t accumulate) {
-  constexpr uint64_t kStep = 32 >> 4;
-  asm volatile(
-      "{\n\t.reg .pred p, e, t;\n\t.reg .b64 a, b;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "setp.eq.b32 t, 0, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
-      "add.s64 a, %1, %5;\n\tadd.s64 b, %2, %5;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
-      "add.s64 a, %1, %6;\n\tadd.s64 b, %2, %6;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
-      "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %7;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kStep), "n"(2 * kStep),
-      "n"(3 * kStep)
       : "memory");
 }
 
