@@ -501,9 +501,13 @@ __global__ void __launch_bounds__(kTopkThreads)
       const uint32_t u = i < P ? key_at(i) : 0u;
       const bool hit = u != 0u && (u & pmask) == prefix;
       const uint32_t bin = hit ? (u >> shift) & 255u : 256u;
-      // one atomic per distinct digit of the warp: most scores share the top digits
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (hit && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      if (shift == 24) {
+        // one atomic per distinct digit of the warp: most scores share the top digit
+        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        if (hit && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      } else if (hit) {
+        atomicAdd(&hist[bin], 1u);  // lower digits spread over the bins: few lanes share one
+      }
     }
     __syncthreads();
     if (tid < 32) {
