@@ -652,9 +652,27 @@ __global__ void __launch_bounds__(kTopkThreads)
     cidx[i] = 0x7fffffff;
   }
   __syncthreads();
-  // ---- bitonic sort: key descending, then position ascending.  Stages whose partner is
-  // 32 or more elements away go through shared memory; the rest of each merge (strides 16
-  // down to 1) runs in registers with warp shuffles, one element per thread and slot.
+  // ---- bitonic sort: key descending, then position ascending, on 64-bit values
+  // (key << 32) | ~position (one unsigned comparison orders both) that take the place of
+  // ckey / cidx.  Stages whose partner is 32 or more elements away go through shared
+  // memory; the rest of each merge (strides 16 down to 1) runs in registers with warp
+  // shuffles, one element per thread and slot.
+  uint64_t* cv = reinterpret_cast<uint64_t*>(ckey);  // [kp2], over ckey and cidx
+  {
+    uint64_t pk[kTopkMaxK / kTopkThreads];
+#pragma unroll
+    for (int r = 0; r < kTopkMaxK / kTopkThreads; ++r) {
+      const int i = tid + r * kTopkThreads;
+      if (i < kp2) pk[r] = ((uint64_t)ckey[i] << 32) | (uint64_t)(~(uint32_t)cidx[i]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kTopkMaxK / kTopkThreads; ++r) {
+      const int i = tid + r * kTopkThreads;
+      if (i < kp2) cv[i] = pk[r];
+    }
+    __syncthreads();
+  }
   for (int size = 2; size <= kp2; size <<= 1) {
     int stride = size >> 1;
     for (; stride >= 32; stride >>= 1) {
@@ -662,14 +680,10 @@ __global__ void __launch_bounds__(kTopkThreads)
         const int j = i ^ stride;
         if (j > i) {
           const bool desc = (i & size) == 0;  // this block sorts "first before second" order
-          const uint32_t ki = ckey[i], kj = ckey[j];
-          const int ii = cidx[i], ij = cidx[j];
-          const bool j_first = kj > ki || (kj == ki && ij < ii);
-          if (desc == j_first) {
-            ckey[i] = kj;
-            ckey[j] = ki;
-            cidx[i] = ij;
-            cidx[j] = ii;
+          const uint64_t vi = cv[i], vj = cv[j];
+          if (desc == (vj > vi)) {
+            cv[i] = vj;
+            cv[j] = vi;
           }
         }
       }
@@ -679,30 +693,21 @@ __global__ void __launch_bounds__(kTopkThreads)
     for (int i0 = 0; i0 < kp2; i0 += kTopkThreads) {  // whole warps: kp2 is a power of two
       const int i = i0 + tid;
       const bool active = i < kp2;
-      uint32_t kx = active ? ckey[i] : 0u;
-      int ix = active ? cidx[i] : 0;
+      uint64_t vx = active ? cv[i] : 0ull;
       const bool desc = (i & size) == 0;
       for (int st = stride; st >= 1; st >>= 1) {
-        const uint32_t ky = __shfl_xor_sync(0xffffffffu, kx, st);
-        const int iy = __shfl_xor_sync(0xffffffffu, ix, st);
-        const bool y_first = ky > kx || (ky == kx && iy < ix);
+        const uint64_t vy = __shfl_xor_sync(0xffffffffu, vx, st);
         const bool lower = (i & st) == 0;
         // the lower element of the pair keeps the one that comes first in this block's
         // order, the upper one the other
-        if (lower == (desc == y_first)) {
-          kx = ky;
-          ix = iy;
-        }
+        if (lower == (desc == (vy > vx))) vx = vy;
       }
-      if (active) {
-        ckey[i] = kx;
-        cidx[i] = ix;
-      }
+      if (active) cv[i] = vx;
     }
     __syncthreads();
   }
   int* out = idx + (long long)row * k;
-  for (int i = tid; i < k; i += kTopkThreads) out[i] = (i < nsel) ? cidx[i] : -1;
+  for (int i = tid; i < k; i += kTopkThreads) out[i] = (i < nsel) ? (int)(~(uint32_t)cv[i]) : -1;
 }
 
 }  // namespace attn_b200
