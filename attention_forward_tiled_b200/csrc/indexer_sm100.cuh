@@ -486,6 +486,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     return topk_key(__ldg(srow + i));
   };
   if constexpr (kCached) {
+#pragma unroll 8
     for (int i = tid; i < P; i += kTopkThreads) rowkeys[i] = topk_key(__ldg(srow + i));
   }
   // ---- radix select of the k-th largest key, 8 bits at a time from the top
