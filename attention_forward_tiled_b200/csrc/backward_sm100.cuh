@@ -213,10 +213,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!warp_flag(abort_flag)) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // 16 queries per k-step: 8 packed TMEM columns
+          // queries 32 h .. 32 h + 31 are packed at columns 32 h .. 32 h + 15
+          const uint32_t pcol = (kk >> 1) * 32 + (kk & 1) * 8;
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          mma_f16_ts_w(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+          mma_f16_ts_w(tmem + C::kColDV, tmem + C::kColS + pcol,
                        make_sdesc_sw128(sDO + kk * 2048, C::kQBox, 1024), idesc_kv, acc);
-          mma_f16_ts_w(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+          mma_f16_ts_w(tmem + C::kColDK, tmem + C::kColDP + pcol,
                        make_sdesc_sw128(sQ + kk * 2048, C::kQBox, 1024), idesc_kv, acc);
         }
       }
@@ -315,9 +317,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           dk2[(c8 + e) >> 1] = pack2<BF16>(dv8[e], dv8[e + 1]);
         }
       }
-      // P^T and dS^T (packed pairs) into the consumed S^T / dP^T columns of this warp's queries
-      tmem_st16(tmem + lane_base + C::kColS + hf * 16, pk);
-      tmem_st16(tmem + lane_base + C::kColDP + hf * 16, dk2);
+      // P^T and dS^T (packed pairs) into the first 16 of the S^T / dP^T columns this warp
+      // itself read (32 hf .. 32 hf + 15): never into columns the other warp of the lane
+      // quarter may still be reading
+      tmem_st16(tmem + lane_base + C::kColS + hf * 32, pk);
+      tmem_st16(tmem + lane_base + C::kColDP + hf * 32, dk2);
       // dS^T row (64 queries, 128 bytes) into shared memory, 128-byte swizzle (MN-major B):
       // this warp's four 16-byte chunks
 #pragma unroll
