@@ -30,8 +30,12 @@
 //     sequence and, under the causal flag, keys after a query's position; the
 //     per-query maximum over the 128 keys is reduced across the four warps through
 //     shared memory; lazy rescale of O^T (only when a query's maximum grows by more
-//     than 2^8); P^T is written to shared memory in the input type, and each thread
-//     keeps per-query partial sums of the rounded P, reduced once per item.
+//     than 2^8); P^T is written to shared memory in fp16, and each thread keeps
+//     per-query partial sums of the rounded P, reduced once per item.  For bf16 inputs
+//     each thread first converts its key's row of the V tile to fp16 in place, so the
+//     O^T product runs in fp16 as the tiled forward's does (bf16's 8-bit P would miss the
+//     output bound for short sequences); a V magnitude with no fp16 value records the
+//     range status.
 // Each item yields per-query partials (o unnormalised, m in base-2 units, l), merged
 // over the key splits by attn_mq_combine_kernel.
 #pragma once
@@ -230,7 +234,8 @@ __global__ void __launch_bounds__(MqCfg<D>::kThreads, 1)
   } else if (warp == C::kMmaWarp) {
     // ======================= tcgen05 MMA issuer (one elected lane issues) ===========
     constexpr uint32_t idesc_s = make_idesc_f16(128, kMqMaxQ, BF16, false, false);  // K Q^T
-    constexpr uint32_t idesc_o = make_idesc_f16(128, kMqMaxQ, BF16, false, true);   // V^T P^T
+    // V^T P^T always in fp16 (bf16 V tiles are converted in shared memory first)
+    constexpr uint32_t idesc_o = make_idesc_f16(128, kMqMaxQ, false, false, true);
     // d = 64: M = 128 reads the 64 head-dim elements twice (lanes 64..127 of O^T unused)
     constexpr uint32_t kLboV = (D == 128) ? C::kBoxBytes : 0;
     const uint32_t colS[2] = {0u, 16u};
@@ -295,6 +300,7 @@ __global__ void __launch_bounds__(MqCfg<D>::kThreads, 1)
     const uint32_t tO = tmem + lane_base + 32u;
     const float cs = p.scale_log2;
     const int Lq = p.Lq;
+    uint32_t vmag = 0;  // bf16: per-halfword max of |bits| over the V elements this thread converted
     int g = 0;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
       const MqItem it = mq_item(p, item);
@@ -370,6 +376,29 @@ __global__ void __launch_bounds__(MqCfg<D>::kThreads, 1)
           tmem_st16(tO, o);
           tmem_st_wait();
         }
+        if constexpr (BF16) {
+          // this key's row of the V tile to fp16, in place (the stage's copies have landed:
+          // its full barrier cannot move on before this tile's product has read it)
+          mbar_wait(BAR(C::kBarFull + gt % C::kStages), (gt / C::kStages) & 1, wctx);
+          __syncwarp();
+          uint8_t* vrow = smem + (gt % C::kStages) * C::kStageBytes + C::kTileBytes + t * 128;
+#pragma unroll
+          for (int bx = 0; bx < C::kBoxes; ++bx) {
+            uint4* w4 = reinterpret_cast<uint4*>(vrow + bx * C::kBoxBytes);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4 w = w4[c];
+              if (key < it.seq_len)  // rows past the sequence hold another page's keys
+                vmag = __vmaxu2(vmag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                               __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+              w.x = bf16x2_to_f16x2_sat(w.x);
+              w.y = bf16x2_to_f16x2_sat(w.y);
+              w.z = bf16x2_to_f16x2_sat(w.z);
+              w.w = bf16x2_to_f16x2_sat(w.w);
+              w4[c] = w;
+            }
+          }
+        }
         // P^T of this tile into P_(gt&1), once the product that read it two tiles ago is done
         if (gt >= 2) mbar_wait(BAR(C::kBarPFree + (gt & 1)), ((gt - 2) >> 1) & 1, wctx);
         __syncwarp();
@@ -378,16 +407,9 @@ __global__ void __launch_bounds__(MqCfg<D>::kThreads, 1)
 #pragma unroll
         for (int q = 0; q < kMqMaxQ; ++q) {
           const float pv = (x[q] == -INFINITY) ? 0.f : ex2_approx(x[q] - m_use[q]);
-          uint16_t hv;
-          if constexpr (BF16) {
-            const __nv_bfloat16 r = __float2bfloat16_rn(pv);
-            hv = *reinterpret_cast<const uint16_t*>(&r);
-            lp[q] += __bfloat162float(r);
-          } else {
-            const __half r = __float2half_rn(pv);
-            hv = *reinterpret_cast<const uint16_t*>(&r);
-            lp[q] += __half2float(r);
-          }
+          const __half r = __float2half_rn(pv);
+          const uint16_t hv = *reinterpret_cast<const uint16_t*>(&r);
+          lp[q] += __half2float(r);
           *reinterpret_cast<uint16_t*>(pb + q * 128 + ((chunk ^ (q & 7)) << 4)) = hv;
         }
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
@@ -432,6 +454,9 @@ __global__ void __launch_bounds__(MqCfg<D>::kThreads, 1)
       }
       named_bar_sync(1, 128);  // redl is read before the next item writes it
       g += ntile;
+    }
+    if constexpr (BF16) {
+      if (max(vmag & 0xFFFFu, vmag >> 16) >= kBf16NoF16) atomicCAS(p.status, 0, kStatusRange);
     }
   }
 

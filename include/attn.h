@@ -211,8 +211,11 @@ ATTN_API int attn_fwd_decode_paged(const void* q, const void* k_cache, const voi
  *   1 <= Lq <= 16; page_size, max_blocks, num_blocks, splits, seq_lens and
  *   table entries as attn_fwd_decode_paged; causal 0/1.
  *
- * The probabilities multiply V in the input type (fp16 or bf16) and O is
- * normalised by the sum of those rounded probabilities.  The workspace of
+ * The probabilities multiply V in fp16 (bf16 V tiles are converted to fp16 on
+ * chip, as attn_fwd does; a bf16 V element of the sequence with no fp16 value,
+ * magnitude 65536 or more, inf or NaN, makes the call record ATTN_ERR_RANGE in
+ * the status word) and O is normalised by the sum of those rounded
+ * probabilities.  The workspace of
  * B*H*splits*Lq*(d+2)*4 bytes is taken stream-ordered from the default pool.
  * Returns ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA;
  * asynchronous like attn_fwd.

@@ -72,3 +72,30 @@ def test_tokens_past_sixteen_are_rejected():
     q, kc, vc, bt, sl = (t.cuda() for t in make_paged_inputs(1, 2, 64, [100], 16, Lq=17, seed=3))
     with pytest.raises(AttnError):
         attn_fwd_paged(q, kc, vc, bt, sl)
+
+
+def test_paged_multi_token_bf16_range_status():
+    """bf16 V tiles are converted to fp16 on chip for the P V product: a V element of a
+    request's sequence with no fp16 value records ATTN_ERR_RANGE; the largest bf16 value
+    below fp16's limit (65280) does not, and neither does a huge value in a cache row that
+    no request reads."""
+    from attention_forward_tiled_b200 import ATTN_ERR_RANGE
+    H, d, page, seq_lens, Lq = 2, 128, 16, [40, 70], 4
+    q, kc, vc, bt, sl = make_paged_inputs(len(seq_lens), H, d, seq_lens, page, dtype="bf16", Lq=Lq, seed=77,
+                                          max_blocks=8)
+    used = int(bt[1, 2])            # a page of request 1 (keys 32..47, inside its 70 keys)
+    spare = kc.shape[0] - 1         # the spare pages at the end of the cache are never listed
+    assert spare not in set(bt[bt >= 0].tolist())
+    args = lambda v: (q.cuda(), kc.cuda(), v.cuda(), bt.cuda(), sl.cuda())  # noqa: E731
+    for bad in (1e5, float("inf")):
+        v = vc.clone()
+        v[used, 3, 1, 5] = bad
+        attn_fwd_paged(*args(v), causal=True)
+        torch.cuda.synchronize()
+        assert get_status() == ATTN_ERR_RANGE, bad
+    v = vc.clone()
+    v[used, 3, 1, 5] = 65280.0
+    v[spare, 0, 0, 0] = 1e5
+    attn_fwd_paged(*args(v), causal=True)
+    torch.cuda.synchronize()
+    assert get_status() == 0
